@@ -1,0 +1,57 @@
+"""Oracle for DeepSeek Sparse Attention (DSA): a plain, slow, float64 CPU implementation.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import it.  The product path
+(the CUDA library and its Python binding) never imports, calls or links anything here, and
+this package imports nothing from the product.
+
+Every function cites the passage of the source pages it follows.  The pages are five web
+pages about the DeepSeek-V3.2 technical report; citations name the page's title and section:
+
+* [MZ] "DeepSeek-V3.2 论文解读：稀疏注意力加疯狂的 RL，把开源带到 IMO 金牌"
+  (mizuki-eaf.pages.dev), section 二 "DeepSeek Sparse Attention（稀疏注意力）":
+  subsections "工作原理" (indexer + top-k), "挂在 MLA 上" (MQA mode, shared latent),
+  "等性能验证" (H800 cost curves, masked-MHA short-prefill mode), and the table
+  "附：DSA 关键参数".
+* [JD] "DeepSeek V3.2 ..." (jienda.com), section 2.1 "DeepSeek稀疏注意力（DSA）：长上下文处理的范式转移".
+* [36] report digest (36881.com.cn), section "DSA：把注意力從 O(L2) 降到 O(Lk)".
+* [DP] news article (digipub.cc), section 二 "基于DeepSeek-V3.1最終版打造，DSA讓模型計算更聰明".
+* [TW] techwalker.com article, section 一 "突破效率瓶颈的稀疏注意力机制".
+
+The indexer formula I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s]), the 576-d latent
+(512 + 64) with a 512-d value, FP8 e4m3 operands with per-token fp32 scales and the
+lower-index tie rule are the method's stated problem definition (the hot-path statement
+this library implements); the pages themselves give the structure in words only.
+
+Parity status per function (what pins it, in ``tests/test_oracle_*.py``):
+
+* ``e4m3_table`` / ``decode_e4m3``: pinned (all 256 codes against an independent library
+  decoder, plus hand-checked code points).
+* ``indexer_scores_query`` / ``indexer_scores``: pinned (exact rational brute force on tiny
+  inputs, single-head closed form against a library matmul, hand-worked golden example,
+  causal-mask and ReLU invariants).
+* ``topk_indices``: pinned (brute-force sort, invariants, argmax and all-equal special cases).
+* ``sparse_mla_token`` / ``sparse_mla``: pinned (k >= L equals dense causal attention from a
+  library routine; single-row, equal-rows and uniform-logit closed forms; permutation
+  invariance).
+* ``paged_gather`` / decode functions: pinned (paged layout equals the contiguous result).
+* Agreement with DeepSeek's trained model: parity unpinned (no weights, no printed values).
+"""
+
+from .dsa_oracle import (  # noqa: F401
+    E4M3_MAX,
+    e4m3_table,
+    decode_e4m3,
+    indexer_scores_query,
+    indexer_scores,
+    indexer_magnitude_query,
+    order_key_f32,
+    topk_indices,
+    topk_rows,
+    sparse_mla_token,
+    sparse_mla,
+    paged_gather,
+    decode_indexer_scores,
+    dsa_prefill_rows,
+    dsa_decode,
+)

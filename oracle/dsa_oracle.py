@@ -1,0 +1,234 @@
+"""Plain float64 definition of the DSA hot path: lightning indexer -> top-k -> sparse MLA (MQA).
+
+TEST INFRASTRUCTURE ONLY (see the package docstring for who may use it and for the page
+citations [MZ], [JD], [36], [DP], [TW]).
+
+Nothing here is blocked, fused or reordered beyond the definitions; numpy's float64 matmul
+is the only library primitive used as a step.  Readings taken where the pages are silent:
+
+* FP8 means OCP E4M3FN (bias 7, subnormals, max 448, S.1111.111 = NaN, no infinities).
+* Dequantisation is per token: q_I[t,j,:] = e4m3(q8[t,j,:]) * q_scale[t],
+  k_I[s,:] = e4m3(k8[s,:]) * k_scale[s].
+* "All preceding tokens" is the causal prefix s <= t (the query's own key included), so a
+  prefill row keeps min(k, t+1) entries; a decode query sits at position ctx-1 and sees all
+  ctx cached keys.
+* Scores are computed in float64 and rounded once to float32 (round to nearest even) before
+  selection; selection orders by score descending, ties to the lower index, -0.0 == +0.0.
+* Selected indices are emitted in ascending order, padded with -1.
+* Attention: logits = sm_scale * q[t,h,:576] . c[i,:576], softmax over the selected i, value
+  = c[i,:512] (the first 512 latent dims); lse is the natural-log sum of exp(logits).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+E4M3_MAX = 448.0
+
+
+# ---------------------------------------------------------------------------------------------
+# FP8 e4m3 ([MZ] "工作原理": the indexer "can run in FP8"; [JD] 2.1: "FP8低精度计算")
+# ---------------------------------------------------------------------------------------------
+def e4m3_table() -> np.ndarray:
+    """Value of every byte under OCP E4M3FN, written from the format definition.
+
+    Bit 7 is the sign, bits 6..3 the exponent (bias 7), bits 2..0 the mantissa.  Exponent 0
+    encodes subnormals m/8 * 2^-6; exponent 15 with mantissa 7 is NaN; there is no infinity.
+    """
+    table = np.empty(256, dtype=np.float64)
+    for code in range(256):
+        sign = -1.0 if code & 0x80 else 1.0
+        exponent = (code >> 3) & 0xF
+        mantissa = code & 0x7
+        if exponent == 0xF and mantissa == 0x7:
+            table[code] = np.nan
+        elif exponent == 0:
+            table[code] = sign * (mantissa / 8.0) * 2.0 ** (1 - 7)
+        else:
+            table[code] = sign * (1.0 + mantissa / 8.0) * 2.0 ** (exponent - 7)
+    return table
+
+
+_E4M3 = e4m3_table()
+
+
+def decode_e4m3(codes: np.ndarray) -> np.ndarray:
+    """float64 values of an array of e4m3 bytes."""
+    return _E4M3[np.asarray(codes, dtype=np.uint8)]
+
+
+# ---------------------------------------------------------------------------------------------
+# Lightning indexer ([MZ] "工作原理"; [36] "第一步：Lightning Indexer"; [DP] 二)
+# ---------------------------------------------------------------------------------------------
+def indexer_scores_query(q8: np.ndarray, q_scale: float, w: np.ndarray, k8: np.ndarray,
+                         k_scale: np.ndarray) -> np.ndarray:
+    """Index scores of one query token against a set of keys.
+
+    I[s] = sum_j w[j] * ReLU(q_I[j] . k_I[s]) with q_I = e4m3(q8) * q_scale and
+    k_I = e4m3(k8) * k_scale (per-token scales).  q8: [H_I, d_I] bytes, w: [H_I],
+    k8: [n, d_I] bytes, k_scale: [n].  Returns float64 [n].
+    """
+    q = decode_e4m3(q8) * float(q_scale)                       # [H_I, d_I]
+    k = decode_e4m3(k8) * np.asarray(k_scale, np.float64)[:, None]  # [n, d_I]
+    dots = q @ k.T                                              # [H_I, n]
+    return np.asarray(w, np.float64) @ np.maximum(dots, 0.0)    # sum over indexer heads j
+
+
+def indexer_magnitude_query(q8, q_scale, w, k8, k_scale) -> np.ndarray:
+    """A[s] = sum_j |w[j]| * ReLU(q_I[j] . k_I[s]): the size of the terms that make up I[s].
+
+    Used as the denominator of the relative score tolerance, since I itself can cancel when
+    the head weights have mixed signs.
+    """
+    return indexer_scores_query(q8, q_scale, np.abs(np.asarray(w, np.float64)), k8, k_scale)
+
+
+def indexer_scores(q8: np.ndarray, q_scale: np.ndarray, w: np.ndarray, k8: np.ndarray,
+                   k_scale: np.ndarray, rows=None) -> np.ndarray:
+    """Prefill index scores of one sequence, for the causal prefix of each query row.
+
+    q8: [L, H_I, d_I], q_scale: [L], w: [L, H_I], k8: [L, d_I], k_scale: [L].
+    Returns float64 [len(rows), L]: I[t, s] for s <= t and -inf for s > t.
+    """
+    L = k8.shape[0]
+    rows = list(range(L)) if rows is None else list(rows)
+    out = np.full((len(rows), L), -np.inf)
+    for r, t in enumerate(rows):
+        out[r, : t + 1] = indexer_scores_query(q8[t], q_scale[t], w[t], k8[: t + 1], k_scale[: t + 1])
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# Fine-grained token selection ([MZ] "工作原理": each query keeps the top-k entries, k = 2048;
+# [36] "第二步：Fine-grained Token Selection"; [DP] 二)
+# ---------------------------------------------------------------------------------------------
+def order_key_f32(scores_f32: np.ndarray) -> np.ndarray:
+    """Map float32 scores to uint32 keys whose unsigned order is the score order (-0 == +0)."""
+    s = np.asarray(scores_f32, dtype=np.float32).copy()
+    s[s == 0] = 0.0                                   # canonical +0
+    u = s.view(np.uint32).astype(np.uint64)
+    neg = (u & 0x80000000) != 0
+    key = np.where(neg, (~u) & 0xFFFFFFFF, u | 0x80000000)
+    return key.astype(np.uint32)
+
+
+def topk_indices(scores: np.ndarray, m: int) -> np.ndarray:
+    """Indices of the m largest entries of a score row (ties to the lower index), ascending.
+
+    scores holds only the valid entries of the row (the causal prefix).  NaN is rejected.
+    """
+    s = np.asarray(scores, dtype=np.float64)
+    if np.isnan(s).any():
+        raise ValueError("NaN score")
+    m = min(int(m), s.shape[0])
+    order = np.lexsort((np.arange(s.shape[0]), -s))   # primary: score desc; secondary: index asc
+    return np.sort(order[:m])
+
+
+def topk_rows(scores: np.ndarray, row_len: np.ndarray, k: int) -> np.ndarray:
+    """Row-wise top-k over the first row_len[r] entries of each row; int32 [rows, k], -1 padded."""
+    scores = np.asarray(scores)
+    out = np.full((scores.shape[0], k), -1, dtype=np.int32)
+    for r in range(scores.shape[0]):
+        sel = topk_indices(scores[r, : int(row_len[r])], k)
+        out[r, : sel.shape[0]] = sel
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# Sparse MLA in MQA mode ([MZ] "挂在 MLA 上": every latent vector is shared by all query heads
+# of a token; [JD] 2.1: MLA compresses K/V into a latent vector space; [MZ] "工作原理": attention
+# runs only over the selected top-k entries)
+# ---------------------------------------------------------------------------------------------
+def sparse_mla_token(q: np.ndarray, latent: np.ndarray, sel: np.ndarray, sm_scale: float,
+                     dv: int = 512):
+    """Attention of all heads of one query over its selected latent rows.
+
+    q: [H, D] (D = 576), latent: [n, D], sel: selected row indices (no padding).
+    Key = the full 576-d latent row, value = its first dv dims.
+    Returns (out [H, dv] float64, lse [H] float64, natural log).
+    """
+    c = np.asarray(latent, np.float64)[np.asarray(sel, np.int64)]   # [m, D]
+    logits = float(sm_scale) * (np.asarray(q, np.float64) @ c.T)     # [H, m]
+    mx = logits.max(axis=1, keepdims=True)
+    e = np.exp(logits - mx)
+    z = e.sum(axis=1, keepdims=True)
+    out = (e / z) @ c[:, :dv]
+    lse = mx[:, 0] + np.log(z[:, 0])
+    return out, lse
+
+
+def sparse_mla(q: np.ndarray, latent: np.ndarray, idx: np.ndarray, sm_scale: float, rows=None,
+               dv: int = 512):
+    """Prefill sparse MLA of one sequence for the given rows; idx [L, k] is -1 padded.
+
+    Returns (out [len(rows), H, dv], lse [len(rows), H]).
+    """
+    L = idx.shape[0]
+    rows = list(range(L)) if rows is None else list(rows)
+    H = q.shape[1]
+    out = np.zeros((len(rows), H, dv))
+    lse = np.zeros((len(rows), H))
+    for r, t in enumerate(rows):
+        sel = idx[t][idx[t] >= 0]
+        out[r], lse[r] = sparse_mla_token(q[t], latent, sel, sm_scale, dv)
+    return out, lse
+
+
+# ---------------------------------------------------------------------------------------------
+# Decode over a paged cache ([MZ] "等性能验证": decoding cost at 128K; paged layout is the
+# library's decode input contract)
+# ---------------------------------------------------------------------------------------------
+def paged_gather(cache: np.ndarray, block_table_row: np.ndarray, ctx: int) -> np.ndarray:
+    """Rows 0..ctx-1 of one sequence from a paged cache [num_blocks, block_size, ...]."""
+    block_size = cache.shape[1]
+    pos = np.arange(int(ctx))
+    return cache[np.asarray(block_table_row)[pos // block_size], pos % block_size]
+
+
+def decode_indexer_scores(q8, q_scale, w, kcache8, kscale_cache, block_table_row, ctx):
+    """Index scores of the decode query (position ctx-1) over all ctx cached keys; float64 [ctx]."""
+    k8 = paged_gather(kcache8, block_table_row, ctx)
+    ks = paged_gather(kscale_cache, block_table_row, ctx)
+    return indexer_scores_query(q8, q_scale, w, k8, ks)
+
+
+# ---------------------------------------------------------------------------------------------
+# Whole path
+# ---------------------------------------------------------------------------------------------
+def dsa_prefill_rows(seq: dict, k: int, sm_scale: float, rows, dv: int = 512):
+    """DSA prefill of one sequence for the given query rows.
+
+    seq holds numpy arrays: q8 [L,H_I,d_I], q_scale [L], w [L,H_I], k8 [L,d_I], k_scale [L],
+    q [L,H,D], latent [L,D].  Returns dict(scores32 per row, idx [rows,k], out, lse).
+    """
+    rows = list(rows)
+    scores = indexer_scores(seq["q8"], seq["q_scale"], seq["w"], seq["k8"], seq["k_scale"], rows)
+    scores32 = scores.astype(np.float32)
+    idx = np.full((len(rows), k), -1, dtype=np.int32)
+    out = np.zeros((len(rows), seq["q"].shape[1], dv))
+    lse = np.zeros((len(rows), seq["q"].shape[1]))
+    for r, t in enumerate(rows):
+        sel = topk_indices(scores32[r, : t + 1], k)
+        idx[r, : sel.shape[0]] = sel
+        out[r], lse[r] = sparse_mla_token(seq["q"][t], seq["latent"], sel, sm_scale, dv)
+    return {"scores32": scores32, "idx": idx, "out": out, "lse": lse}
+
+
+def dsa_decode(seq: dict, k: int, sm_scale: float, dv: int = 512):
+    """DSA decode step of one sequence: indexer over the paged FP8 keys, top-k, sparse MLA over
+    the paged latent cache.
+
+    seq holds numpy arrays: q8 [H_I,d_I], q_scale (scalar), w [H_I], kcache8 [nb,bs,d_I],
+    kscale_cache [nb,bs], latent_cache [nb,bs,D], block_table [max_blocks], ctx, q [H,D].
+    """
+    ctx = int(seq["ctx"])
+    scores = decode_indexer_scores(seq["q8"], seq["q_scale"], seq["w"], seq["kcache8"],
+                                   seq["kscale_cache"], seq["block_table"], ctx)
+    scores32 = scores.astype(np.float32)
+    sel = topk_indices(scores32, k)
+    latent = paged_gather(seq["latent_cache"], seq["block_table"], ctx)
+    out, lse = sparse_mla_token(seq["q"], latent, sel, sm_scale, dv)
+    idx = np.full(k, -1, dtype=np.int32)
+    idx[: sel.shape[0]] = sel
+    return {"scores32": scores32, "idx": idx, "out": out, "lse": lse}
