@@ -1,0 +1,162 @@
+/*
+ * dsa.h — C ABI of the B200 (sm_100a) DeepSeek Sparse Attention hot path.
+ *
+ * The method (DeepSeek-V3.2 technical report, as described on the source pages):
+ *   1. a lightning indexer scores every query token t against each token s of its causal
+ *      prefix, I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s]), with few heads, ReLU and FP8
+ *      operands ("DeepSeek-V3.2 论文解读", section 二 "DeepSeek Sparse Attention", subsection
+ *      "工作原理"; 36881.com.cn digest, section "DSA：把注意力從 O(L2) 降到 O(Lk)",
+ *      "第一步：Lightning Indexer");
+ *   2. fine-grained token selection keeps the top-k (k = 2048) index scores of each query
+ *      (same subsections; "第二步：Fine-grained Token Selection");
+ *   3. attention runs only over the selected entries, on MLA in MQA mode: one 576-d latent
+ *      row per token (512 "nope" + 64 "rope" dims) serves as the key of every query head, and
+ *      its first 512 dims are the value ("DeepSeek-V3.2 论文解读", subsection "挂在 MLA 上";
+ *      jienda.com section 2.1 on MLA's latent compression of K/V).
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller; the library never allocates,
+ *     frees or synchronises (dsa_device_error is the one call that synchronises).  All work
+ *     is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *   - Layouts are row-major and dense unless a leading dimension is given.  bf16 tensors are
+ *     passed as `const void*`.  FP8 operands are OCP e4m3 bytes with one fp32 scale per token
+ *     (dequantised value = e4m3(byte) * scale).
+ *   - Indices are sequence-local token positions.  A prefill query at local position t has
+ *     the causal prefix 0..t (min(k, t+1) entries are selected); a decode query sits at
+ *     position ctx-1 and sees all ctx cached tokens.
+ *   - Selected indices are written in ascending order and padded with -1.  Ties in the
+ *     index score go to the lower index; -0.0 equals +0.0.
+ *   - Host-side validation runs before any launch: NULL or misaligned pointers and
+ *     inconsistent sizes return DSA_ERR_INVALID_ARGUMENT, shapes outside the supported set
+ *     return DSA_ERR_UNSUPPORTED, a launch failure returns DSA_ERR_CUDA.  Errors found on the
+ *     device (a bounded wait that expired, NaN scores) are recorded in a per-process device
+ *     error word and reported by dsa_device_error().
+ *   - Supported shapes: indexer heads H_I in {4, 64} with d_I in {64, 128}; query heads
+ *     H = 128 (prefill and decode) or 16 (prefill only); latent dim 576 with value dim 512;
+ *     1 <= k <= 2048 with k a multiple of 64 for attention; paged block size 64.
+ */
+#ifndef DSA_B200_H_
+#define DSA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARGUMENT = 1,
+  DSA_ERR_UNSUPPORTED = 2,
+  DSA_ERR_WORKSPACE_TOO_SMALL = 3,
+  DSA_ERR_CUDA = 4,
+  DSA_ERR_TIMEOUT = 5,      /* a device-side bounded wait expired */
+  DSA_ERR_DEVICE_CHECK = 6  /* a device-side input check failed (e.g. NaN index score) */
+} dsa_status;
+
+typedef enum { DSA_KV_CONTIGUOUS = 0, DSA_KV_PAGED = 1 } dsa_kv_kind;
+typedef enum { DSA_MODE_PREFILL = 0, DSA_MODE_DECODE = 1 } dsa_mode;
+
+/*
+ * Describes one per-token operand: the FP8 indexer keys (data = e4m3 bytes, scale = fp32 per
+ * token) or the bf16 latent (scale = NULL).
+ *   contiguous: data [total_tokens, D]; scale [total_tokens]; cu_seqlens [B+1] (device) gives
+ *               each sequence's token range; in prefill the queries are the same tokens.
+ *   paged:      data [num_blocks, block_size, D]; scale [num_blocks, block_size];
+ *               block_table [B, max_blocks_per_seq] (device) maps a sequence's logical block
+ *               p/block_size to a physical block; context_lens [B] (device) = ctx per sequence.
+ * total_tokens and max_seqlen are host copies (max_seqlen: longest sequence or context).
+ */
+typedef struct {
+  int32_t kind;
+  const void* data;
+  const float* scale;
+  const int32_t* cu_seqlens;
+  const int32_t* block_table;
+  const int32_t* context_lens;
+  int64_t total_tokens;
+  int32_t max_seqlen;
+  int32_t num_blocks;
+  int32_t block_size;
+  int32_t max_blocks_per_seq;
+} dsa_kv_desc;
+
+/*
+ * Lightning indexer scores (method step 1), written to HBM for a range of query rows.
+ *   prefill (keys contiguous): rows are packed query tokens [row_begin, row_end) of
+ *     q_fp8 [T, H_I, d_I], q_scale [T], w [T, H_I]; row r (local position t in a sequence
+ *     of length n) gets scores[(r-row_begin)*ld_scores + s] = I[t,s] for s <= t and -INFINITY
+ *     for t < s < n.  ld_scores >= keys->max_seqlen and a multiple of 4.
+ *   decode (keys paged): rows are sequences b in [row_begin, row_end) with q_fp8 [B, H_I, d_I],
+ *     q_scale [B], w [B, H_I]; scores[(b-row_begin)*ld_scores + s] = I for s < ctx[b].
+ * Scores are fp32, accumulated in fp32 on the tensor cores (e4m3 x e4m3).
+ */
+dsa_status dsa_indexer_scores(const uint8_t* q_fp8, const float* q_scale, const float* w,
+                              const dsa_kv_desc* keys, int32_t B, int32_t H_I, int32_t d_I,
+                              int64_t row_begin, int64_t row_end, float* scores, int64_t ld_scores,
+                              void* stream);
+
+/*
+ * Top-k selection (method step 2) over score rows: for row r the first row_len[r] entries
+ * of scores[r*ld_scores ...] are candidates; idx[r*k ...] receives the indices of the
+ * min(k, row_len[r]) largest (ties -> lower index), ascending, -1 padded.  row_len is a device
+ * array.  scores must be 16-byte aligned and ld_scores a multiple of 4.  NaN scores set
+ * DSA_ERR_DEVICE_CHECK in the device error word.
+ */
+dsa_status dsa_topk(const float* scores, int64_t ld_scores, int64_t rows, const int32_t* row_len,
+                    int32_t k, int32_t* idx, void* stream);
+
+/*
+ * Sparse MLA prefill (method step 3): for every packed query token t and head h,
+ *   out[t,h,:] = sum_i softmax_i(sm_scale * q[t,h,:] . c[idx[t,i],:]) * c[idx[t,i], 0:512]
+ * over the valid (>= 0) entries of idx [T, k]; c is the contiguous latent of t's sequence.
+ * q [T, H, 576] bf16, out [T, H, 512] bf16, lse [T, H] fp32 natural log (may be NULL).
+ * Every row must hold at least one valid index.
+ */
+dsa_status dsa_sparse_mla_prefill(const void* q, const dsa_kv_desc* latent, const int32_t* idx,
+                                  int32_t B, int32_t H, int32_t k, float sm_scale, void* out,
+                                  float* lse, void* stream);
+
+/*
+ * Sparse MLA decode: one query per sequence, q [B, H, 576]; idx [B, k] holds logical positions
+ * (< ctx[b]) resolved through the paged latent cache (latent->kind == DSA_KV_PAGED).  The work
+ * is split over the k selected rows; partial results go to `workspace`
+ * (dsa_workspace_size(DSA_MODE_DECODE, ...) bytes) and are merged by log-sum-exp.
+ */
+dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const int32_t* idx,
+                                 int32_t B, int32_t H, int32_t k, float sm_scale, void* out,
+                                 float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Whole DSA forward.
+ *   DSA_MODE_PREFILL: indexer and top-k run fused (no score matrix is written to HBM), then
+ *     sparse MLA.  keys/latent contiguous with the same cu_seqlens; q_fp8 [T, H_I, d_I], etc.
+ *   DSA_MODE_DECODE: paged indexer scores for each sequence's context, top-k, then split
+ *     sparse MLA with a log-sum-exp merge.
+ * idx_out [rows, k] receives the selection when not NULL (otherwise it lives in workspace).
+ */
+dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale, const float* w,
+                       const dsa_kv_desc* keys, const void* q, const dsa_kv_desc* latent, int32_t B,
+                       int32_t H_I, int32_t d_I, int32_t H, int32_t k, float sm_scale, void* out,
+                       float* lse, int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of workspace dsa_forward / dsa_sparse_mla_decode need (0 when none). */
+size_t dsa_workspace_size(int32_t mode, int32_t B, int64_t total_tokens, int32_t max_ctx, int32_t H,
+                          int32_t H_I, int32_t k);
+
+/* Static description of a status code. */
+const char* dsa_status_string(int32_t status);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the current device.
+ * *code receives DSA_OK or the first DSA_ERR_TIMEOUT / DSA_ERR_DEVICE_CHECK recorded since the
+ * last call.  Returns DSA_ERR_CUDA if synchronisation failed.
+ */
+dsa_status dsa_device_error(int32_t* code, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_B200_H_ */

@@ -1,0 +1,182 @@
+"""Python binding of libdsa (the B200 DeepSeek Sparse Attention library).
+
+Argument marshalling only: every function passes device pointers (``tensor.data_ptr()``),
+sizes and the current CUDA stream to the C ABI declared in ``include/dsa.h`` and raises
+``DSAError`` on a non-zero status.  All computation happens in the library's CUDA kernels;
+there is no fallback.  Importing fails if the library has not been built
+(``python sparse_attention_09_b200/build.py``).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libdsa.so is not built ({_LIB_PATH}); run: python sparse_attention_09_b200/build.py")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+DSA_OK = 0
+DSA_ERR_INVALID_ARGUMENT = 1
+DSA_ERR_UNSUPPORTED = 2
+DSA_ERR_WORKSPACE_TOO_SMALL = 3
+DSA_ERR_CUDA = 4
+DSA_ERR_TIMEOUT = 5
+DSA_ERR_DEVICE_CHECK = 6
+DSA_KV_CONTIGUOUS = 0
+DSA_KV_PAGED = 1
+DSA_MODE_PREFILL = 0
+DSA_MODE_DECODE = 1
+
+EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_prefill", "dsa_sparse_mla_decode",
+            "dsa_forward", "dsa_workspace_size", "dsa_status_string", "dsa_device_error")
+
+
+class KVDesc(ctypes.Structure):
+    _fields_ = [
+        ("kind", ctypes.c_int32),
+        ("data", ctypes.c_void_p),
+        ("scale", ctypes.c_void_p),
+        ("cu_seqlens", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p),
+        ("context_lens", ctypes.c_void_p),
+        ("total_tokens", ctypes.c_int64),
+        ("max_seqlen", ctypes.c_int32),
+        ("num_blocks", ctypes.c_int32),
+        ("block_size", ctypes.c_int32),
+        ("max_blocks_per_seq", ctypes.c_int32),
+    ]
+
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_F32 = ctypes.c_float
+_SZ = ctypes.c_size_t
+_DESC = ctypes.POINTER(KVDesc)
+
+_lib.dsa_status_string.argtypes = [_I32]
+_lib.dsa_status_string.restype = ctypes.c_char_p
+_lib.dsa_device_error.argtypes = [ctypes.POINTER(_I32), _P]
+_lib.dsa_device_error.restype = _I32
+_lib.dsa_topk.argtypes = [_P, _I64, _I64, _P, _I32, _P, _P]
+_lib.dsa_topk.restype = _I32
+_lib.dsa_indexer_scores.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I64, _I64, _P, _I64, _P]
+_lib.dsa_indexer_scores.restype = _I32
+_lib.dsa_sparse_mla_prefill.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P]
+_lib.dsa_sparse_mla_prefill.restype = _I32
+_lib.dsa_sparse_mla_decode.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P, _SZ, _P]
+_lib.dsa_sparse_mla_decode.restype = _I32
+_lib.dsa_forward.argtypes = [_I32, _P, _P, _P, _DESC, _P, _DESC, _I32, _I32, _I32, _I32, _I32, _F32, _P, _P, _P,
+                             _P, _SZ, _P]
+_lib.dsa_forward.restype = _I32
+_lib.dsa_workspace_size.argtypes = [_I32, _I32, _I64, _I32, _I32, _I32, _I32]
+_lib.dsa_workspace_size.restype = _SZ
+
+
+class DSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {dsa_status_string(status)} (status {status})")
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def dsa_status_string(status: int) -> str:
+    return _lib.dsa_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status, where):
+    if status != DSA_OK:
+        raise DSAError(status, where)
+
+
+class Desc:
+    """A dsa_kv_desc plus references to the tensors it points at."""
+
+    def __init__(self, struct: KVDesc, refs):
+        self.struct = struct
+        self._refs = refs
+
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+
+def contiguous_desc(data, cu_seqlens, max_seqlen, scale=None) -> Desc:
+    """Contiguous per-token operand: data [T, D] (e4m3 bytes with scale [T], or bf16 latent)."""
+    s = KVDesc(kind=DSA_KV_CONTIGUOUS, data=data.data_ptr(), scale=None if scale is None else scale.data_ptr(),
+               cu_seqlens=cu_seqlens.data_ptr(), block_table=None, context_lens=None,
+               total_tokens=int(data.shape[0]), max_seqlen=int(max_seqlen), num_blocks=0, block_size=0,
+               max_blocks_per_seq=0)
+    return Desc(s, (data, scale, cu_seqlens))
+
+
+def paged_desc(data, block_table, context_lens, max_ctx, scale=None) -> Desc:
+    """Paged operand: data [num_blocks, block_size, D]; block_table [B, max_blocks]; context_lens [B]."""
+    s = KVDesc(kind=DSA_KV_PAGED, data=data.data_ptr(), scale=None if scale is None else scale.data_ptr(),
+               cu_seqlens=None, block_table=block_table.data_ptr(), context_lens=context_lens.data_ptr(),
+               total_tokens=0, max_seqlen=int(max_ctx), num_blocks=int(data.shape[0]),
+               block_size=int(data.shape[1]), max_blocks_per_seq=int(block_table.shape[1]))
+    return Desc(s, (data, scale, block_table, context_lens))
+
+
+def dsa_topk(scores, row_len, k, idx, stream=None):
+    """idx[r, :] = top-k indices (ascending, -1 padded) of scores[r, :row_len[r]]."""
+    _check(_lib.dsa_topk(_ptr(scores), scores.stride(0), scores.shape[0], _ptr(row_len), int(k), _ptr(idx),
+                         _stream(stream)), "dsa_topk")
+    return idx
+
+
+def dsa_indexer_scores(q_fp8, q_scale, w, keys: Desc, B, H_I, d_I, row_begin, row_end, scores, stream=None):
+    _check(_lib.dsa_indexer_scores(_ptr(q_fp8), _ptr(q_scale), _ptr(w), keys.ref(), int(B), int(H_I), int(d_I),
+                                   int(row_begin), int(row_end), _ptr(scores), scores.stride(0), _stream(stream)),
+           "dsa_indexer_scores")
+    return scores
+
+
+def dsa_sparse_mla_prefill(q, latent: Desc, idx, B, H, k, sm_scale, out, lse=None, stream=None):
+    _check(_lib.dsa_sparse_mla_prefill(_ptr(q), latent.ref(), _ptr(idx), int(B), int(H), int(k), float(sm_scale),
+                                       _ptr(out), _ptr(lse), _stream(stream)), "dsa_sparse_mla_prefill")
+    return out
+
+
+def dsa_sparse_mla_decode(q, latent: Desc, idx, B, H, k, sm_scale, out, lse=None, workspace=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.dsa_sparse_mla_decode(_ptr(q), latent.ref(), _ptr(idx), int(B), int(H), int(k), float(sm_scale),
+                                      _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)),
+           "dsa_sparse_mla_decode")
+    return out
+
+
+def dsa_forward(mode, q_fp8, q_scale, w, keys: Desc, q, latent: Desc, B, H_I, d_I, H, k, sm_scale, out, lse=None,
+                idx_out=None, workspace=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.dsa_forward(int(mode), _ptr(q_fp8), _ptr(q_scale), _ptr(w), keys.ref(), _ptr(q), latent.ref(),
+                            int(B), int(H_I), int(d_I), int(H), int(k), float(sm_scale), _ptr(out), _ptr(lse),
+                            _ptr(idx_out), _ptr(workspace), ws_bytes, _stream(stream)), "dsa_forward")
+    return out
+
+
+def dsa_workspace_size(mode, B, total_tokens, max_ctx, H, H_I, k) -> int:
+    return int(_lib.dsa_workspace_size(int(mode), int(B), int(total_tokens), int(max_ctx), int(H), int(H_I), int(k)))
+
+
+def dsa_device_error(stream=None) -> int:
+    code = _I32(0)
+    _check(_lib.dsa_device_error(ctypes.byref(code), _stream(stream)), "dsa_device_error")
+    return int(code.value)

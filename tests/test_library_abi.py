@@ -1,0 +1,48 @@
+"""The C-ABI library loads, exports every entry point include/dsa.h declares, and validates
+arguments on the host (no GPU work is launched by these calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    import sparse_attention_09_b200 as dsa
+    lib = ctypes.CDLL(dsa.lib_path())
+    names = _declared()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(dsa.EXPORTED) <= set(names)
+
+
+def test_status_strings():
+    import sparse_attention_09_b200 as dsa
+    assert dsa.dsa_status_string(0) == "ok"
+    assert "timed out" in dsa.dsa_status_string(dsa.DSA_ERR_TIMEOUT)
+    assert dsa.dsa_status_string(999) == "unknown status"
+
+
+def test_host_validation_rejects_bad_arguments_before_launch():
+    import sparse_attention_09_b200 as dsa
+    lib = dsa._lib
+    null = ctypes.c_void_p(0)
+    # NULL scores / bad k / misaligned leading dimension
+    assert lib.dsa_topk(null, 8, 4, null, 4, null, null) == dsa.DSA_ERR_INVALID_ARGUMENT
+    assert lib.dsa_topk(ctypes.c_void_p(256), 8, 4, ctypes.c_void_p(256), 0, ctypes.c_void_p(256), null) == \
+        dsa.DSA_ERR_INVALID_ARGUMENT
+    assert lib.dsa_topk(ctypes.c_void_p(256), 6, 4, ctypes.c_void_p(256), 4, ctypes.c_void_p(256), null) == \
+        dsa.DSA_ERR_INVALID_ARGUMENT
+    assert lib.dsa_topk(ctypes.c_void_p(260), 8, 4, ctypes.c_void_p(256), 4, ctypes.c_void_p(256), null) == \
+        dsa.DSA_ERR_INVALID_ARGUMENT
+    # zero rows is a no-op
+    assert lib.dsa_topk(null, 8, 0, null, 4, null, null) == dsa.DSA_OK
