@@ -98,6 +98,17 @@ dsa_status dsa_indexer_scores(const uint8_t* q_fp8, const float* q_scale, const 
                               void* stream);
 
 /*
+ * Fused lightning indexer + top-k for prefill (method steps 1 and 2 together): for every
+ * packed query token of q_fp8 [T, H_I, d_I] (keys contiguous, queries == keys per sequence),
+ * idx_out[t*k ...] receives the min(k, t+1) highest-scoring causal-prefix positions,
+ * ascending, -1 padded.  Scores stay on chip: each CTA keeps a per-token candidate set in
+ * shared memory with a rising threshold.  The selection equals dsa_topk applied to the
+ * scores dsa_indexer_scores writes (same fp32 arithmetic).  keys->max_seqlen <= 262144.
+ */
+dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, const float* w, const dsa_kv_desc* keys,
+                            int32_t B, int32_t H_I, int32_t d_I, int32_t k, int32_t* idx_out, void* stream);
+
+/*
  * Top-k selection (method step 2) over score rows: for row r the first row_len[r] entries
  * of scores[r*ld_scores ...] are candidates; idx[r*k ...] receives the indices of the
  * min(k, row_len[r]) largest (ties -> lower index), ascending, -1 padded.  row_len is a device

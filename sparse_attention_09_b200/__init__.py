@@ -31,7 +31,7 @@ DSA_KV_PAGED = 1
 DSA_MODE_PREFILL = 0
 DSA_MODE_DECODE = 1
 
-EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_prefill", "dsa_sparse_mla_decode",
+EXPORTED = ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_mla_prefill", "dsa_sparse_mla_decode",
             "dsa_forward", "dsa_workspace_size", "dsa_status_string", "dsa_device_error")
 
 

@@ -11,6 +11,7 @@
 
 #include "../../include/dsa.h"
 #include "common.cuh"
+#include "indexer.cuh"
 #include "topk.cuh"
 
 namespace dsa {
@@ -22,6 +23,114 @@ inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 inline dsa_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ---- TMA descriptors (encoded on the host through the driver entry point) -------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major [rows, cols] tensor; box = [box_rows, box_cols].
+bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t rows,
+                 uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---- lightning indexer -------------------------------------------------------------------
+constexpr int kIdxStages = 4;
+constexpr int kIdxTok = 4;            // prefill query tokens per CTA
+constexpr int kDecodeTilesPerCta = 16;  // decode: 2048 keys per CTA
+
+template <int D_I, int H_I, int TOK, int MODE, bool PAGED>
+dsa_status launch_indexer_t(const CUtensorMap& qm, const CUtensorMap& km, const IndexerParams& p, dim3 grid,
+                            cudaStream_t s) {
+  auto kern = indexer_kernel<D_I, H_I, TOK, MODE, PAGED, kIdxStages>;
+  const int smem = indexer_smem_bytes<D_I, H_I, TOK, MODE, kIdxStages>(p.cap) + 1024;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  kern<<<grid, 192, smem, s>>>(qm, km, p);
+  return launch_status();
+}
+
+template <int MODE, bool PAGED>
+dsa_status launch_indexer(int d_I, int H_I, const CUtensorMap& qm, const CUtensorMap& km, const IndexerParams& p,
+                          dim3 grid, cudaStream_t s) {
+  constexpr int TOK = PAGED ? 1 : kIdxTok;
+  if constexpr (PAGED) {
+    if (H_I != 64) return DSA_ERR_UNSUPPORTED;
+    if (d_I == 128) return launch_indexer_t<128, 64, TOK, MODE, PAGED>(qm, km, p, grid, s);
+    if (d_I == 64) return launch_indexer_t<64, 64, TOK, MODE, PAGED>(qm, km, p, grid, s);
+    return DSA_ERR_UNSUPPORTED;
+  } else {
+    if (d_I == 128 && H_I == 64) return launch_indexer_t<128, 64, TOK, MODE, PAGED>(qm, km, p, grid, s);
+  if (d_I == 64 && H_I == 64) return launch_indexer_t<64, 64, TOK, MODE, PAGED>(qm, km, p, grid, s);
+  if (d_I == 128 && H_I == 4) return launch_indexer_t<128, 4, TOK, MODE, PAGED>(qm, km, p, grid, s);
+  if (d_I == 64 && H_I == 4) return launch_indexer_t<64, 4, TOK, MODE, PAGED>(qm, km, p, grid, s);
+  return DSA_ERR_UNSUPPORTED;
+  }
+}
+
+bool indexer_shape_ok(int H_I, int d_I) { return (H_I == 4 || H_I == 64) && (d_I == 64 || d_I == 128); }
+
+// Validates the common indexer arguments and builds the Q / K tensor maps.
+dsa_status indexer_common(const uint8_t* q_fp8, const float* q_scale, const float* w, const dsa_kv_desc* keys,
+                          int32_t B, int32_t H_I, int32_t d_I, CUtensorMap* qm, CUtensorMap* km,
+                          IndexerParams* p) {
+  if (q_fp8 == nullptr || q_scale == nullptr || w == nullptr || keys == nullptr || keys->data == nullptr ||
+      keys->scale == nullptr || B <= 0)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(q_fp8, 16) || !aligned(keys->data, 16)) return DSA_ERR_INVALID_ARGUMENT;
+  if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED;
+  const CUtensorMapSwizzle sw = d_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  std::memset(p, 0, sizeof(*p));
+  p->q_scale = q_scale;
+  p->w = w;
+  p->k_scale = keys->scale;
+  if (keys->kind == DSA_KV_CONTIGUOUS) {
+    if (keys->cu_seqlens == nullptr || keys->total_tokens <= 0 || keys->max_seqlen <= 0) return DSA_ERR_INVALID_ARGUMENT;
+    if (keys->total_tokens * H_I > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+    const uint64_t T = static_cast<uint64_t>(keys->total_tokens);
+    if (!make_map_2d(qm, q_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, d_I, T * H_I, d_I, d_I, kIdxTok * H_I, sw) ||
+        !make_map_2d(km, keys->data, CU_TENSOR_MAP_DATA_TYPE_UINT8, d_I, T, d_I, d_I, 128, sw))
+      return DSA_ERR_INVALID_ARGUMENT;
+    p->cu_seqlens = keys->cu_seqlens;
+  } else if (keys->kind == DSA_KV_PAGED) {
+    if (keys->block_table == nullptr || keys->context_lens == nullptr || keys->num_blocks <= 0 ||
+        keys->max_blocks_per_seq <= 0 || keys->max_seqlen <= 0)
+      return DSA_ERR_INVALID_ARGUMENT;
+    if (keys->block_size != 64 || H_I != 64) return DSA_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(keys->max_seqlen) > static_cast<int64_t>(keys->max_blocks_per_seq) * 64)
+      return DSA_ERR_INVALID_ARGUMENT;
+    if (static_cast<int64_t>(keys->num_blocks) * 64 > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+    const uint64_t rows = static_cast<uint64_t>(keys->num_blocks) * 64;
+    if (!make_map_2d(qm, q_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, d_I, static_cast<uint64_t>(B) * H_I, d_I, d_I, H_I,
+                     sw) ||
+        !make_map_2d(km, keys->data, CU_TENSOR_MAP_DATA_TYPE_UINT8, d_I, rows, d_I, d_I, 64, sw))
+      return DSA_ERR_INVALID_ARGUMENT;
+    p->block_table = keys->block_table;
+    p->context_lens = keys->context_lens;
+    p->max_blocks_per_seq = keys->max_blocks_per_seq;
+    p->tiles_per_cta = kDecodeTilesPerCta;
+  } else {
+    return DSA_ERR_INVALID_ARGUMENT;
+  }
+  return DSA_OK;
 }
 
 }  // namespace
@@ -71,9 +180,49 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, int64_t rows, const 
   return launch_status();
 }
 
-dsa_status dsa_indexer_scores(const uint8_t*, const float*, const float*, const dsa_kv_desc*, int32_t, int32_t,
-                              int32_t, int64_t, int64_t, float*, int64_t, void*) {
-  return DSA_ERR_UNSUPPORTED;
+dsa_status dsa_indexer_scores(const uint8_t* q_fp8, const float* q_scale, const float* w, const dsa_kv_desc* keys,
+                              int32_t B, int32_t H_I, int32_t d_I, int64_t row_begin, int64_t row_end,
+                              float* scores, int64_t ld_scores, void* stream) {
+  if (scores == nullptr || row_begin < 0 || row_end < row_begin) return DSA_ERR_INVALID_ARGUMENT;
+  if (keys == nullptr) return DSA_ERR_INVALID_ARGUMENT;
+  if (row_end == row_begin) return DSA_OK;
+  CUtensorMap qm, km;
+  IndexerParams p;
+  dsa_status st = indexer_common(q_fp8, q_scale, w, keys, B, H_I, d_I, &qm, &km, &p);
+  if (st != DSA_OK) return st;
+  if (ld_scores < keys->max_seqlen) return DSA_ERR_INVALID_ARGUMENT;
+  p.scores = scores;
+  p.ld = ld_scores;
+  p.row_begin = row_begin;
+  p.row_end = row_end;
+  if (keys->kind == DSA_KV_CONTIGUOUS) {
+    if (row_end > keys->total_tokens) return DSA_ERR_INVALID_ARGUMENT;
+    dim3 grid((keys->max_seqlen + kIdxTok - 1) / kIdxTok, B);
+    return launch_indexer<kIdxScores, false>(d_I, H_I, qm, km, p, grid, as_stream(stream));
+  }
+  if (row_end > B) return DSA_ERR_INVALID_ARGUMENT;
+  dim3 grid((keys->max_seqlen + 128 * kDecodeTilesPerCta - 1) / (128 * kDecodeTilesPerCta), B);
+  return launch_indexer<kIdxScores, true>(d_I, H_I, qm, km, p, grid, as_stream(stream));
+}
+
+dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, const float* w, const dsa_kv_desc* keys,
+                            int32_t B, int32_t H_I, int32_t d_I, int32_t k, int32_t* idx_out, void* stream) {
+  if (idx_out == nullptr || keys == nullptr || k <= 0) return DSA_ERR_INVALID_ARGUMENT;
+  if (keys->kind != DSA_KV_CONTIGUOUS) return DSA_ERR_UNSUPPORTED;
+  if (k > 2048) return DSA_ERR_UNSUPPORTED;
+  CUtensorMap qm, km;
+  IndexerParams p;
+  dsa_status st = indexer_common(q_fp8, q_scale, w, keys, B, H_I, d_I, &qm, &km, &p);
+  if (st != DSA_OK) return st;
+  // the final ascending emission uses a bitmap of the causal prefix inside the key ring
+  const int64_t bitmap_bytes = (static_cast<int64_t>(keys->max_seqlen) + 31) / 32 * 4;
+  if (bitmap_bytes > static_cast<int64_t>(kIdxStages) * 128 * d_I || keys->max_seqlen > (1 << 24))
+    return DSA_ERR_UNSUPPORTED;
+  p.idx_out = idx_out;
+  p.k = k;
+  p.cap = k + 1024;
+  dim3 grid((keys->max_seqlen + kIdxTok - 1) / kIdxTok, B);
+  return launch_indexer<kIdxTopk, false>(d_I, H_I, qm, km, p, grid, as_stream(stream));
 }
 
 dsa_status dsa_sparse_mla_prefill(const void*, const dsa_kv_desc*, const int32_t*, int32_t, int32_t, int32_t, float,
