@@ -103,7 +103,7 @@ dsa_status dsa_indexer_scores(const uint8_t* q_fp8, const float* q_scale, const 
  * idx_out[t*k ...] receives the min(k, t+1) highest-scoring causal-prefix positions,
  * ascending, -1 padded.  Scores stay on chip: each CTA keeps a per-token candidate set in
  * shared memory with a rising threshold.  The selection equals dsa_topk applied to the
- * scores dsa_indexer_scores writes (same fp32 arithmetic).  keys->max_seqlen <= 262144.
+ * scores dsa_indexer_scores writes (same fp32 arithmetic).  keys->max_seqlen <= 196608 (d_I = 128) or 98304 (d_I = 64).
  */
 dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, const float* w, const dsa_kv_desc* keys,
                             int32_t B, int32_t H_I, int32_t d_I, int32_t k, int32_t* idx_out, void* stream);

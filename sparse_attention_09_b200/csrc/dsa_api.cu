@@ -53,18 +53,21 @@ bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint6
 }
 
 // ---- lightning indexer -------------------------------------------------------------------
-constexpr int kIdxStages = 4;
+constexpr int kIdxStages = 4;      // key-tile ring depth, scores mode
+constexpr int kIdxStagesTopk = 3;  // fused top-k mode (the candidate sets need the SMEM)
+constexpr int kIdxCapMax = 4096;   // candidate capacity per token, fused top-k mode
 constexpr int kIdxTok = 4;            // prefill query tokens per CTA
 constexpr int kDecodeTilesPerCta = 16;  // decode: 2048 keys per CTA
 
 template <int D_I, int H_I, int TOK, int MODE, bool PAGED>
 dsa_status launch_indexer_t(const CUtensorMap& qm, const CUtensorMap& km, const IndexerParams& p, dim3 grid,
                             cudaStream_t s) {
-  auto kern = indexer_kernel<D_I, H_I, TOK, MODE, PAGED, kIdxStages>;
-  const int smem = indexer_smem_bytes<D_I, H_I, TOK, MODE, kIdxStages>(p.cap) + 1024;
+  constexpr int STAGES = MODE == kIdxTopk ? kIdxStagesTopk : kIdxStages;
+  auto kern = indexer_kernel<D_I, H_I, TOK, MODE, PAGED, STAGES>;
+  const int smem = indexer_smem_bytes<D_I, H_I, TOK, MODE, STAGES>(p.cap) + 1024;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return DSA_ERR_CUDA;
-  kern<<<grid, 192, smem, s>>>(qm, km, p);
+  kern<<<grid, IdxGroups<TOK>::kThreads, smem, s>>>(qm, km, p);
   return launch_status();
 }
 
@@ -216,11 +219,13 @@ dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, const fl
   if (st != DSA_OK) return st;
   // the final ascending emission uses a bitmap of the causal prefix inside the key ring
   const int64_t bitmap_bytes = (static_cast<int64_t>(keys->max_seqlen) + 31) / 32 * 4;
-  if (bitmap_bytes > static_cast<int64_t>(kIdxStages) * 128 * d_I || keys->max_seqlen > (1 << 24))
+  // (each of the two epilogue groups of a CTA has half of the key ring for its bitmap)
+  if (bitmap_bytes > static_cast<int64_t>(kIdxStagesTopk) * 128 * d_I / 2 || keys->max_seqlen > (1 << 24))
     return DSA_ERR_UNSUPPORTED;
   p.idx_out = idx_out;
   p.k = k;
-  p.cap = k + 1024;
+  p.cap = k + 1024 < 2 * k ? 2 * k : k + 1024;
+  if (p.cap > kIdxCapMax) p.cap = kIdxCapMax;
   dim3 grid((keys->max_seqlen + kIdxTok - 1) / kIdxTok, B);
   return launch_indexer<kIdxTopk, false>(d_I, H_I, qm, km, p, grid, as_stream(stream));
 }

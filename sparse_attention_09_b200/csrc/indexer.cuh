@@ -10,8 +10,10 @@
 // over heads in registers: ReLU, the per-head weight (w * q_scale), the head sum, k_scale and
 // the causal mask all happen in the epilogue, straight out of TMEM.
 //
-// Warp roles (192 threads): warps 0-3 epilogue (thread e owns TMEM lane e = key e of the
-// tile), warp 4 lane 0 TMA producer, warp 5 lane 0 MMA issuer (warp 5 also owns TMEM).
+// Warp roles: EG groups of 4 epilogue warps (warp q of a group owns TMEM lanes 32q..32q+31,
+// i.e. keys 32q.. of the tile; group g owns tokens g*TOK/EG ..), then one TMA producer warp
+// and one MMA-issuer warp (which also owns TMEM).  Prefill uses EG = 2 (8 epilogue warps,
+// two tokens each), decode EG = 1.
 // Key tiles flow through a STAGES-deep SMEM ring; the accumulator is double-buffered in TMEM
 // so the epilogue of tile i overlaps the MMA of tile i+1.
 //
@@ -26,6 +28,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "select.cuh"
 #include "sm100.cuh"
 
 namespace dsa {
@@ -51,34 +54,6 @@ struct IndexerParams {
 
 namespace idx_detail {
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-// Barrier over the 128 epilogue threads that also ORs a predicate across them, so that a
-// decision to leave a loop is the same in every thread (a named barrier cannot time out).
-__device__ __forceinline__ bool epi_any(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.or.pred p, 1, 128, q;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v))
-      : "memory");
-  return r != 0;
-}
-
-// Exclusive scan over the 128 epilogue threads (4 warps); `scratch` holds 4 ints.
-__device__ __forceinline__ int epi_scan(int v, int* scratch, int& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int inc = warp_inclusive_scan(v);
-  if (lane == 31) scratch[warp] = inc;
-  epi_sync();
-  const int w0 = scratch[0], w1 = scratch[1], w2 = scratch[2], w3 = scratch[3];
-  total = w0 + w1 + w2 + w3;
-  const int wprefix = (warp > 0 ? w0 : 0) + (warp > 1 ? w1 : 0) + (warp > 2 ? w2 : 0);
-  epi_sync();
-  return wprefix + inc - v;
-}
-
 // 16-byte shared-memory load that the compiler may not hoist out of the tile loop (the
 // per-head weights of all TOK tokens would not fit in registers).
 __device__ __forceinline__ float4 lds128(const float* p) {
@@ -87,125 +62,6 @@ __device__ __forceinline__ float4 lds128(const float* p) {
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(dev::smem_addr(p)));
   return v;
-}
-
-struct SelectScratch {
-  uint32_t hist[256];
-  int scan[4];
-  uint32_t bin, rem;
-};
-
-// Among n candidate (key, idx) pairs, keep exactly the m best (key descending, idx
-// ascending) and compact them to the front.  Returns the key of the m-th best.
-// Called by the 128 epilogue threads together; requires 1 <= m < n.
-__device__ uint32_t select_compact(uint32_t* ck, int32_t* ci, int n, int m, SelectScratch& S) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // --- radix select on the key (descending) ---
-  uint32_t prefix = 0, mask = 0, remaining = static_cast<uint32_t>(m);
-#pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    S.hist[tid] = 0u;
-    S.hist[tid + 128] = 0u;
-    epi_sync();
-    for (int e = tid; e < n; e += 128) {
-      const uint32_t key = ck[e];
-      if ((key & mask) == prefix) atomicAdd(&S.hist[(key >> shift) & 255u], 1u);
-    }
-    epi_sync();
-    if (warp == 0) {
-      uint32_t c[8], sum = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        c[j] = S.hist[255 - (8 * lane + j)];
-        sum += c[j];
-      }
-      const uint32_t inc = static_cast<uint32_t>(warp_inclusive_scan(static_cast<int>(sum)));
-      const uint32_t before = inc - sum;
-      if (before < remaining && remaining <= inc) {
-        uint32_t acc = before;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (acc + c[j] >= remaining) {
-            S.bin = 255u - static_cast<uint32_t>(8 * lane + j);
-            S.rem = remaining - acc;
-            break;
-          }
-          acc += c[j];
-        }
-      }
-    }
-    epi_sync();
-    prefix |= S.bin << shift;
-    mask |= 255u << shift;
-    remaining = S.rem;
-  }
-  const uint32_t kth = prefix;
-  const uint32_t need_eq = remaining;
-  // --- among keys equal to kth, the need_eq smallest indices (idx < 2^24) ---
-  uint32_t iprefix = 0, imask = 0, irem = need_eq;
-#pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = 16 - 8 * pass;
-    S.hist[tid] = 0u;
-    S.hist[tid + 128] = 0u;
-    epi_sync();
-    for (int e = tid; e < n; e += 128) {
-      const uint32_t id = static_cast<uint32_t>(ci[e]);
-      if (ck[e] == kth && (id & imask) == iprefix) atomicAdd(&S.hist[(id >> shift) & 255u], 1u);
-    }
-    epi_sync();
-    if (warp == 0) {
-      uint32_t c[8], sum = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        c[j] = S.hist[8 * lane + j];
-        sum += c[j];
-      }
-      const uint32_t inc = static_cast<uint32_t>(warp_inclusive_scan(static_cast<int>(sum)));
-      const uint32_t before = inc - sum;
-      if (before < irem && irem <= inc) {
-        uint32_t acc = before;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (acc + c[j] >= irem) {
-            S.bin = static_cast<uint32_t>(8 * lane + j);
-            S.rem = irem - acc;
-            break;
-          }
-          acc += c[j];
-        }
-      }
-    }
-    epi_sync();
-    iprefix |= S.bin << shift;
-    imask |= 255u << shift;
-    irem = S.rem;
-  }
-  const uint32_t idx_thr = iprefix;  // the need_eq-th smallest index among the ties
-  // --- in-place compaction, one chunk of 128 entries at a time ---
-  int base = 0;
-#pragma unroll 1
-  for (int c0 = 0; c0 < n; c0 += 128) {
-    const int e = c0 + tid;
-    uint32_t key = 0;
-    int32_t id = 0;
-    bool keep = false;
-    if (e < n) {
-      key = ck[e];
-      id = ci[e];
-      keep = key > kth || (key == kth && static_cast<uint32_t>(id) <= idx_thr);
-    }
-    int total;
-    const int pos = base + epi_scan(keep ? 1 : 0, S.scan, total);
-    if (keep) {
-      ck[pos] = key;
-      ci[pos] = id;
-    }
-    base += total;
-  }
-  epi_sync();
-  return kth;
 }
 
 }  // namespace idx_detail
@@ -217,6 +73,12 @@ struct IdxLayout {
   static constexpr int kKeyTileBytes = 128 * D_I;
 };
 
+template <int TOK>
+struct IdxGroups {
+  static constexpr int kEG = TOK >= 2 ? 2 : 1;   // epilogue groups
+  static constexpr int kThreads = (4 * kEG + 2) * 32;
+};
+
 // Shared-memory bytes the kernel needs (besides the 1 KB alignment slack).
 template <int D_I, int H_I, int TOK, int MODE, int STAGES>
 __host__ __device__ constexpr int indexer_smem_bytes(int cap) {
@@ -225,16 +87,21 @@ __host__ __device__ constexpr int indexer_smem_bytes(int cap) {
 }
 
 template <int D_I, int H_I, int TOK, int MODE, bool PAGED, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                    const IndexerParams p) {
   using namespace dev;
   using L = IdxLayout<D_I>;
+  constexpr int EG = IdxGroups<TOK>::kEG;
+  constexpr int TPG = TOK / EG;          // tokens per epilogue group
   constexpr int N = TOK * H_I;
+  constexpr int NG = N / EG;             // accumulator columns per group
   constexpr int Q_BYTES = N * D_I;
   constexpr int TMEM_COLS = (2 * N < 32) ? 32 : 2 * N;
   constexpr uint32_t IDESC = idesc_e4m3(128, N);
+  constexpr int PRODUCER_WARP = 4 * EG, MMA_WARP = 4 * EG + 1;
   static_assert(N % 16 == 0 && N <= 256, "MMA N must be a multiple of 16 in [16, 256]");
+  static_assert(NG % 8 == 0, "group column slice must be a multiple of 8");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -247,9 +114,8 @@ __global__ void __launch_bounds__(192, 1)
   __shared__ uint64_t bar_kfull[STAGES], bar_kempty[STAGES], bar_accfull[2], bar_accempty[2], bar_q;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ int s_cnt[TOK];
-  __shared__ long long s_thr[TOK];
-  __shared__ idx_detail::SelectScratch s_sel;
+  __shared__ int s_cnt[TOK][4];       // candidate count per token and warp region
+  __shared__ sel::Scratch s_sel[EG];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -295,13 +161,13 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_accfull[i], 1);
-      mbar_init(&bar_accempty[i], 4);
+      mbar_init(&bar_accempty[i], 4 * EG);
     }
     mbar_init(&bar_q, 1);
     s_abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == MMA_WARP) {
     tmem_alloc(&s_tmem, TMEM_COLS);
     tmem_relinquish();
   }
@@ -314,16 +180,12 @@ __global__ void __launch_bounds__(192, 1)
     }
     sWq[i] = v;
   }
-  if (MODE == kIdxTopk && tid < TOK) {
-    s_cnt[tid] = 0;
-    s_thr[tid] = -1;
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
 
-  if (warp == 4) {
+  if (warp == PRODUCER_WARP) {
     // ================= TMA producer =================
     if (lane == 0) {
       tma_prefetch_desc(&q_map);
@@ -356,7 +218,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == MMA_WARP) {
     // ================= MMA issuer =================
     if (lane == 0) {
       bool ok = mbar_wait(&bar_q, 0);
@@ -390,61 +252,76 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // ================= epilogue (warps 0-3) =================
-    const int e = tid;  // TMEM lane == key within the tile
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    // ================= epilogue groups =================
+    const int g = warp >> 2;                    // group
+    const int q = warp & 3;                     // TMEM lane quadrant
+    const sel::Group G{1 + g, tid - 128 * g};
+    const int e = 32 * q + lane;                // key within the tile
+    const int tg0 = g * TPG;                    // first token of this group
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + g * NG;
     const int seq_start = PAGED ? 0 : p.cu_seqlens[b];
     const int32_t* bt = PAGED ? p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq : nullptr;
+    const int Q = p.cap / 4;
     bool aborted = false;
+    // fused top-k state in registers: this warp's region fill count, the acceptance
+    // threshold (uniform), and the smallest / largest key this thread appended
+    int wcnt[TPG];
+    long long thr[TPG];
+    uint32_t kmin[TPG], kmax[TPG];
+#pragma unroll
+    for (int tt = 0; tt < TPG; ++tt) {
+      wcnt[tt] = 0;
+      thr[tt] = -1;
+      kmin[tt] = 0xFFFFFFFFu;
+      kmax[tt] = 0u;
+    }
 #pragma unroll 1
     for (int it = 0; it < ntiles; ++it) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       const int s = (tile0 + it) * 128 + e;  // local key position
-      // k_scale of this lane's key (0 beyond the sequence)
-      float ksc = 0.f;
+      float ksc = 0.f;                       // k_scale of this lane's key (0 beyond the sequence)
       if (s < len) {
         if constexpr (!PAGED) ksc = p.k_scale[seq_start + s];
         else ksc = p.k_scale[static_cast<int64_t>(bt[s >> 6]) * 64 + (s & 63)];
       }
       const bool ok = mbar_wait(&bar_accfull[acc], aph);
       if (!ok) record_device_error(DSA_ERR_TIMEOUT);
-      if (idx_detail::epi_any(!ok)) {
+      if (sel::gany(G, !ok)) {
         aborted = true;
         break;
       }
       tc_fence_after();
-      float part[TOK][2];
+      float part[TPG][2];
 #pragma unroll
-      for (int tt = 0; tt < TOK; ++tt) part[tt][0] = part[tt][1] = 0.f;
-      if constexpr (N == 16) {
-        uint32_t r[16];
-        tmem_ld16(lane_base + acc * N, r);
+      for (int tt = 0; tt < TPG; ++tt) part[tt][0] = part[tt][1] = 0.f;
+      constexpr int CH = NG >= 32 ? 32 : NG;
+#pragma unroll
+      for (int c0 = 0; c0 < NG; c0 += CH) {
+        uint32_t r[32];
+        if constexpr (CH == 32) {
+          tmem_ld32(lane_base + acc * N + c0, r);
+        } else if constexpr (CH == 16) {
+          tmem_ld16(lane_base + acc * N + c0, *reinterpret_cast<uint32_t(*)[16]>(r));
+        } else {
+          uint32_t r16[16];
+          static_assert(CH == 8, "unsupported column slice");
+          asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                       : "=r"(r16[0]), "=r"(r16[1]), "=r"(r16[2]), "=r"(r16[3]), "=r"(r16[4]), "=r"(r16[5]),
+                         "=r"(r16[6]), "=r"(r16[7])
+                       : "r"(lane_base + acc * N + c0));
+#pragma unroll
+          for (int u = 0; u < 8; ++u) r[u] = r16[u];
+        }
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 16; c += 4) {
-          const float4 w4 = idx_detail::lds128(sWq + c);
+        for (int c = 0; c < CH; c += 4) {
+          const float4 w4 = idx_detail::lds128(sWq + g * NG + c0 + c);
           const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            part[(c + u) / H_I][u & 1] =
-                fmaf(wv[u], fmaxf(__uint_as_float(r[c + u]), 0.f), part[(c + u) / H_I][u & 1]);
-        }
-      } else {
-#pragma unroll
-        for (int c0 = 0; c0 < N; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(lane_base + acc * N + c0, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            const float4 w4 = idx_detail::lds128(sWq + c0 + c);
-            const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int col = c0 + c + u;
-              part[col / H_I][u & 1] = fmaf(wv[u], fmaxf(__uint_as_float(r[c + u]), 0.f), part[col / H_I][u & 1]);
-            }
+          for (int u = 0; u < 4; ++u) {
+            const int col = c0 + c + u;  // column inside the group's slice
+            part[col / H_I][u & 1] = fmaf(wv[u], fmaxf(__uint_as_float(r[c + u]), 0.f), part[col / H_I][u & 1]);
           }
         }
       }
@@ -454,48 +331,62 @@ __global__ void __launch_bounds__(192, 1)
 
       if constexpr (MODE == kIdxScores) {
 #pragma unroll
-        for (int tt = 0; tt < TOK; ++tt) {
-          if (tt >= ntok) break;
-          const int t = t0 + tt;
+        for (int tt = 0; tt < TPG; ++tt) {
+          if (tg0 + tt >= ntok) break;
+          const int t = t0 + tg0 + tt;
           const float score = (part[tt][0] + part[tt][1]) * ksc;
           if constexpr (!PAGED) {
-            const int64_t g = seq_start + t;
-            if (g >= p.row_begin && g < p.row_end && s < len)
-              p.scores[(g - p.row_begin) * p.ld + s] = s <= t ? score : -INFINITY;
+            const int64_t gr = seq_start + t;
+            if (gr >= p.row_begin && gr < p.row_end && s < len)
+              p.scores[(gr - p.row_begin) * p.ld + s] = s <= t ? score : -INFINITY;
           } else {
             if (s < len) p.scores[(b - p.row_begin) * p.ld + s] = score;
           }
         }
       } else {
+        bool need_cut = false;
 #pragma unroll
-        for (int tt = 0; tt < TOK; ++tt) {
-          if (tt >= ntok) break;
-          const int t = t0 + tt;
-          if (s <= t && s < len) {
-            const float score = (part[tt][0] + part[tt][1]) * ksc;
-            const uint32_t u = __float_as_uint(score);
-            if (is_nan_bits(u)) record_device_error(DSA_ERR_DEVICE_CHECK);
-            const uint32_t key = order_key(score);
-            if (static_cast<long long>(key) > s_thr[tt]) {
-              const int pos = atomicAdd(&s_cnt[tt], 1);
-              sCandKey[tt * p.cap + pos] = key;
-              sCandIdx[tt * p.cap + pos] = s;
-            }
+        for (int tt = 0; tt < TPG; ++tt) {
+          const int t = t0 + tg0 + tt;
+          const float score = (part[tt][0] + part[tt][1]) * ksc;
+          const bool valid = tg0 + tt < ntok && s <= t && s < len;
+          if (valid && is_nan_bits(__float_as_uint(score))) record_device_error(DSA_ERR_DEVICE_CHECK);
+          const uint32_t key = order_key(score);
+          const bool take = valid && static_cast<long long>(key) > thr[tt];
+          const uint32_t m = __ballot_sync(0xffffffffu, take);
+          if (take) {
+            const int pos = (tg0 + tt) * p.cap + q * Q + wcnt[tt] + __popc(m & ((1u << lane) - 1u));
+            sCandKey[pos] = key;
+            sCandIdx[pos] = s;
+            kmin[tt] = min(kmin[tt], key);
+            kmax[tt] = max(kmax[tt], key);
           }
+          wcnt[tt] += __popc(m);
+          need_cut |= wcnt[tt] > Q - 32;  // the next tile could add 32 more to this region
         }
-        idx_detail::epi_sync();
-#pragma unroll 1
-        for (int tt = 0; tt < ntok; ++tt) {
-          const int n = s_cnt[tt];
-          if (n > p.cap - 128) {
-            const uint32_t kth = idx_detail::select_compact(sCandKey + tt * p.cap, sCandIdx + tt * p.cap, n, p.k,
-                                                            s_sel);
-            if (tid == 0) {
-              s_cnt[tt] = p.k;
-              s_thr[tt] = static_cast<long long>(kth);
-            }
-            idx_detail::epi_sync();
+        if (sel::gany(G, need_cut)) {
+          if (lane == 0) {
+#pragma unroll
+            for (int tt = 0; tt < TPG; ++tt) s_cnt[tg0 + tt][q] = wcnt[tt];
           }
+          sel::gsync(G);
+#pragma unroll
+          for (int tt = 0; tt < TPG; ++tt) {
+            const int tok = tg0 + tt;
+            const bool full = s_cnt[tok][0] > Q - 32 || s_cnt[tok][1] > Q - 32 || s_cnt[tok][2] > Q - 32 ||
+                              s_cnt[tok][3] > Q - 32;
+            if (full) {  // uniform over the group
+              uint32_t lo, hi;
+              sel::group_minmax(G, s_sel[g], kmin[tt], kmax[tt], lo, hi);
+              if (thr[tt] >= 0) lo = min(lo, static_cast<uint32_t>(thr[tt]));  // the smallest kept key
+              sel::Cands C{sCandKey + tok * p.cap, sCandIdx + tok * p.cap, &s_cnt[tok][0], Q};
+              const uint32_t nthr = sel::cut_stream(G, C, s_sel[g], p.k, p.cap - 512, lo, hi);
+              thr[tt] = static_cast<long long>(nthr);
+              kmin[tt] = 0xFFFFFFFFu;  // every later key is > thr
+            }
+            wcnt[tt] = s_cnt[tok][q];
+          }
+          sel::gsync(G);
         }
       }
     }
@@ -504,46 +395,34 @@ __global__ void __launch_bounds__(192, 1)
       if constexpr (MODE == kIdxScores && !PAGED) {
         // columns past the last computed tile are outside every causal prefix of this CTA
         const int s_begin = ntiles * 128;
-        for (int tt = 0; tt < ntok; ++tt) {
-          const int64_t g = seq_start + t0 + tt;
-          if (g < p.row_begin || g >= p.row_end) continue;
-          float* row = p.scores + (g - p.row_begin) * p.ld;
+        for (int tt = 0; tt < TPG; ++tt) {
+          if (tg0 + tt >= ntok) break;
+          const int64_t gr = seq_start + t0 + tg0 + tt;
+          if (gr < p.row_begin || gr >= p.row_end) continue;
+          float* row = p.scores + (gr - p.row_begin) * p.ld;
           for (int s = s_begin + e; s < len; s += 128) row[s] = -INFINITY;
         }
       }
       if constexpr (MODE == kIdxTopk) {
-        // final cut to min(k, t+1) and ascending emission through a bitmap (aliases the key ring)
-        uint32_t* bitmap = reinterpret_cast<uint32_t*>(sK);
+        // final cut to min(k, t+1) and ascending emission through a bitmap (aliases the key
+        // ring; each group has its own half)
+        if (lane == 0) {
+#pragma unroll
+          for (int tt = 0; tt < TPG; ++tt) s_cnt[tg0 + tt][q] = wcnt[tt];
+        }
+        sel::gsync(G);
+        uint32_t* bitmap = reinterpret_cast<uint32_t*>(sK + g * (STAGES * L::kKeyTileBytes / EG));
 #pragma unroll 1
-        for (int tt = 0; tt < ntok; ++tt) {
-          const int t = t0 + tt;
-          const int m = min(p.k, t + 1);
-          uint32_t* ck = sCandKey + tt * p.cap;
-          int32_t* ci = sCandIdx + tt * p.cap;
-          const int n = s_cnt[tt];
-          if (n > m) idx_detail::select_compact(ck, ci, n, m, s_sel);
-          const int nwords = (t + 1 + 31) / 32;
-          for (int wd = e; wd < nwords; wd += 128) bitmap[wd] = 0u;
-          idx_detail::epi_sync();
-          for (int i = e; i < m; i += 128) atomicOr(&bitmap[ci[i] >> 5], 1u << (ci[i] & 31));
-          idx_detail::epi_sync();
-          const int per = (nwords + 127) / 128;
-          const int w0 = min(nwords, e * per), w1 = min(nwords, w0 + per);
-          int bits = 0;
-          for (int wd = w0; wd < w1; ++wd) bits += __popc(bitmap[wd]);
-          int total;
-          int pos = idx_detail::epi_scan(bits, s_sel.scan, total);
-          int32_t* out = p.idx_out + static_cast<int64_t>(seq_start + t) * p.k;
-          for (int wd = w0; wd < w1; ++wd) {
-            uint32_t word = bitmap[wd];
-            while (word) {
-              const int bit = __ffs(word) - 1;
-              out[pos++] = wd * 32 + bit;
-              word &= word - 1;
-            }
-          }
-          for (int i = m + e; i < p.k; i += 128) out[i] = -1;
-          idx_detail::epi_sync();
+        for (int tt = 0; tt < TPG; ++tt) {
+          const int tok = tg0 + tt;
+          if (tok >= ntok) break;
+          const int t = t0 + tok;
+          uint32_t lo, hi;
+          sel::group_minmax(G, s_sel[g], kmin[tt], kmax[tt], lo, hi);
+          if (thr[tt] >= 0) lo = min(lo, static_cast<uint32_t>(thr[tt]));  // the smallest kept key
+          sel::Cands C{sCandKey + tok * p.cap, sCandIdx + tok * p.cap, &s_cnt[tok][0], Q};
+          sel::cut_final(G, C, s_sel[g], min(p.k, t + 1), lo, hi);
+          sel::emit_sorted(G, C, s_sel[g], bitmap, t + 1, p.idx_out + static_cast<int64_t>(seq_start + t) * p.k, p.k);
         }
       }
     }
@@ -551,7 +430,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
