@@ -73,6 +73,8 @@ _lib.dsa_sparse_mla_decode.restype = _I32
 _lib.dsa_forward.argtypes = [_I32, _P, _P, _P, _DESC, _P, _DESC, _I32, _I32, _I32, _I32, _I32, _F32, _P, _P, _P,
                              _P, _SZ, _P]
 _lib.dsa_forward.restype = _I32
+_lib.dsa_indexer_topk.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I32, _P, _P]
+_lib.dsa_indexer_topk.restype = _I32
 _lib.dsa_workspace_size.argtypes = [_I32, _I32, _I64, _I32, _I32, _I32, _I32]
 _lib.dsa_workspace_size.restype = _SZ
 
@@ -180,3 +182,10 @@ def dsa_device_error(stream=None) -> int:
     code = _I32(0)
     _check(_lib.dsa_device_error(ctypes.byref(code), _stream(stream)), "dsa_device_error")
     return int(code.value)
+
+
+def dsa_indexer_topk(q_fp8, q_scale, w, keys: Desc, B, H_I, d_I, k, idx_out, stream=None):
+    """Fused indexer + top-k for prefill: idx_out [T, k] (ascending, -1 padded)."""
+    _check(_lib.dsa_indexer_topk(_ptr(q_fp8), _ptr(q_scale), _ptr(w), keys.ref(), int(B), int(H_I), int(d_I), int(k),
+                                 _ptr(idx_out), _stream(stream)), "dsa_indexer_topk")
+    return idx_out

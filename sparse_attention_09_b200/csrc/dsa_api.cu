@@ -12,6 +12,7 @@
 #include "../../include/dsa.h"
 #include "common.cuh"
 #include "indexer.cuh"
+#include "sparse_mla.cuh"
 #include "topk.cuh"
 
 namespace dsa {
@@ -136,6 +137,40 @@ dsa_status indexer_common(const uint8_t* q_fp8, const float* q_scale, const floa
   return DSA_OK;
 }
 
+// ---- sparse MLA ------------------------------------------------------------------------------
+constexpr int kMlaClusters = 74;   // one CTA pair per two SMs of a 148-SM B200
+constexpr int kDecodeSplits = 4;   // decode: splits of each sequence's selection
+constexpr int kLatentDim = 576, kValueDim = 512;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t decode_partials_bytes(int B, int H, int splits) {
+  return align256(static_cast<size_t>(B) * splits * H * kValueDim * 4) + align256(static_cast<size_t>(B) * splits * H * 2 * 4);
+}
+
+int decode_splits(int k) { return k / 64 < kDecodeSplits ? k / 64 : kDecodeSplits; }
+
+bool make_latent_maps(const void* data, uint64_t rows, CUtensorMap* m128, CUtensorMap* m64) {
+  return make_map_2d(m128, data, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kLatentDim, rows, kLatentDim * 2, 64, 1,
+                     CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map_2d(m64, data, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kLatentDim, rows, kLatentDim * 2, 32, 1,
+                     CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+template <bool DECODE>
+dsa_status launch_mla(const CUtensorMap& m128, const CUtensorMap& m64, const MlaParams& p, int64_t units,
+                      cudaStream_t s) {
+  auto kern = sparse_mla_kernel<DECODE>;
+  const int smem = mla::kSmemBytes + 1024;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  const int clusters = static_cast<int>(units < kMlaClusters ? units : kMlaClusters);
+  kern<<<2 * clusters, 192, smem, s>>>(m128, m64, p);
+  return launch_status();
+}
+
+bool mla_shape_ok(int H, int k) { return H >= 1 && H <= 128 && k >= 64 && k <= 2048 && k % 64 == 0; }
+
 }  // namespace
 }  // namespace dsa
 
@@ -230,22 +265,124 @@ dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, const fl
   return launch_indexer<kIdxTopk, false>(d_I, H_I, qm, km, p, grid, as_stream(stream));
 }
 
-dsa_status dsa_sparse_mla_prefill(const void*, const dsa_kv_desc*, const int32_t*, int32_t, int32_t, int32_t, float,
-                                  void*, float*, void*) {
-  return DSA_ERR_UNSUPPORTED;
+dsa_status dsa_sparse_mla_prefill(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B, int32_t H,
+                                  int32_t k, float sm_scale, void* out, float* lse, void* stream) {
+  if (q == nullptr || latent == nullptr || latent->data == nullptr || idx == nullptr || out == nullptr || B <= 0)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (latent->kind != DSA_KV_CONTIGUOUS || latent->cu_seqlens == nullptr || latent->total_tokens <= 0)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(latent->data, 16) || !aligned(idx, 16) || !aligned(out, 16))
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (!mla_shape_ok(H, k)) return DSA_ERR_UNSUPPORTED;
+  if (latent->total_tokens > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+  CUtensorMap m128, m64;
+  if (!make_latent_maps(latent->data, static_cast<uint64_t>(latent->total_tokens), &m128, &m64))
+    return DSA_ERR_INVALID_ARGUMENT;
+  MlaParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.idx = idx;
+  p.cu_seqlens = latent->cu_seqlens;
+  p.B = B;
+  p.H = H;
+  p.k = k;
+  p.rows = latent->total_tokens;
+  p.splits = 1;
+  p.scale_log2 = sm_scale * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  return launch_mla<false>(m128, m64, p, p.rows, as_stream(stream));
 }
 
-dsa_status dsa_sparse_mla_decode(const void*, const dsa_kv_desc*, const int32_t*, int32_t, int32_t, int32_t, float,
-                                 void*, float*, void*, size_t, void*) {
-  return DSA_ERR_UNSUPPORTED;
+dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B, int32_t H,
+                                 int32_t k, float sm_scale, void* out, float* lse, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  if (q == nullptr || latent == nullptr || latent->data == nullptr || idx == nullptr || out == nullptr || B <= 0)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (latent->kind != DSA_KV_PAGED || latent->block_table == nullptr || latent->context_lens == nullptr ||
+      latent->num_blocks <= 0 || latent->max_blocks_per_seq <= 0)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (latent->block_size != 64) return DSA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(latent->data, 16) || !aligned(idx, 16) || !aligned(out, 16))
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (!mla_shape_ok(H, k)) return DSA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(latent->num_blocks) * 64 > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+  const int splits = decode_splits(k);
+  if (workspace == nullptr || ws_bytes < decode_partials_bytes(B, H, splits) || !aligned(workspace, 256))
+    return workspace == nullptr ? DSA_ERR_INVALID_ARGUMENT : DSA_ERR_WORKSPACE_TOO_SMALL;
+  CUtensorMap m128, m64;
+  if (!make_latent_maps(latent->data, static_cast<uint64_t>(latent->num_blocks) * 64, &m128, &m64))
+    return DSA_ERR_INVALID_ARGUMENT;
+  MlaParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.idx = idx;
+  p.block_table = latent->block_table;
+  p.context_lens = latent->context_lens;
+  p.max_blocks_per_seq = latent->max_blocks_per_seq;
+  p.B = B;
+  p.H = H;
+  p.k = k;
+  p.rows = B;
+  p.splits = splits;
+  p.scale_log2 = sm_scale * 1.4426950408889634f;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                       align256(static_cast<size_t>(B) * splits * H * kValueDim * 4));
+  cudaStream_t s = as_stream(stream);
+  dsa_status st = launch_mla<true>(m128, m64, p, static_cast<int64_t>(B) * splits, s);
+  if (st != DSA_OK) return st;
+  mla_combine_kernel<<<dim3(H, B), 128, 0, s>>>(p.part_o, p.part_ml, splits, H, static_cast<__nv_bfloat16*>(out), lse);
+  return launch_status();
 }
 
-dsa_status dsa_forward(int32_t, const uint8_t*, const float*, const float*, const dsa_kv_desc*, const void*,
-                       const dsa_kv_desc*, int32_t, int32_t, int32_t, int32_t, int32_t, float, void*, float*,
-                       int32_t*, void*, size_t, void*) {
-  return DSA_ERR_UNSUPPORTED;
+dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale, const float* w,
+                       const dsa_kv_desc* keys, const void* q, const dsa_kv_desc* latent, int32_t B, int32_t H_I,
+                       int32_t d_I, int32_t H, int32_t k, float sm_scale, void* out, float* lse, int32_t* idx_out,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  if (keys == nullptr || latent == nullptr || B <= 0) return DSA_ERR_INVALID_ARGUMENT;
+  if (!mla_shape_ok(H, k)) return DSA_ERR_UNSUPPORTED;
+  const size_t need = dsa_workspace_size(mode, B, keys->total_tokens, keys->max_seqlen, H, H_I, k);
+  if (mode == DSA_MODE_PREFILL) {
+    if (keys->kind != DSA_KV_CONTIGUOUS || latent->kind != DSA_KV_CONTIGUOUS) return DSA_ERR_INVALID_ARGUMENT;
+    int32_t* idx = idx_out;
+    if (idx == nullptr) {
+      if (workspace == nullptr) return DSA_ERR_INVALID_ARGUMENT;
+      if (ws_bytes < need) return DSA_ERR_WORKSPACE_TOO_SMALL;
+      idx = static_cast<int32_t*>(workspace);
+    }
+    dsa_status st = dsa_indexer_topk(q_fp8, q_scale, w, keys, B, H_I, d_I, k, idx, stream);
+    if (st != DSA_OK) return st;
+    return dsa_sparse_mla_prefill(q, latent, idx, B, H, k, sm_scale, out, lse, stream);
+  }
+  if (mode != DSA_MODE_DECODE) return DSA_ERR_INVALID_ARGUMENT;
+  if (keys->kind != DSA_KV_PAGED || latent->kind != DSA_KV_PAGED) return DSA_ERR_INVALID_ARGUMENT;
+  if (workspace == nullptr) return DSA_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < need || !aligned(workspace, 256)) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  // workspace: [decode partials][scores B x ld][selection B x k]
+  const int splits = decode_splits(k);
+  const size_t part = decode_partials_bytes(B, H, splits);
+  const int64_t ld = (static_cast<int64_t>(keys->max_seqlen) + 3) / 4 * 4;
+  float* scores = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + part);
+  int32_t* idx = idx_out != nullptr
+                     ? idx_out
+                     : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + part +
+                                                  align256(static_cast<size_t>(B) * ld * 4));
+  dsa_status st = dsa_indexer_scores(q_fp8, q_scale, w, keys, B, H_I, d_I, 0, B, scores, ld, stream);
+  if (st != DSA_OK) return st;
+  st = dsa_topk(scores, ld, B, keys->context_lens, k, idx, stream);
+  if (st != DSA_OK) return st;
+  return dsa_sparse_mla_decode(q, latent, idx, B, H, k, sm_scale, out, lse, workspace, part, stream);
 }
 
-size_t dsa_workspace_size(int32_t, int32_t, int64_t, int32_t, int32_t, int32_t, int32_t) { return 0; }
+size_t dsa_workspace_size(int32_t mode, int32_t B, int64_t total_tokens, int32_t max_ctx, int32_t H, int32_t H_I,
+                          int32_t k) {
+  (void)H_I;
+  if (B <= 0 || k <= 0 || H <= 0) return 0;
+  if (mode == DSA_MODE_PREFILL) return align256(static_cast<size_t>(total_tokens > 0 ? total_tokens : 0) * k * 4);
+  const int64_t ld = (static_cast<int64_t>(max_ctx > 0 ? max_ctx : 0) + 3) / 4 * 4;
+  return decode_partials_bytes(B, H, decode_splits(k)) + align256(static_cast<size_t>(B) * ld * 4) +
+         align256(static_cast<size_t>(B) * k * 4);
+}
 
 }  // extern "C"

@@ -41,15 +41,56 @@ def indexer_topk(inp, k):
     dsa = lib()
     T = inp["q8"].shape[0]
     idx = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
-    lib_fn = dsa._lib.dsa_indexer_topk
-    import ctypes
-    st = lib_fn(ctypes.c_void_p(inp["q8"].data_ptr()), ctypes.c_void_p(inp["q_scale"].data_ptr()),
-                ctypes.c_void_p(inp["w"].data_ptr()), keys_desc(inp).ref(), len(inp["seqlens"]), inp["H_I"],
-                inp["d_I"], k, ctypes.c_void_p(idx.data_ptr()),
-                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
-    assert st == 0, dsa.dsa_status_string(st)
+    dsa.dsa_indexer_topk(inp["q8"], inp["q_scale"], inp["w"], keys_desc(inp), len(inp["seqlens"]), inp["H_I"],
+                         inp["d_I"], k, idx)
     assert dsa.dsa_device_error() == 0
     return idx
+
+
+def random_selection(seqlens, k, seed, device="cuda", scatter_pad=False):
+    """A valid selection per token: min(k, t+1) distinct causal positions, ascending, -1 padded
+    (or, with scatter_pad, the -1 entries shuffled among the valid ones)."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    rows = []
+    for L in seqlens:
+        r = torch.rand(L, L, generator=g, device=device)
+        r = r.masked_fill(torch.ones(L, L, dtype=torch.bool, device=device).triu(1), -1.0)
+        kk = min(k, L)
+        top = torch.topk(r, kk, dim=1).indices
+        vals = torch.gather(r, 1, top)
+        top = torch.where(vals >= 0, top, torch.full_like(top, 1 << 30))
+        top = torch.sort(top, dim=1).values
+        top = torch.where(top >= (1 << 30), torch.full_like(top, -1), top).to(torch.int32)
+        sel = torch.full((L, k), -1, dtype=torch.int32, device=device)
+        sel[:, :kk] = top
+        if scatter_pad:
+            perm = torch.argsort(torch.rand(L, k, generator=g, device=device), dim=1)
+            sel = torch.gather(sel, 1, perm)
+        rows.append(sel)
+    return torch.cat(rows, 0).contiguous()
+
+
+def sparse_mla_prefill(inp, idx, k, sm_scale, with_lse=True):
+    dsa = lib()
+    T, H = inp["q"].shape[0], inp["q"].shape[1]
+    out = torch.full((T, H, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((T, H), float("nan"), device="cuda") if with_lse else None
+    dsa.dsa_sparse_mla_prefill(inp["q"], latent_desc(inp), idx, len(inp["seqlens"]), H, k, sm_scale, out, lse)
+    assert dsa.dsa_device_error() == 0
+    return out, lse
+
+
+def assert_attention_close(got, ref, what=""):
+    """The stated bar (max-abs 2e-2, mean-abs 2e-3 after bf16 rounding) plus a relative bar
+    (1e-2 of the reference norm), since the synthetic outputs are only ~1e-2 in size."""
+    g = np.asarray(got, dtype=np.float64)
+    r = np.asarray(torch.from_numpy(np.asarray(ref, dtype=np.float32)).to(torch.bfloat16).float().numpy(),
+                   dtype=np.float64)
+    d = np.abs(g - r)
+    assert d.max() <= 2e-2, f"{what} max-abs {d.max():.3e}"
+    assert d.mean() <= 2e-3, f"{what} mean-abs {d.mean():.3e}"
+    rel = np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30)
+    assert rel <= 1e-2, f"{what} relative {rel:.3e}"
 
 
 def oracle_scores(seq_np, rows):

@@ -1,0 +1,115 @@
+"""Sparse MLA (2-CTA cluster, tcgen05 BF16, TMA gather) against the oracle on the GPU's own
+index set: max-abs <= 2e-2 and mean-abs <= 2e-3 after bf16 rounding (the stated bar), plus
+relative error <= 1e-2 (outputs here are ~1e-2, so the absolute bar alone would be loose).
+
+lse bound: each softmax weight is the product of two bf16-rounded factors, rounded again to
+bf16 for the P.V product, so it carries up to 3 * 2^-9 ~ 5.9e-3 relative error; the row sum l
+inherits at most that, hence |lse_gpu - lse_ref| <= 1e-2."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import assert_attention_close, random_selection, sparse_mla_prefill
+
+pytestmark = pytest.mark.gpu
+
+LSE_TOL = 1e-2
+
+
+def _check_rows(inp, idx, rows_per_seq, sm_scale, out, lse):
+    cu = inp["cu_seqlens"].cpu().numpy()
+    idx_h = idx.cpu().numpy()
+    out_h = out.float().cpu().numpy()
+    lse_h = lse.cpu().numpy() if lse is not None else None
+    H = inp["q"].shape[1]
+    for b, rows in enumerate(rows_per_seq):
+        seq = synth.seq_slice_numpy(inp, b, rows=rows)
+        for t in rows:
+            g = cu[b] + t
+            sel = idx_h[g][idx_h[g] >= 0]
+            ref, ref_lse = oracle.sparse_mla_token(seq["q"][t], seq["latent"], sel, sm_scale)
+            assert_attention_close(out_h[g], ref, f"seq {b} row {t}")
+            if lse_h is not None:
+                assert np.allclose(lse_h[g], ref_lse, rtol=0, atol=LSE_TOL), f"lse seq {b} row {t}"
+
+
+@pytest.mark.parametrize("name,seqlens,k,rows", [
+    ("tiny_256", [256], 64, None),
+    ("tiny_256", [100, 37, 256], 64, None),
+    ("prefill_8k", [3000], 2048, [0, 1, 63, 64, 65, 2047, 2048, 2999]),
+    ("prefill_8k", [700, 1300], 512, [0, 511, 512, 699]),
+])
+def test_prefill_matches_oracle(name, seqlens, k, rows):
+    cfg = dict(synth.WORKLOADS[name])
+    cfg["seqlens"] = seqlens
+    inp = synth.prefill_inputs(device="cuda", **cfg)
+    idx = random_selection(seqlens, k, seed=len(seqlens) + k)
+    sm = 1.0 / math.sqrt(576)
+    out, lse = sparse_mla_prefill(inp, idx, k, sm)
+    rows_per_seq = [list(range(L)) if rows is None else [r for r in rows if r < L] for L in seqlens]
+    _check_rows(inp, idx, rows_per_seq, sm, out, lse)
+
+
+def test_scattered_padding_and_large_logits():
+    # large logits exercise the running-max updates and rescaling; scattered -1 entries the masks
+    cfg = dict(synth.WORKLOADS["prefill_8k"])
+    cfg["seqlens"] = [1500]
+    inp = synth.prefill_inputs(device="cuda", **cfg)
+    inp["q"] = (inp["q"].float() * 3000.0).to(torch.bfloat16)
+    k = 1024
+    idx = random_selection([1500], k, seed=9, scatter_pad=True)
+    sm = 1.0 / math.sqrt(576)
+    out, lse = sparse_mla_prefill(inp, idx, k, sm)
+    _check_rows(inp, idx, [[0, 3, 100, 1023, 1024, 1499]], sm, out, lse)
+
+
+def test_k_at_least_L_is_dense_causal_attention():
+    cfg = dict(synth.WORKLOADS["prefill_8k"])
+    L = 200
+    cfg["seqlens"] = [L]
+    inp = synth.prefill_inputs(device="cuda", **cfg)
+    k = 256
+    idx = torch.full((L, k), -1, dtype=torch.int32, device="cuda")
+    for t in range(L):
+        idx[t, : t + 1] = torch.arange(t + 1, dtype=torch.int32)
+    sm = 1.0 / math.sqrt(576)
+    out, _ = sparse_mla_prefill(inp, idx, k, sm)
+    q = inp["q"].float().permute(1, 0, 2).double().cpu()
+    lat = inp["latent"].double().cpu()
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q, lat[None].expand(q.shape[0], -1, -1), lat[None, :, :512].expand(q.shape[0], -1, -1), is_causal=True,
+        scale=sm).permute(1, 0, 2).numpy()
+    for t in range(L):
+        assert_attention_close(out[t].float().cpu().numpy(), ref[t], f"row {t}")
+
+
+def test_decode_paged_matches_oracle():
+    import sparse_attention_09_b200 as dsa
+    B, k = 5, 2048
+    d = synth.decode_inputs(B=B, ctx_lo=1, ctx_hi=5000, H_I=64, d_I=128, H=128, seed=4, device="cuda",
+                            ctx=[1, 300, 2048, 2049, 4999])
+    idx = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(1)
+    for b, c in enumerate(d["ctx_host"]):
+        m = min(k, c)
+        sel = torch.sort(torch.randperm(c, generator=g, device="cuda")[:m]).values
+        idx[b, :m] = sel.to(torch.int32)
+    latent = dsa.paged_desc(d["latent_cache"], d["block_table"], d["ctx"], d["max_ctx"])
+    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, 64, k), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.full((B, 128, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, 128), float("nan"), device="cuda")
+    sm = 1.0 / math.sqrt(576)
+    dsa.dsa_sparse_mla_decode(d["q"], latent, idx, B, 128, k, sm, out, lse, ws)
+    assert dsa.dsa_device_error() == 0
+    for b in range(B):
+        seq = synth.decode_seq_numpy(d, b)
+        lat = oracle.paged_gather(seq["latent_cache"], seq["block_table"], seq["ctx"])
+        sel = idx[b].cpu().numpy()
+        ref, ref_lse = oracle.sparse_mla_token(seq["q"], lat, sel[sel >= 0], sm)
+        assert_attention_close(out[b].float().cpu().numpy(), ref, f"seq {b}")
+        assert np.allclose(lse[b].cpu().numpy(), ref_lse, rtol=0, atol=LSE_TOL)
