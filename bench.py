@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA hot path (lightning indexer -> top-k -> sparse MLA) on B200.
+
+One step = one DSA prefill forward over the L = 131072 workload (k = 2048, 64 FP8 indexer
+heads, 128-head MLA-MQA): the fused indexer + top-k kernel, then the sparse MLA kernel, both
+through the C ABI.  The decode chain (64 sequences, 8K-128K contexts, paged caches) is timed in
+the same run and reported under "decode".  Inputs are seeded synthetic tensors generated on
+the device (about 40 GB per prefill step, far larger than L2, so no flush is needed).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs an independent prefill problem of the same size
+(no data-path collective; weak scaling) and the step time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "DSA prefill tokens/s at L=128K, k=2048; decode tokens/s; % of roofline"
+PREFILL = "prefill_128k"
+DECODE = "decode_64"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = {
+    "indexer_topk": ["indexer.cuh", "select.cuh", "sm100.cuh", "common.cuh"],
+    "sparse_mla": ["sparse_mla.cuh", "sm100.cuh", "common.cuh"],
+}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(kernel):
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "sparse_attention_09_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{PREFILL}.txt")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("source_sha") != source_hash(kernel):
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+
+    def __init__(self, index):
+        self.path = tempfile.mktemp(suffix=".csv")
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------------------------
+# oracle timing (the CPU baseline and the reference arm)
+# ------------------------------------------------------------------------------------------
+def oracle_prefill_sample(inp, k, rows, sm):
+    import oracle
+    seq = synth.seq_slice_numpy(inp, 0, rows=rows)
+    t0 = time.perf_counter()
+    oracle.dsa_prefill_rows(seq, k, sm, rows)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads") for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------
+def prefill_work(cfg):
+    L = cfg["seqlens"][0]
+    pairs = sum(s * (s + 1) // 2 for s in cfg["seqlens"])
+    sel_pairs = sum(sum(min(cfg["k"], t + 1) for t in range(s)) for s in cfg["seqlens"])
+    idx_flops = pairs * 2 * cfg["H_I"] * cfg["d_I"]
+    mla_flops = sel_pairs * 2 * cfg["H"] * (576 + 512)
+    return L, idx_flops, mla_flops, sel_pairs
+
+
+def run_ours(args, world, rank, local):
+    import sparse_attention_09_b200 as dsa
+
+    peaks, peak_src = load_peaks()
+    cfg = dict(synth.WORKLOADS[PREFILL])
+    cfg["seed"] = cfg["seed"] + rank
+    k, sm = cfg["k"], 1.0 / math.sqrt(576)
+    inp = synth.prefill_inputs(device="cuda", **cfg)
+    T = inp["q"].shape[0]
+    H = cfg["H"]
+    keys = dsa.contiguous_desc(inp["k8"], inp["cu_seqlens"], max(inp["seqlens"]), scale=inp["k_scale"])
+    lat = dsa.contiguous_desc(inp["latent"], inp["cu_seqlens"], max(inp["seqlens"]))
+    out = torch.empty((T, H, 512), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dsa.dsa_indexer_topk(inp["q8"], inp["q_scale"], inp["w"], keys, 1, cfg["H_I"], cfg["d_I"], k, idx)
+        if ev is not None:
+            ev[1].record(stream)
+        dsa.dsa_sparse_mla_prefill(inp["q"], lat, idx, 1, H, k, sm, out)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert dsa.dsa_device_error() == 0, "device error during warm-up"
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    idx_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    mla_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    err = dsa.dsa_device_error()
+    assert err == 0, f"device error {err}"
+    total_ms = max_over_ranks(total_ms, world)
+    ms_per_step = total_ms / args.steps
+    L, idx_flops, mla_flops, sel_pairs = prefill_work(cfg)
+    value = world * T / (ms_per_step * 1e-3)
+
+    fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]     # nominal fp8/bf16 ratio 2 (4.5 / 2.25 PF)
+    bf16_peak = peaks["bf16_tflops_sustained"]
+    kernels = {
+        "indexer_topk": {"ms": idx_ms, "tflops": idx_flops / (idx_ms * 1e-3) / 1e12, "peak_tflops": fp8_peak,
+                         "dtype": "e4m3", "flops": idx_flops},
+        "sparse_mla": {"ms": mla_ms, "tflops": mla_flops / (mla_ms * 1e-3) / 1e12, "peak_tflops": bf16_peak,
+                       "dtype": "bf16", "flops": mla_flops,
+                       "gather_gbs": sel_pairs * 1152 / (mla_ms * 1e-3) / 1e9},
+    }
+    for kk in kernels.values():
+        kk["frac"] = kk["tflops"] / kk["peak_tflops"]
+    dom = max(kernels, key=lambda n: kernels[n]["ms"])
+    dk = kernels[dom]
+    traffic = profile_traffic(dom)
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": dk["tflops"], "peak": dk["peak_tflops"],
+                "unit": "TFLOP/s", "frac": dk["frac"], "traffic": traffic,
+                "peak_source": f"{peak_src} (bf16 sustained x{'2 for e4m3' if dom == 'indexer_topk' else '1'})"}
+
+    # ---- decode chain, same process ----
+    decode = run_decode(args, dsa, sm) if rank == 0 else None
+
+    # ---- end to end through dsa_forward with host buffers ----
+    e2e = run_e2e(args, dsa, inp, cfg, sm) if (rank == 0 and not args.no_e2e) else None
+
+    # ---- oracle on a bounded sample ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = synth.sample_rows(L, k, args.cpu_rows, seed=3)
+        secs = oracle_prefill_sample(inp, k, rows, sm)
+        cpu = {"value": len(rows) / secs, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{len(rows)} query rows of the L=131072 prefill (full causal prefix each: indexer, "
+                         f"top-k, attention), {secs:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
+            "config": {"workload": f"{PREFILL}: DSA prefill, batch 1 per GPU, L=131072, top-k 2048, 64 e4m3 "
+                                   "indexer heads d_I=128, 128-head MLA-MQA (576 qk / 512 v), bf16, 5% planted keys",
+                       "global_batch": world, "seq_len": L, "k": k, "parallelism": f"independent problems x{world}",
+                       "l2": "inputs (~40 GB/step) larger than L2; no flush"},
+            "roofline": roofline, "kernels": kernels, "decode": decode, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clk, "gpu_launches": 2 * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_decode(args, dsa, sm):
+    cfg = dict(synth.WORKLOADS[DECODE])
+    d = synth.decode_inputs(device="cuda", **cfg)
+    B, k = d["B"], cfg["k"]
+    keys = dsa.paged_desc(d["kcache8"], d["block_table"], d["ctx"], d["max_ctx"], scale=d["kscale_cache"])
+    lat = dsa.paged_desc(d["latent_cache"], d["block_table"], d["ctx"], d["max_ctx"])
+    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, 64, k), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty((B, 128, 512), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        dsa.dsa_forward(dsa.DSA_MODE_DECODE, d["q8"], d["q_scale"], d["w"], keys, d["q"], lat, B, 64, 128, 128, k, sm,
+                        out, None, None, ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    n = max(10, args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    assert dsa.dsa_device_error() == 0
+    ms = e0.elapsed_time(e1) / n
+    keys_scanned = int(sum(d["ctx_host"]))
+    return {"workload": f"{DECODE}: 64 sequences, ctx ~ U[8192,131072] (sum {keys_scanned}), paged 64-token blocks",
+            "value": B / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": n,
+            "indexer_key_bytes": keys_scanned * 132, "indexer_gbs_equiv": keys_scanned * 132 / (ms * 1e-3) / 1e9,
+            "gpu_launches_per_step": 4}
+
+
+def run_e2e(args, dsa, inp, cfg, sm):
+    """dsa_forward with inputs copied from pinned host memory and the output copied back, every step."""
+    names = ["q8", "q_scale", "w", "k8", "k_scale", "q", "latent", "cu_seqlens"]
+    host = {}
+    for n in names:
+        t = inp[n]
+        try:
+            h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        except RuntimeError:
+            h = torch.empty(t.shape, dtype=t.dtype)
+        h.copy_(t)
+        host[n] = h
+    dev = {n: torch.empty_like(inp[n]) for n in names}
+    T, H, k = inp["q"].shape[0], cfg["H"], cfg["k"]
+    out = torch.empty((T, H, 512), dtype=torch.bfloat16, device="cuda")
+    try:
+        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    except RuntimeError:
+        out_h = torch.empty(out.shape, dtype=out.dtype)
+    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_PREFILL, 1, T, T, H, cfg["H_I"], k), dtype=torch.uint8,
+                     device="cuda")
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = out.numel() * out.element_size()
+
+    def step():
+        for n in names:
+            dev[n].copy_(host[n], non_blocking=True)
+        keys = dsa.contiguous_desc(dev["k8"], dev["cu_seqlens"], T, scale=dev["k_scale"])
+        lat = dsa.contiguous_desc(dev["latent"], dev["cu_seqlens"], T)
+        dsa.dsa_forward(dsa.DSA_MODE_PREFILL, dev["q8"], dev["q_scale"], dev["w"], keys, dev["q"], lat, 1, cfg["H_I"],
+                        cfg["d_I"], H, k, sm, out, None, None, ws)
+        out_h.copy_(out, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, args.e2e_steps))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    assert dsa.dsa_device_error() == 0
+    ms = e0.elapsed_time(e1) / n
+    return {"value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": n,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "pinned": bool(host["q"].is_pinned())}
+
+
+# ------------------------------------------------------------------------------------------
+# reference arm: the oracle, on the host cores
+# ------------------------------------------------------------------------------------------
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    cfg = dict(synth.WORKLOADS[PREFILL])
+    k, sm = cfg["k"], 1.0 / math.sqrt(576)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = synth.prefill_inputs(device=dev, **cfg)
+    L = cfg["seqlens"][0]
+    per_step = args.ref_rows
+    rs = np.random.default_rng(0)
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = sorted(rs.choice(L, size=per_step, replace=False).tolist())
+        secs = oracle_prefill_sample(inp, k, rows, sm)
+        if i >= args.warmup:
+            times.append(secs)
+    ms = 1e3 * float(np.mean(times))
+    value = per_step / (ms * 1e-3)
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{PREFILL}: DSA prefill, L=131072, top-k 2048 (oracle on {per_step} sampled "
+                                   "query rows per step)", "seq_len": L, "k": k},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{per_step} random query rows per step of the L=131072 prefill"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--ref-rows", type=int, default=2)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("warm-up raised to the minimum of 3 steps")
+        args.warmup = 3
+    if args.impl == "reference":  # rank 0 runs the oracle; other ranks exit without work
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup(args)
+    run_ours(args, world, rank, local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
