@@ -140,6 +140,26 @@ dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const
                                  float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Same as dsa_sparse_mla_decode, but it allocates nothing and takes no workspace: the split
+ * partial results live in a scratch array that the library itself holds in device memory
+ * (DSA_NOALLOC_SCRATCH_BYTES per GPU that loads the library, kept until the process exits).
+ * This entry point has no counterpart in the method's description; it exists for callers that
+ * cannot allocate device memory on the call path, for example a serving engine that hands
+ * all device memory to its own pool at start-up, or a latency-critical loop that cannot
+ * afford cudaMalloc's implicit device-wide synchronisation.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array, which keeps the last call's contents: calls
+ *     whose kernels overlap on the GPU (different streams, no ordering) race with each other.
+ *   - Sizes whose partial results do not fit (B * H * splits * 2056 bytes, splits = min(4, k/64))
+ *     return DSA_ERR_UNSUPPORTED before any launch.
+ */
+#define DSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B,
+                                         int32_t H, int32_t k, float sm_scale, void* out, float* lse,
+                                         void* stream);
+
+/*
  * Whole DSA forward.
  *   DSA_MODE_PREFILL: indexer and top-k run fused (no score matrix is written to HBM), then
  *     sparse MLA.  keys/latent contiguous with the same cu_seqlens; q_fp8 [T, H_I, d_I], etc.

@@ -32,7 +32,8 @@ DSA_MODE_PREFILL = 0
 DSA_MODE_DECODE = 1
 
 EXPORTED = ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_mla_prefill", "dsa_sparse_mla_decode",
-            "dsa_forward", "dsa_workspace_size", "dsa_status_string", "dsa_device_error")
+            "dsa_forward", "dsa_workspace_size", "dsa_status_string", "dsa_device_error",
+            "dsa_sparse_mla_decode_noalloc")
 
 
 class KVDesc(ctypes.Structure):
@@ -75,6 +76,8 @@ _lib.dsa_forward.argtypes = [_I32, _P, _P, _P, _DESC, _P, _DESC, _I32, _I32, _I3
 _lib.dsa_forward.restype = _I32
 _lib.dsa_indexer_topk.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I32, _P, _P]
 _lib.dsa_indexer_topk.restype = _I32
+_lib.dsa_sparse_mla_decode_noalloc.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P]
+_lib.dsa_sparse_mla_decode_noalloc.restype = _I32
 _lib.dsa_workspace_size.argtypes = [_I32, _I32, _I64, _I32, _I32, _I32, _I32]
 _lib.dsa_workspace_size.restype = _SZ
 
@@ -189,3 +192,12 @@ def dsa_indexer_topk(q_fp8, q_scale, w, keys: Desc, B, H_I, d_I, k, idx_out, str
     _check(_lib.dsa_indexer_topk(_ptr(q_fp8), _ptr(q_scale), _ptr(w), keys.ref(), int(B), int(H_I), int(d_I), int(k),
                                  _ptr(idx_out), _stream(stream)), "dsa_indexer_topk")
     return idx_out
+
+
+def dsa_sparse_mla_decode_noalloc(q, latent: Desc, idx, B, H, k, sm_scale, out, lse=None, stream=None):
+    """Decode sparse MLA that allocates nothing: partial results go to the library's own
+    per-device scratch array.  Calls that overlap on the GPU share that array and race."""
+    _check(_lib.dsa_sparse_mla_decode_noalloc(_ptr(q), latent.ref(), _ptr(idx), int(B), int(H), int(k),
+                                              float(sm_scale), _ptr(out), _ptr(lse), _stream(stream)),
+           "dsa_sparse_mla_decode_noalloc")
+    return out

@@ -171,6 +171,29 @@ dsa_status launch_mla(const CUtensorMap& m128, const CUtensorMap& m64, const Mla
 
 bool mla_shape_ok(int H, int k) { return H >= 1 && H <= 128 && k >= 64 && k <= 2048 && k % 64 == 0; }
 
+// ---- decode with library-held scratch (no allocation on the call path) ---------------------
+// One array per device, in this translation unit.  Host code cannot pass the symbol itself to
+// a kernel (on the host it is only a stand-in), so each device's address is looked up once,
+// with that device current, and cached.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[DSA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 256;
+
+dsa_status noalloc_scratch(void** ptr) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return DSA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return DSA_OK;
+}
+
 }  // namespace
 }  // namespace dsa
 
@@ -334,6 +357,18 @@ dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const
   if (st != DSA_OK) return st;
   mla_combine_kernel<<<dim3(H, B), 128, 0, s>>>(p.part_o, p.part_ml, splits, H, static_cast<__nv_bfloat16*>(out), lse);
   return launch_status();
+}
+
+dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B,
+                                         int32_t H, int32_t k, float sm_scale, void* out, float* lse, void* stream) {
+  if (B <= 0) return DSA_ERR_INVALID_ARGUMENT;
+  if (!mla_shape_ok(H, k)) return DSA_ERR_UNSUPPORTED;
+  if (decode_partials_bytes(B, H, decode_splits(k)) > DSA_NOALLOC_SCRATCH_BYTES) return DSA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  const dsa_status st = noalloc_scratch(&scratch);
+  if (st != DSA_OK) return st;
+  return dsa_sparse_mla_decode(q, latent, idx, B, H, k, sm_scale, out, lse, scratch, DSA_NOALLOC_SCRATCH_BYTES,
+                               stream);
 }
 
 dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale, const float* w,
