@@ -150,22 +150,14 @@ size_t decode_partials_bytes(int B, int H, int splits) {
 
 int decode_splits(int k) { return k / 64 < kDecodeSplits ? k / 64 : kDecodeSplits; }
 
-bool make_latent_maps(const void* data, uint64_t rows, CUtensorMap* m128, CUtensorMap* m64) {
-  return make_map_2d(m128, data, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kLatentDim, rows, kLatentDim * 2, 64, 1,
-                     CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_map_2d(m64, data, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kLatentDim, rows, kLatentDim * 2, 32, 1,
-                     CU_TENSOR_MAP_SWIZZLE_64B);
-}
-
 template <bool DECODE>
-dsa_status launch_mla(const CUtensorMap& m128, const CUtensorMap& m64, const MlaParams& p, int64_t units,
-                      cudaStream_t s) {
+dsa_status launch_mla(const void* latent, const MlaParams& p, int64_t units, cudaStream_t s) {
   auto kern = sparse_mla_kernel<DECODE>;
   const int smem = mla::kSmemBytes + 1024;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return DSA_ERR_CUDA;
   const int clusters = static_cast<int>(units < kMlaClusters ? units : kMlaClusters);
-  kern<<<2 * clusters, 192, smem, s>>>(m128, m64, p);
+  kern<<<2 * clusters, mla::kThreads, smem, s>>>(static_cast<const __nv_bfloat16*>(latent), p);
   return launch_status();
 }
 
@@ -298,9 +290,6 @@ dsa_status dsa_sparse_mla_prefill(const void* q, const dsa_kv_desc* latent, cons
     return DSA_ERR_INVALID_ARGUMENT;
   if (!mla_shape_ok(H, k)) return DSA_ERR_UNSUPPORTED;
   if (latent->total_tokens > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
-  CUtensorMap m128, m64;
-  if (!make_latent_maps(latent->data, static_cast<uint64_t>(latent->total_tokens), &m128, &m64))
-    return DSA_ERR_INVALID_ARGUMENT;
   MlaParams p;
   std::memset(&p, 0, sizeof(p));
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -314,7 +303,7 @@ dsa_status dsa_sparse_mla_prefill(const void* q, const dsa_kv_desc* latent, cons
   p.scale_log2 = sm_scale * 1.4426950408889634f;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  return launch_mla<false>(m128, m64, p, p.rows, as_stream(stream));
+  return launch_mla<false>(latent->data, p, p.rows, as_stream(stream));
 }
 
 dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B, int32_t H,
@@ -333,9 +322,6 @@ dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const
   const int splits = decode_splits(k);
   if (workspace == nullptr || ws_bytes < decode_partials_bytes(B, H, splits) || !aligned(workspace, 256))
     return workspace == nullptr ? DSA_ERR_INVALID_ARGUMENT : DSA_ERR_WORKSPACE_TOO_SMALL;
-  CUtensorMap m128, m64;
-  if (!make_latent_maps(latent->data, static_cast<uint64_t>(latent->num_blocks) * 64, &m128, &m64))
-    return DSA_ERR_INVALID_ARGUMENT;
   MlaParams p;
   std::memset(&p, 0, sizeof(p));
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -353,7 +339,7 @@ dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const
   p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                        align256(static_cast<size_t>(B) * splits * H * kValueDim * 4));
   cudaStream_t s = as_stream(stream);
-  dsa_status st = launch_mla<true>(m128, m64, p, static_cast<int64_t>(B) * splits, s);
+  dsa_status st = launch_mla<true>(latent->data, p, static_cast<int64_t>(B) * splits, s);
   if (st != DSA_OK) return st;
   mla_combine_kernel<<<dim3(H, B), 128, 0, s>>>(p.part_o, p.part_ml, splits, H, static_cast<__nv_bfloat16*>(out), lse);
   return launch_status();

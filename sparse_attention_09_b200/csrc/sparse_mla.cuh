@@ -21,10 +21,18 @@
 // exceeds its reference by more than 2^8 (then O_r and the row sum are rescaled); both ranks
 // see the same (m_0, m_1) and take the same decisions.
 //
-// Per CTA: warps 0-3 softmax/epilogue (thread h = head h = TMEM lane h), warp 4 TMA gather
-// producer, warp 5 MMA issuer and TMEM owner.  TMEM columns: O_r [0,256), Q_r [256,400),
-// S_r [400,464), P [464,496).  SMEM: a 4-stage ring of gathered chunks (64 rows x 576 B) and
-// a double-buffered exchange area written by the peer.
+// The row sums of P come from the tensor cores too: one more small MMA multiplies P by a tile
+// of ones into 16 extra accumulator columns, so they are rescaled together with O_r.
+//
+// Per CTA: warps 0-3 softmax/epilogue (thread h = head h = TMEM lane h), warps 4-7 gather
+// producers, warp 8 MMA issuer and TMEM owner.  The gather uses per-thread cp.async rather
+// than TMA gather4: on B200 one gather4 instruction costs 65-130 cycles of the TMA engine, far
+// too slow for 64 rows x 576 bytes per 64-key chunk, while a warp-wide cp.async moves one
+// row's 512-byte nope segment in a single coalesced instruction.  TMEM columns: O_r [0,256), Q_r [256,400),
+// S_r [400,464), P [464,496), row sums [496,512).  SMEM: a 4-stage ring of gathered chunks
+// (64 rows x 576 B), a double-buffered exchange area written by the peer, the ones tile.
+// The softmax warps run one chunk ahead: they compute and send their factor of chunk c+1
+// before they wait for the peer's factor of chunk c, which hides the exchange latency.
 //
 // The same kernel serves decode: a work item is then (sequence, split of its selection) over
 // a paged latent cache, and the unnormalised partial result (O, M, l) goes to a workspace
@@ -64,9 +72,11 @@ constexpr int kRopeBlockBytes = kChunk * 64;       // 64 rows x 32 dims bf16, 64
 constexpr int kStageBytes = 4 * kNopeBlockBytes + kRopeBlockBytes;  // 36864
 constexpr int kXRowBytes = 144;                    // exchange row: 64 bf16 + m + pad
 constexpr int kXBufBytes = 128 * kXRowBytes;
-constexpr int kSmemBytes = kStages * kStageBytes + 2 * kXBufBytes;
-constexpr uint32_t kColO = 0, kColQ = 256, kColS = 400, kColP = 464;
+constexpr int kOnesBytes = 16 * 128;               // B tile of ones for the row sums
+constexpr int kSmemBytes = kStages * kStageBytes + 4 * kXBufBytes + kOnesBytes;
+constexpr uint32_t kColO = 0, kColQ = 256, kColS = 400, kColP = 464, kColL = 496;
 constexpr float kTau = 8.f;                        // lazy-rescale margin (log2 units)
+constexpr uint32_t kXBytesPerChunk = kXBufBytes;  // one bulk copy of the whole row block per chunk
 
 __device__ __forceinline__ void sm_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
@@ -79,6 +89,17 @@ __device__ __forceinline__ bool sm_any(bool v) {
       : "r"(static_cast<uint32_t>(v))
       : "memory");
   return r != 0;
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
 }
 
 // Number of 64-entry chunks up to the last valid (>= 0) index of a selection row, computed by
@@ -94,24 +115,30 @@ __device__ __forceinline__ int active_chunks(const int32_t* row, int k) {
 
 }  // namespace mla
 
+namespace mla {
+constexpr int kThreads = 9 * 32;  // 4 softmax + 4 producer + 1 MMA warps
+}  // namespace mla
+
 template <bool DECODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap lat128, const __grid_constant__ CUtensorMap lat64,
-                      const MlaParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
+    sparse_mla_kernel(const __nv_bfloat16* __restrict__ latent, const MlaParams p) {
   using namespace dev;
   using namespace mla;
   constexpr uint32_t IDESC_QK = idesc_bf16(128, kChunk, false, false);
   constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, false, true);
+  constexpr uint32_t IDESC_L = idesc_bf16(128, 16, false, false);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sKV = smem;                                     // [kStages][kStageBytes]
   uint8_t* sX = smem + kStages * kStageBytes;              // [2][128][kXRowBytes], written by the peer
+  uint8_t* sXout = sX + 2 * kXBufBytes;                    // [2][128][kXRowBytes], staged for the peer
+  uint8_t* sOnes = sXout + 2 * kXBufBytes;                 // [16][64] bf16 ones (K-major, 1024-aligned)
 
   __shared__ uint64_t bar_kvfull[kStages], bar_kvempty[kStages];
   __shared__ uint64_t bar_qfull, bar_sfull, bar_sfree, bar_pfull, bar_pvdone, bar_ofree;
   __shared__ uint64_t bar_xfull[2], bar_xempty[2];
-  __shared__ uint64_t s_vmask[kStages];                    // valid rows of each staged chunk
+  __shared__ uint64_t s_vmask[kStages];                    // valid rows of each staged chunk (16 bits per producer warp)
   __shared__ uint32_t s_tmem;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -121,7 +148,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&bar_kvfull[i], 1);
+      mbar_init(&bar_kvfull[i], 128);  // every producer thread, once its copies landed
       mbar_init(&bar_kvempty[i], 1);
     }
     mbar_init(&bar_qfull, 128);
@@ -131,15 +158,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     mbar_init(&bar_pvdone, 1);
     mbar_init(&bar_ofree, 4);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar_xfull[i], 128);   // 128 remote arrivals from the peer's softmax threads
-      mbar_init(&bar_xempty[i], 128);
+      mbar_init(&bar_xfull[i], 1);     // own arm (expect_tx) + the peer's asynchronous stores
+      mbar_init(&bar_xempty[i], 1);    // one remote arrival: the peer has read this CTA's row block
     }
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 8) {
     tmem_alloc(&s_tmem, 512);
     tmem_relinquish();
   }
+  if (tid < kOnesBytes / 16)  // bf16 1.0 everywhere: invariant under the 128-byte swizzle
+    *reinterpret_cast<uint4*>(sOnes + 16 * tid) = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // barriers of both CTAs are initialised before any remote arrival
@@ -181,10 +211,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     if (c1 <= c0) c1 = c0 + 1;  // always at least one chunk (all masked if empty)
   };
 
-  if (warp == 4) {
-    // ================= gather producer =================
+  if (warp >= 4 && warp < 8) {
+    // ================= gather producers (warps 4-7) =================
+    // Warp pw copies keys [16 pw, 16 pw + 16) of each 64-key chunk: one warp instruction per key
+    // for its 512-byte nope segment (lane l -> 16-byte chunk l, written at its 128-byte-swizzle
+    // position), two more for the 64-byte rope halves of the 16 keys (64-byte swizzle).  A
+    // stage is announced on its barrier one chunk later, after cp.async.wait_group has seen its
+    // copies land and a proxy fence has made them visible to the tensor cores.
+    const int pw = warp - 4;
     uint32_t g = 0;
     bool ok = true;
+    int pending_stage = -1;
+    auto announce = [&](int st) {
+      fence_proxy_async_smem();
+      mbar_arrive(&bar_kvfull[st]);
+    };
     for (int64_t u = cid; ok && u < nunits; u += ncl) {
       int64_t qrow;
       int kbeg, kend, seq, seq_start, seq_len, c0, c1;
@@ -194,110 +235,148 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       const int32_t* bt = DECODE ? p.block_table + static_cast<int64_t>(seq) * p.max_blocks_per_seq : nullptr;
       for (int c = c0; c < c1; ++c, ++g) {
         const int stage = static_cast<int>(g % kStages);
-        const uint32_t ph = (g / kStages) & 1u;
-        if (!mbar_wait(&bar_kvempty[stage], ph ^ 1u)) {
+        if (!mbar_wait(&bar_kvempty[stage], ((g / kStages) & 1u) ^ 1u)) {
           record_device_error(DSA_ERR_TIMEOUT);
           ok = false;
           break;
         }
-        // lanes 0..15 each gather 4 rows
-        int4 ix = make_int4(-1, -1, -1, -1);
-        if (lane < 16) ix = *reinterpret_cast<const int4*>(row + c * kChunk + 4 * lane);
-        int v[4] = {ix.x, ix.y, ix.z, ix.w};
-        uint32_t valid4 = 0;
-        int phys[4];
+        const int v = lane < 16 ? row[c * kChunk + 16 * pw + lane] : -1;
+        const bool valid = lane < 16 && v >= 0 && v < seq_len;
+        const int pos = valid ? v : 0;  // masked rows still copy a real row (never NaN bits)
+        int prow;
+        if constexpr (DECODE) prow = bt[pos >> 6] * 64 + (pos & 63);
+        else prow = seq_start + pos;
+        const uint32_t vbits = __ballot_sync(0xffffffffu, valid) & 0xFFFFu;
+        if (lane == 0) reinterpret_cast<uint16_t*>(&s_vmask[stage])[pw] = static_cast<uint16_t>(vbits);
+        const uint32_t st = smem_addr(sKV + stage * kStageBytes);
+#pragma unroll 4
+        for (int j = 0; j < 16; ++j) {  // nope: 32 lanes x 16 bytes of one key
+          const int r = 16 * pw + j;
+          const int kr = __shfl_sync(0xffffffffu, prow, j);
+          const __nv_bfloat16* src = latent + static_cast<int64_t>(kr) * 576 + 256 * rank + 8 * lane;
+          const int blk = lane >> 3, ch = lane & 7;
+          cp_async16(st + blk * kNopeBlockBytes + r * 128 + ((ch ^ (r & 7)) << 4), src);
+        }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const bool okj = lane < 16 && v[j] >= 0 && v[j] < seq_len;
-          valid4 |= okj ? (1u << j) : 0u;
-          const int pos = okj ? v[j] : 0;
-          if constexpr (DECODE) phys[j] = bt[pos >> 6] * 64 + (pos & 63);
-          else phys[j] = seq_start + pos;
+        for (int h2 = 0; h2 < 2; ++h2) {  // rope: 8 keys x 4 chunks of 16 bytes per instruction
+          const int j = 8 * h2 + (lane >> 2), ch = lane & 3;
+          const int r = 16 * pw + j;
+          const int kr = __shfl_sync(0xffffffffu, prow, j);
+          const __nv_bfloat16* src = latent + static_cast<int64_t>(kr) * 576 + 512 + 32 * rank + 8 * ch;
+          cp_async16(st + 4 * kNopeBlockBytes + r * 64 + ((ch ^ ((r >> 1) & 3)) << 4), src);
         }
-        // 64-bit validity mask of the chunk: lane l contributes bits 4l..4l+3
-        uint64_t mask = static_cast<uint64_t>(valid4) << (4 * (lane & 15));
-        mask |= __shfl_xor_sync(0xffffffffu, mask, 1);
-        mask |= __shfl_xor_sync(0xffffffffu, mask, 2);
-        mask |= __shfl_xor_sync(0xffffffffu, mask, 4);
-        mask |= __shfl_xor_sync(0xffffffffu, mask, 8);
-        if (lane == 0) {
-          s_vmask[stage] = mask;
-          mbar_arrive_expect_tx(&bar_kvfull[stage], kStageBytes);
+        cp_async_commit();
+        if (pending_stage >= 0) {
+          cp_async_wait<1>();
+          announce(pending_stage);
         }
-        __syncwarp();
-        if (lane < 16) {
-          uint8_t* st = sKV + stage * kStageBytes;
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tma_gather4(st + j * kNopeBlockBytes + lane * 512, &lat128, &bar_kvfull[stage],
-                        static_cast<int32_t>(256 * rank + 64 * j), phys[0], phys[1], phys[2], phys[3]);
-          tma_gather4(st + 4 * kNopeBlockBytes + lane * 256, &lat64, &bar_kvfull[stage],
-                      static_cast<int32_t>(512 + 32 * rank), phys[0], phys[1], phys[2], phys[3]);
-        }
-        __syncwarp();
+        pending_stage = stage;
       }
     }
-  } else if (warp == 5) {
+    if (pending_stage >= 0) {
+      cp_async_wait<0>();
+      announce(pending_stage);
+    }
+  } else if (warp == 8) {
     // ================= MMA issuer =================
-    uint32_t g = 0, tok = 0;
-    bool ok = true;
-    int64_t pend = -1;           // chunk whose P.V is still to be issued
-    bool pend_first = false;     // ... and whether it starts its unit
-    uint32_t pend_tok = 0;
-    auto issue_pv = [&]() -> bool {
-      const uint32_t x = static_cast<uint32_t>(pend);
-      if (!mbar_wait(&bar_pfull, x & 1u)) return false;
-      if (pend_first && pend_tok > 0 && !mbar_wait(&bar_ofree, (pend_tok - 1) & 1u)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t st = smem_addr(sKV + (x % kStages) * kStageBytes);
-#pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk)
-          umma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, make_smem_desc(st + kk * 2048, 8192, 1024, kSwizzle128B),
-                       IDESC_PV, (pend_first && kk == 0) ? 0u : 1u);
-        umma_commit(&bar_pvdone);
-        umma_commit(&bar_kvempty[x % kStages]);
-      }
-      __syncwarp();
-      return true;
+    // Two cursors walk the same chunk sequence: Q.K^T of a chunk is issued as soon as its keys
+    // are staged and the single S buffer has been read, P.V as soon as P is ready, so the
+    // tensor core computes the logits of the next chunk while the softmax warps work.
+    struct Cursor {
+      int64_t u;
+      int c, c0, c1;
+      uint32_t g, tok;
+      bool valid;
     };
-    for (int64_t u = cid; ok && u < nunits; u += ncl, ++tok) {
+    auto enter_unit = [&](Cursor& cu) {
+      cu.valid = cu.u < nunits;
+      if (!cu.valid) return;
       int64_t qrow;
-      int kbeg, kend, seq, seq_start, seq_len, c0, c1;
-      unit_info(u, qrow, kbeg, kend, seq, seq_start, seq_len);
-      unit_chunks(qrow, kbeg, kend, c0, c1);
-      for (int c = c0; c < c1; ++c, ++g) {
-        const int stage = static_cast<int>(g % kStages);
-        if (!mbar_wait(&bar_kvfull[stage], (g / kStages) & 1u) || (c == c0 && !mbar_wait(&bar_qfull, tok & 1u)) ||
-            (g > 0 && !mbar_wait(&bar_sfree, (g - 1) & 1u))) {
+      int kbeg, kend, seq, seq_start, seq_len;
+      unit_info(cu.u, qrow, kbeg, kend, seq, seq_start, seq_len);
+      unit_chunks(qrow, kbeg, kend, cu.c0, cu.c1);
+      cu.c = cu.c0;
+    };
+    auto advance = [&](Cursor& cu) {
+      ++cu.g;
+      if (++cu.c >= cu.c1) {
+        cu.u += ncl;
+        ++cu.tok;
+        enter_unit(cu);
+      }
+    };
+    Cursor qk{cid, 0, 0, 0, 0, 0, false}, pv{cid, 0, 0, 0, 0, 0, false};
+    enter_unit(qk);
+    enter_unit(pv);
+    bool ok = true;
+    uint64_t idle_since = 0;
+    while (pv.valid) {
+      bool did = false;
+      if (qk.valid) {
+        const int stage = static_cast<int>(qk.g % kStages);
+        bool ready = mbar_poll(smem_addr(&bar_kvfull[stage]), (qk.g / kStages) & 1u) &&
+                     (qk.g == 0 || mbar_poll(smem_addr(&bar_sfree), (qk.g - 1) & 1u)) &&
+                     (qk.c != qk.c0 || mbar_poll(smem_addr(&bar_qfull), qk.tok & 1u));
+        ready = __shfl_sync(0xffffffffu, ready, 0);
+        if (ready) {
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t st = smem_addr(sKV + stage * kStageBytes);
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk)  // 256 nope dims: 4 blocks x 4 steps of 16
+              umma_bf16_ts(tmem + kColS, tmem + kColQ + kk * 8,
+                           make_smem_desc(st + (kk >> 2) * kNopeBlockBytes + (kk & 3) * 32, 16, 1024, kSwizzle128B),
+                           IDESC_QK, kk > 0 ? 1u : 0u);
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)   // 32 rope dims
+              umma_bf16_ts(tmem + kColS, tmem + kColQ + (16 + kk) * 8,
+                           make_smem_desc(st + 4 * kNopeBlockBytes + kk * 32, 16, 512, kSwizzle64B), IDESC_QK, 1u);
+            umma_commit(&bar_sfull);
+          }
+          __syncwarp();
+          advance(qk);
+          did = true;
+        }
+      }
+      if (pv.g < qk.g) {
+        const bool first = pv.c == pv.c0;
+        bool ready = mbar_poll(smem_addr(&bar_pfull), pv.g & 1u) &&
+                     (!first || pv.tok == 0 || mbar_poll(smem_addr(&bar_ofree), (pv.tok - 1) & 1u));
+        ready = __shfl_sync(0xffffffffu, ready, 0);
+        if (ready) {
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t st = smem_addr(sKV + (pv.g % kStages) * kStageBytes);
+#pragma unroll
+            for (int kk = 0; kk < kChunk / 16; ++kk)
+              umma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8,
+                           make_smem_desc(st + kk * 2048, 8192, 1024, kSwizzle128B), IDESC_PV,
+                           (first && kk == 0) ? 0u : 1u);
+            const uint32_t ones = smem_addr(sOnes);
+#pragma unroll
+            for (int kk = 0; kk < kChunk / 16; ++kk)  // row sums of P
+              umma_bf16_ts(tmem + kColL, tmem + kColP + kk * 8,
+                           make_smem_desc(ones + kk * 32, 16, 1024, kSwizzle128B), IDESC_L,
+                           (first && kk == 0) ? 0u : 1u);
+            umma_commit(&bar_pvdone);
+            umma_commit(&bar_kvempty[pv.g % kStages]);
+          }
+          __syncwarp();
+          advance(pv);
+          did = true;
+        }
+      }
+      if (did) {
+        idle_since = 0;
+      } else {
+        const uint64_t now = global_timer_ns();
+        if (idle_since == 0) idle_since = now;
+        else if (now - idle_since > kWaitLimitNs) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t st = smem_addr(sKV + stage * kStageBytes);
-#pragma unroll
-          for (int kk = 0; kk < 16; ++kk)  // 256 nope dims: 4 blocks x 4 steps of 16
-            umma_bf16_ts(tmem + kColS, tmem + kColQ + kk * 8,
-                         make_smem_desc(st + (kk >> 2) * kNopeBlockBytes + (kk & 3) * 32, 16, 1024, kSwizzle128B),
-                         IDESC_QK, kk > 0 ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)   // 32 rope dims
-            umma_bf16_ts(tmem + kColS, tmem + kColQ + (16 + kk) * 8,
-                         make_smem_desc(st + 4 * kNopeBlockBytes + kk * 32, 16, 512, kSwizzle64B), IDESC_QK, 1u);
-          umma_commit(&bar_sfull);
-        }
-        __syncwarp();
-        if (pend >= 0 && !issue_pv()) {
-          ok = false;
-          break;
-        }
-        pend = g;
-        pend_first = c == c0;
-        pend_tok = tok;
       }
     }
-    if (ok && pend >= 0) ok = issue_pv();
     if (!ok && lane == 0) record_device_error(DSA_ERR_TIMEOUT);
   } else {
     // ================= softmax / exchange / epilogue (warps 0-3) =================
@@ -343,131 +422,154 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       unit_info(cid, qrow, kbeg, kend, seq, ss, sl);
       load_q(qrow);
     }
+    // Stage A of chunk gg: read the partial logits, form this rank's factor
+    // P_own = 2^(x*S_r - m_own) as bf16 and send it with m_own to the peer.
+    auto stage_a = [&](uint32_t gg, bool last_of_unit, int64_t next_unit, float& m_own, uint32_t(&pown)[32],
+                       float& m_sent) -> bool {
+      const int stage = static_cast<int>(gg % kStages);
+      bool ok = mbar_wait(&bar_sfull, gg & 1u);
+      if (sm_any(!ok)) return false;
+      tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld32(lane_base + kColS, *reinterpret_cast<uint32_t(*)[32]>(sr));
+      tmem_ld32(lane_base + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_sfree);
+      if (last_of_unit && next_unit < nunits) {  // the unit's last Q.K^T is done: stage the next Q
+        int64_t nq;
+        int a, bb, cc, dd, ee;
+        unit_info(next_unit, nq, a, bb, cc, dd, ee);
+        load_q(nq);
+      }
+      // the validity mask was written by the producer before it armed this stage's barrier
+      ok = mbar_wait(&bar_kvfull[stage], (gg / kStages) & 1u);
+      if (sm_any(!ok)) return false;
+      const uint64_t vmask = s_vmask[stage];
+      const bool full = vmask == ~0ull;
+      float smax = -INFINITY;
+      if (full) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) smax = fmaxf(smax, __uint_as_float(sr[i]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if ((vmask >> i) & 1ull) smax = fmaxf(smax, __uint_as_float(sr[i]));
+      }
+      const float cmax = smax * p.scale_log2;  // scale > 0
+      if (cmax > m_own + kTau || (m_own == -INFINITY && cmax > -INFINITY)) m_own = cmax;
+      const float neg_m = -m_own;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        float a = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), p.scale_log2, neg_m));
+        float bq = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), p.scale_log2, neg_m));
+        if (!full) {
+          a = ((vmask >> (2 * i)) & 1ull) ? a : 0.f;
+          bq = ((vmask >> (2 * i + 1)) & 1ull) ? bq : 0.f;
+        }
+        pown[i] = pack_bf16x2(a, bq);
+      }
+      // The peer has read the block of chunk gg-2 (so that copy, which read this staging
+      // buffer, is complete): stage this chunk's rows locally and let the TMA engine push the
+      // whole block to the peer, keeping the load/store path free.
+      const int xb = static_cast<int>(gg & 1u);
+      ok = mbar_wait_cluster(&bar_xempty[xb], ((gg >> 1) & 1u) ^ 1u);
+      if (sm_any(!ok)) return false;
+      uint8_t* row = sXout + xb * kXBufBytes + h * kXRowBytes;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<uint4*>(row + 16 * i) = make_uint4(pown[4 * i], pown[4 * i + 1], pown[4 * i + 2], pown[4 * i + 3]);
+      *reinterpret_cast<float*>(row + 128) = m_own;
+      fence_proxy_async_smem();
+      sm_sync();
+      if (tid == 0)
+        bulk_copy_to_peer(x_peer + xb * kXBufBytes, sXout + xb * kXBufBytes, kXBufBytes, xbar_full_peer[xb]);
+      m_sent = m_own;
+      return true;
+    };
+    // Stage B of chunk gg: receive the peer's factor, form P = P_own * P_peer relative to
+    // M = m_own + m_peer (identical in both ranks), rescale O_r and the row sums if M moved,
+    // and hand P to the tensor cores.
+    auto stage_b = [&](uint32_t gg, bool first_of_unit, const uint32_t(&pown)[32], float m_sent, float& M) -> bool {
+      const int xb = static_cast<int>(gg & 1u);
+      if (tid == 0) mbar_arrive_expect_tx(&bar_xfull[xb], kXBytesPerChunk);  // may land before or after the data
+      bool ok = mbar_wait_cluster(&bar_xfull[xb], (gg >> 1) & 1u);
+      if (sm_any(!ok)) return false;
+      const uint8_t* src = sX + xb * kXBufBytes + h * kXRowBytes;
+      uint32_t pp[32];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 w = *reinterpret_cast<const uint4*>(src + 16 * i);
+        pp[4 * i] = bf16x2_mul(pown[4 * i], w.x);
+        pp[4 * i + 1] = bf16x2_mul(pown[4 * i + 1], w.y);
+        pp[4 * i + 2] = bf16x2_mul(pown[4 * i + 2], w.z);
+        pp[4 * i + 3] = bf16x2_mul(pown[4 * i + 3], w.w);
+      }
+      const float m_peer = *reinterpret_cast<const float*>(src + 128);
+      const float Mn = m_sent + m_peer;
+      if (gg > 0) {  // the previous P.V must be done before P is overwritten or O rescaled
+        ok = mbar_wait(&bar_pvdone, (gg - 1) & 1u);
+        if (sm_any(!ok)) return false;
+        tc_fence_after();
+      } else {
+        sm_sync();
+      }
+      // every thread has read its row of the peer's block (the barrier above): release it.
+      // (Not thread 0: its cluster-scope release would also wait for the bulk copy it issued.)
+      if (tid == 32) mbar_arrive_remote(xbar_empty_peer[xb]);
+      // tcgen05.ld/st are warp-collective: the whole warp runs the rescale if any row needs it
+      const bool need_rescale = !first_of_unit && Mn != M && M > -INFINITY;
+      if (__any_sync(0xffffffffu, need_rescale)) {
+        const float alpha = need_rescale ? exp2f(M - Mn) : 1.f;
+#pragma unroll 1
+        for (int c32 = 0; c32 < 256; c32 += 32) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + kColO + c32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(lane_base + kColO + c32, o);
+        }
+        uint32_t lv[16];
+        tmem_ld16(lane_base + kColL, lv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) lv[i] = __float_as_uint(__uint_as_float(lv[i]) * alpha);
+        tmem_st16(lane_base + kColL, lv);
+      }
+      M = Mn;
+      tmem_st32(lane_base + kColP, pp);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_pfull);
+      return true;
+    };
+
     for (int64_t u = cid; u < nunits; u += ncl, ++tok) {
       int64_t qrow;
       int kbeg, kend, seq, seq_start, seq_len, c0, c1;
       unit_info(u, qrow, kbeg, kend, seq, seq_start, seq_len);
       unit_chunks(qrow, kbeg, kend, c0, c1);
-      float m_own = -INFINITY, m_peer = -INFINITY, M = -INFINITY, l = 0.f;
+      float m_own = -INFINITY, M = -INFINITY, m_cur = -INFINITY, m_next = -INFINITY;
+      uint32_t p_cur[32], p_next[32];
+      if (!stage_a(g, c0 == c1 - 1, u + ncl, m_own, p_cur, m_cur)) {
+        aborted = true;
+        break;
+      }
       for (int c = c0; c < c1; ++c, ++g) {
-        const int stage = static_cast<int>(g % kStages);
-        bool ok = mbar_wait(&bar_sfull, g & 1u);
-        if (sm_any(!ok)) {
+        if (c + 1 < c1 && !stage_a(g + 1, c + 1 == c1 - 1, u + ncl, m_own, p_next, m_next)) {
           aborted = true;
           break;
         }
-        tc_fence_after();
-        uint32_t sr[64];
-        tmem_ld32(lane_base + kColS, *reinterpret_cast<uint32_t(*)[32]>(sr));
-        tmem_ld32(lane_base + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_sfree);
-        if (c == c1 - 1 && u + ncl < nunits) {  // the last Q.K^T of this unit is done: stage the next Q
-          int64_t nq;
-          int a, bb, cc, dd, ee;
-          unit_info(u + ncl, nq, a, bb, cc, dd, ee);
-          load_q(nq);
-        }
-        // own partial logits (log2 units) and this chunk's maximum; the validity mask was
-        // written by the producer before it armed this stage's barrier, so acquire that
-        // barrier's (still current) phase before reading it
-        ok = mbar_wait(&bar_kvfull[stage], (g / kStages) & 1u);
-        if (sm_any(!ok)) {
+        if (!stage_b(g, c == c0, p_cur, m_cur, M)) {
           aborted = true;
           break;
         }
-        const uint64_t vmask = s_vmask[stage];
-        float cmax = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float xv = __uint_as_float(sr[i]) * p.scale_log2;
-          sr[i] = __float_as_uint(xv);
-          if ((vmask >> i) & 1ull) cmax = fmaxf(cmax, xv);
-        }
-        if (cmax > m_own + kTau || (m_own == -INFINITY && cmax > -INFINITY)) m_own = cmax;
-        uint32_t pown[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float a = ((vmask >> (2 * i)) & 1ull) ? exp2f(__uint_as_float(sr[2 * i]) - m_own) : 0.f;
-          const float bq = ((vmask >> (2 * i + 1)) & 1ull) ? exp2f(__uint_as_float(sr[2 * i + 1]) - m_own) : 0.f;
-          pown[i] = pack_bf16x2(a, bq);
-        }
-        // exchange with the peer: send my row, then read the peer's row of the same chunk
-        const int xb = static_cast<int>(g & 1u);
-        const uint32_t xuse = g >> 1;
-        ok = mbar_wait_cluster(&bar_xempty[xb], (xuse & 1u) ^ 1u);  // the peer has read my previous row
-        if (sm_any(!ok)) {
-          aborted = true;
-          break;
-        }
-        const uint32_t dst = x_peer + xb * kXBufBytes + h * kXRowBytes;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          st_cluster_v4(dst + 16 * i, pown[4 * i], pown[4 * i + 1], pown[4 * i + 2], pown[4 * i + 3]);
-        st_cluster_f32(dst + 128, m_own);
-        mbar_arrive_remote(xbar_full_peer[xb]);
-        ok = mbar_wait_cluster(&bar_xfull[xb], xuse & 1u);
-        if (sm_any(!ok)) {
-          aborted = true;
-          break;
-        }
-        const uint8_t* src = sX + xb * kXBufBytes + h * kXRowBytes;
-        uint32_t ppeer[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 w = *reinterpret_cast<const uint4*>(src + 16 * i);
-          ppeer[4 * i] = w.x;
-          ppeer[4 * i + 1] = w.y;
-          ppeer[4 * i + 2] = w.z;
-          ppeer[4 * i + 3] = w.w;
-        }
-        m_peer = *reinterpret_cast<const float*>(src + 128);
-        mbar_arrive_remote(xbar_empty_peer[xb]);
-        // P = P_own * P_peer relative to M = m_own + m_peer (identical in both ranks)
-        const float Mn = m_own + m_peer;
-        float psum = 0.f;
-        uint32_t pp[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 a = unpack_bf16x2(pown[i]), bq = unpack_bf16x2(ppeer[i]);
-          pp[i] = pack_bf16x2(a.x * bq.x, a.y * bq.y);
-          const float2 r = unpack_bf16x2(pp[i]);
-          psum += r.x + r.y;
-        }
-        // the previous chunk's P.V must be done before P is overwritten (and before O is rescaled)
-        if (g > 0) {
-          ok = mbar_wait(&bar_pvdone, (g - 1) & 1u);
-          if (sm_any(!ok)) {
-            aborted = true;
-            break;
-          }
-          tc_fence_after();
-        }
-        // Rescale O_r when M moved.  tcgen05.ld/st are warp-collective, so the whole warp runs
-        // the loop if any of its rows needs it (alpha = 1 for the others).
-        const bool need_rescale = c > c0 && Mn != M && M > -INFINITY;
-        if (__any_sync(0xffffffffu, need_rescale)) {
-          const float alpha = need_rescale ? exp2f(M - Mn) : 1.f;
-          l *= alpha;
-#pragma unroll 1
-          for (int c32 = 0; c32 < 256; c32 += 32) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + kColO + c32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(lane_base + kColO + c32, o);
-          }
-        }
-        M = Mn;
-        l += psum;
-        tmem_st32(lane_base + kColP, pp);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_pfull);
+        for (int i = 0; i < 32; ++i) p_cur[i] = p_next[i];
+        m_cur = m_next;
       }
       if (aborted) break;
       // epilogue of the unit: O_r / l
@@ -477,6 +579,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         break;
       }
       tc_fence_after();
+      uint32_t lv[16];
+      tmem_ld16(lane_base + kColL, lv);
+      tmem_wait_ld();
+      const float l = __uint_as_float(lv[0]);
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       if constexpr (!DECODE) {
         __nv_bfloat16* orow = p.out + (qrow * p.H + h) * 512 + 256 * rank;
@@ -527,7 +633,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // the peer no longer writes into this CTA's shared memory
-  if (warp == 5) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
