@@ -24,8 +24,8 @@
 // The row sums of P come from the tensor cores too: one more small MMA multiplies P by a tile
 // of ones into 16 extra accumulator columns, so they are rescaled together with O_r.
 //
-// Per CTA: warps 0-3 softmax/epilogue (thread h = head h = TMEM lane h), warps 4-7 gather
-// producers, warp 8 MMA issuer and TMEM owner.  The gather uses per-thread cp.async rather
+// Per CTA: warps 0-3 softmax/epilogue (thread h = head h = TMEM lane h), warps 4-5 gather
+// producers, warp 6 MMA issuer and TMEM owner.  The gather uses per-thread cp.async rather
 // than TMA gather4: on B200 one gather4 instruction costs 65-130 cycles of the TMA engine, far
 // too slow for 64 rows x 576 bytes per 64-key chunk, while a warp-wide cp.async moves one
 // row's 512-byte nope segment in a single coalesced instruction.  TMEM columns: O_r [0,256), Q_r [256,400),
@@ -116,7 +116,11 @@ __device__ __forceinline__ int active_chunks(const int32_t* row, int k) {
 }  // namespace mla
 
 namespace mla {
-constexpr int kThreads = 9 * 32;  // 4 softmax + 4 producer + 1 MMA warps
+// 4 softmax + 2 producer + 1 MMA warps.  At most 2 warps per SM sub-partition keeps the full
+// 255 registers per thread available (9 warps would put 3 on one and cap them at 168).
+constexpr int kThreads = 7 * 32;
+constexpr int kProducerWarps = 2;
+constexpr int kMmaWarp = 4 + kProducerWarps;
 }  // namespace mla
 
 template <bool DECODE>
@@ -138,7 +142,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
   __shared__ uint64_t bar_kvfull[kStages], bar_kvempty[kStages];
   __shared__ uint64_t bar_qfull, bar_sfull, bar_sfree, bar_pfull, bar_pvdone, bar_ofree;
   __shared__ uint64_t bar_xfull[2], bar_xempty[2];
-  __shared__ uint64_t s_vmask[kStages];                    // valid rows of each staged chunk (16 bits per producer warp)
+  __shared__ uint64_t s_vmask[kStages];                    // valid rows of each staged chunk (32 bits per producer warp)
   __shared__ uint32_t s_tmem;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -148,7 +152,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&bar_kvfull[i], 128);  // every producer thread, once its copies landed
+      mbar_init(&bar_kvfull[i], 32 * kProducerWarps);  // every producer thread (plus its copies in flight)
       mbar_init(&bar_kvempty[i], 1);
     }
     mbar_init(&bar_qfull, 128);
@@ -163,7 +167,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
     }
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&s_tmem, 512);
     tmem_relinquish();
   }
@@ -211,21 +215,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
     if (c1 <= c0) c1 = c0 + 1;  // always at least one chunk (all masked if empty)
   };
 
-  if (warp >= 4 && warp < 8) {
-    // ================= gather producers (warps 4-7) =================
-    // Warp pw copies keys [16 pw, 16 pw + 16) of each 64-key chunk: one warp instruction per key
+  if (warp >= 4 && warp < kMmaWarp) {
+    // ================= gather producers =================
+    // Warp pw copies keys [32 pw, 32 pw + 32) of each 64-key chunk: one warp instruction per key
     // for its 512-byte nope segment (lane l -> 16-byte chunk l, written at its 128-byte-swizzle
-    // position), two more for the 64-byte rope halves of the 16 keys (64-byte swizzle).  A
-    // stage is announced on its barrier one chunk later, after cp.async.wait_group has seen its
-    // copies land and a proxy fence has made them visible to the tensor cores.
+    // position), four more for the 64-byte rope halves of the 32 keys (64-byte swizzle).  The
+    // stage's barrier completes on its own once the copies have landed (an asynchronous
+    // arrival per thread); the MMA warp fences the proxies before the tensor cores read it.
     const int pw = warp - 4;
     uint32_t g = 0;
     bool ok = true;
-    int pending_stage = -1;
-    auto announce = [&](int st) {
-      fence_proxy_async_smem();
-      mbar_arrive(&bar_kvfull[st]);
-    };
     for (int64_t u = cid; ok && u < nunits; u += ncl) {
       int64_t qrow;
       int kbeg, kend, seq, seq_start, seq_len, c0, c1;
@@ -240,44 +239,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
           ok = false;
           break;
         }
-        const int v = lane < 16 ? row[c * kChunk + 16 * pw + lane] : -1;
-        const bool valid = lane < 16 && v >= 0 && v < seq_len;
+        const int v = row[c * kChunk + 32 * pw + lane];
+        const bool valid = v >= 0 && v < seq_len;
         const int pos = valid ? v : 0;  // masked rows still copy a real row (never NaN bits)
         int prow;
         if constexpr (DECODE) prow = bt[pos >> 6] * 64 + (pos & 63);
         else prow = seq_start + pos;
-        const uint32_t vbits = __ballot_sync(0xffffffffu, valid) & 0xFFFFu;
-        if (lane == 0) reinterpret_cast<uint16_t*>(&s_vmask[stage])[pw] = static_cast<uint16_t>(vbits);
+        const uint32_t vbits = __ballot_sync(0xffffffffu, valid);
+        if (lane == 0) reinterpret_cast<uint32_t*>(&s_vmask[stage])[pw] = vbits;
         const uint32_t st = smem_addr(sKV + stage * kStageBytes);
 #pragma unroll 4
-        for (int j = 0; j < 16; ++j) {  // nope: 32 lanes x 16 bytes of one key
-          const int r = 16 * pw + j;
+        for (int j = 0; j < 32; ++j) {  // nope: 32 lanes x 16 bytes of one key
+          const int r = 32 * pw + j;
           const int kr = __shfl_sync(0xffffffffu, prow, j);
           const __nv_bfloat16* src = latent + static_cast<int64_t>(kr) * 576 + 256 * rank + 8 * lane;
           const int blk = lane >> 3, ch = lane & 7;
           cp_async16(st + blk * kNopeBlockBytes + r * 128 + ((ch ^ (r & 7)) << 4), src);
         }
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {  // rope: 8 keys x 4 chunks of 16 bytes per instruction
+        for (int h2 = 0; h2 < 4; ++h2) {  // rope: 8 keys x 4 chunks of 16 bytes per instruction
           const int j = 8 * h2 + (lane >> 2), ch = lane & 3;
-          const int r = 16 * pw + j;
+          const int r = 32 * pw + j;
           const int kr = __shfl_sync(0xffffffffu, prow, j);
           const __nv_bfloat16* src = latent + static_cast<int64_t>(kr) * 576 + 512 + 32 * rank + 8 * ch;
           cp_async16(st + 4 * kNopeBlockBytes + r * 64 + ((ch ^ ((r >> 1) & 3)) << 4), src);
         }
         cp_async_commit();
-        if (pending_stage >= 0) {
-          cp_async_wait<1>();
-          announce(pending_stage);
-        }
-        pending_stage = stage;
+        cp_async_mbar_arrive(&bar_kvfull[stage]);
+        mbar_arrive(&bar_kvfull[stage]);  // releases the validity mask written above
       }
     }
-    if (pending_stage >= 0) {
-      cp_async_wait<0>();
-      announce(pending_stage);
-    }
-  } else if (warp == 8) {
+    cp_async_wait<0>();
+  } else if (warp == kMmaWarp) {
     // ================= MMA issuer =================
     // Two cursors walk the same chunk sequence: Q.K^T of a chunk is issued as soon as its keys
     // are staged and the single S buffer has been read, P.V as soon as P is ready, so the
@@ -321,6 +314,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
         if (ready) {
           tc_fence_after();
           if (lane == 0) {
+            fence_proxy_async_smem();  // the gathered rows were written through the generic proxy
             const uint32_t st = smem_addr(sKV + stage * kStageBytes);
 #pragma unroll
             for (int kk = 0; kk < 16; ++kk)  // 256 nope dims: 4 blocks x 4 steps of 16
@@ -369,6 +363,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       if (did) {
         idle_since = 0;
       } else {
+        // back off briefly: this warp shares an SM sub-partition with a softmax warp, and a
+        // tight polling loop would take issue slots from it
+        __nanosleep(64);
         const uint64_t now = global_timer_ns();
         if (idle_since == 0) idle_since = now;
         else if (now - idle_since > kWaitLimitNs) {
@@ -388,26 +385,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       xbar_full_peer[i] = map_to_rank(smem_addr(&bar_xfull[i]), peer);
       xbar_empty_peer[i] = map_to_rank(smem_addr(&bar_xempty[i]), peer);
     }
-    // Q rows of this rank's dims into TMEM columns [kColQ, kColQ + 144)
+    // Q rows of this rank's dims into TMEM columns [kColQ, kColQ + 144): three batches of
+    // twelve 16-byte loads, so the row costs three memory round trips rather than nine.
     auto load_q = [&](int64_t qrow) {
       const __nv_bfloat16* qr = p.q + (qrow * p.H + h) * 576;
       const bool real = h < p.H;
 #pragma unroll
-      for (int c = 0; c < 144; c += 16) {
-        uint32_t v[16];
+      for (int c0 = 0; c0 < 144; c0 += 48) {
+        uint32_t v[48];
 #pragma unroll
-        for (int j = 0; j < 16; j += 4) {
-          const int col = c + j;  // packed column: dims 2col, 2col+1 of D_r
+        for (int j = 0; j < 48; j += 4) {
+          const int col = c0 + j;  // packed column: dims 2col, 2col+1 of D_r
           const int d = 2 * col < 256 ? 256 * static_cast<int>(rank) + 2 * col
                                       : 512 + 32 * static_cast<int>(rank) + (2 * col - 256);
           uint4 w = make_uint4(0u, 0u, 0u, 0u);
-          if (real) w = *reinterpret_cast<const uint4*>(qr + d);
+          if (real) w = __ldg(reinterpret_cast<const uint4*>(qr + d));
           v[j] = w.x;
           v[j + 1] = w.y;
           v[j + 2] = w.z;
           v[j + 3] = w.w;
         }
-        tmem_st16(lane_base + kColQ + c, v);
+#pragma unroll
+        for (int c = 0; c < 48; c += 16) tmem_st16(lane_base + kColQ + c0 + c, *reinterpret_cast<uint32_t(*)[16]>(v + c));
       }
       tmem_wait_st();
       tc_fence_before();
@@ -552,6 +551,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       int kbeg, kend, seq, seq_start, seq_len, c0, c1;
       unit_info(u, qrow, kbeg, kend, seq, seq_start, seq_len);
       unit_chunks(qrow, kbeg, kend, c0, c1);
+      if (u + ncl < nunits && h < p.H) {  // warm L2 with the next unit's Q row (loaded near this unit's end)
+        int64_t nq;
+        int a, bb, cc, dd, ee;
+        unit_info(u + ncl, nq, a, bb, cc, dd, ee);
+        const char* qn = reinterpret_cast<const char*>(p.q + (nq * p.H + h) * 576);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) prefetch_l2(qn + 512 * rank + 128 * i);
+        prefetch_l2(qn + 1024 + 64 * rank);
+      }
       float m_own = -INFINITY, M = -INFINITY, m_cur = -INFINITY, m_next = -INFINITY;
       uint32_t p_cur[32], p_next[32];
       if (!stage_a(g, c0 == c1 - 1, u + ncl, m_own, p_cur, m_cur)) {
@@ -633,7 +641,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // the peer no longer writes into this CTA's shared memory
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
