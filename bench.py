@@ -142,12 +142,19 @@ def dist_setup(args):
 
 
 def max_over_ranks(x, world):
+    """The slowest rank's value (device time of the timed region), identical on every rank."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(world, tokens_per_rank, ms_per_step):
+    """Whole-job throughput: the tokens all ranks processed in one step over the slowest rank's step."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
 
 
 def barrier(world):
@@ -242,7 +249,7 @@ def run_ours(args, world, rank, local):
     total_ms = max_over_ranks(total_ms, world)
     ms_per_step = total_ms / args.steps
     L, idx_flops, mla_flops, sel_pairs = prefill_work(cfg)
-    value = world * T / (ms_per_step * 1e-3)
+    value = job_value(world, T, ms_per_step)
 
     fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]     # nominal fp8/bf16 ratio 2 (4.5 / 2.25 PF)
     bf16_peak = peaks["bf16_tflops_sustained"]
