@@ -24,8 +24,9 @@
 // The row sums of P come from the tensor cores too: one more small MMA multiplies P by a tile
 // of ones into 16 extra accumulator columns, so they are rescaled together with O_r.
 //
-// Per CTA: warps 0-3 softmax/epilogue (thread h = head h = TMEM lane h), warps 4-5 gather
-// producers, warp 6 MMA issuer and TMEM owner.  The gather uses per-thread cp.async rather
+// Per CTA: warps 0-7 softmax/epilogue (warps w and w+4 share head rows 32(w%4).. = their TMEM
+// lanes; w takes keys 0-31 of each chunk and O columns 0-127, w+4 keys 32-63 and columns
+// 128-255), warps 8-9 gather producers, warp 10 MMA issuer and TMEM owner.  The gather uses per-thread cp.async rather
 // than TMA gather4: on B200 one gather4 instruction costs 65-130 cycles of the TMA engine, far
 // too slow for 64 rows x 576 bytes per 64-key chunk, while a warp-wide cp.async moves one
 // row's 512-byte nope segment in a single coalesced instruction.  TMEM columns: O_r [0,256), Q_r [256,400),
@@ -76,15 +77,18 @@ constexpr int kOnesBytes = 16 * 128;               // B tile of ones for the row
 constexpr int kSmemBytes = kStages * kStageBytes + 4 * kXBufBytes + kOnesBytes;
 constexpr uint32_t kColO = 0, kColQ = 256, kColS = 400, kColP = 464, kColL = 496;
 constexpr float kTau = 8.f;                        // lazy-rescale margin (log2 units)
+constexpr int kPolyPairsOf4 = 1;                   // exponentials by polynomial: this many of every 4 pairs
 constexpr uint32_t kXBytesPerChunk = kXBufBytes;  // one bulk copy of the whole row block per chunk
 
-__device__ __forceinline__ void sm_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barriers: 1 = all softmax warps (256 threads), 2 + q = the two warps of lane quadrant q.
+__device__ __forceinline__ void sm_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void pair_sync(int q) { asm volatile("bar.sync %0, 64;" ::"r"(2 + q) : "memory"); }
 
 __device__ __forceinline__ bool sm_any(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.or.pred p, 1, 128, q;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+      "bar.red.or.pred p, 1, 256, q;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(r)
       : "r"(static_cast<uint32_t>(v))
       : "memory");
@@ -95,6 +99,22 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe, to take part of the exponentials off the special-function unit:
+// Cody-Waite style range reduction x = n + f with n = round(x) (the 1.5*2^23 shifter leaves n in
+// the low mantissa bits of t) and |f| <= 1/2, then a cubic for 2^f whose coefficients were fitted
+// for least maximum relative error on [-1/2, 1/2] (7.5e-5, far below the bf16 rounding the
+// result gets), and n added to the exponent field.  Inputs are clamped at -125 so the exponent
+// never underflows; callers pass x <= 8 (the lazy-rescale margin).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  float p = fmaf(f, 0.0551716648f, 0.2426111251f);
+  p = fmaf(p, f, 0.6932609677f);
+  p = fmaf(p, f, 0.9999280572f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
@@ -116,11 +136,13 @@ __device__ __forceinline__ int active_chunks(const int32_t* row, int k) {
 }  // namespace mla
 
 namespace mla {
-// 4 softmax + 2 producer + 1 MMA warps.  At most 2 warps per SM sub-partition keeps the full
-// 255 registers per thread available (9 warps would put 3 on one and cap them at 168).
-constexpr int kThreads = 7 * 32;
+// 8 softmax warps (two per TMEM lane quadrant), 2 gather producers, 1 MMA issuer.
+constexpr int kSoftmaxWarps = 8;
+constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
 constexpr int kProducerWarps = 2;
-constexpr int kMmaWarp = 4 + kProducerWarps;
+constexpr int kFirstProducerWarp = kSoftmaxWarps;
+constexpr int kMmaWarp = kSoftmaxWarps + kProducerWarps;
+constexpr int kThreads = 32 * (kMmaWarp + 1);
 }  // namespace mla
 
 template <bool DECODE>
@@ -144,6 +166,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
   __shared__ uint64_t bar_xfull[2], bar_xempty[2];
   __shared__ uint64_t s_vmask[kStages];                    // valid rows of each staged chunk (32 bits per producer warp)
   __shared__ uint32_t s_tmem;
+  __shared__ float s_rmax[2][128];                         // per-half row maxima of the current chunk
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
@@ -155,12 +178,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       mbar_init(&bar_kvfull[i], 32 * kProducerWarps);  // every producer thread (plus its copies in flight)
       mbar_init(&bar_kvempty[i], 1);
     }
-    mbar_init(&bar_qfull, 128);
+    mbar_init(&bar_qfull, kSoftmaxThreads);
     mbar_init(&bar_sfull, 1);
-    mbar_init(&bar_sfree, 4);
-    mbar_init(&bar_pfull, 4);
+    mbar_init(&bar_sfree, kSoftmaxWarps);
+    mbar_init(&bar_pfull, kSoftmaxWarps);
     mbar_init(&bar_pvdone, 1);
-    mbar_init(&bar_ofree, 4);
+    mbar_init(&bar_ofree, kSoftmaxWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_xfull[i], 1);     // own arm (expect_tx) + the peer's asynchronous stores
       mbar_init(&bar_xempty[i], 1);    // one remote arrival: the peer has read this CTA's row block
@@ -215,14 +238,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
     if (c1 <= c0) c1 = c0 + 1;  // always at least one chunk (all masked if empty)
   };
 
-  if (warp >= 4 && warp < kMmaWarp) {
+  if (warp >= kFirstProducerWarp && warp < kMmaWarp) {
     // ================= gather producers =================
     // Warp pw copies keys [32 pw, 32 pw + 32) of each 64-key chunk: one warp instruction per key
     // for its 512-byte nope segment (lane l -> 16-byte chunk l, written at its 128-byte-swizzle
     // position), four more for the 64-byte rope halves of the 32 keys (64-byte swizzle).  The
     // stage's barrier completes on its own once the copies have landed (an asynchronous
     // arrival per thread); the MMA warp fences the proxies before the tensor cores read it.
-    const int pw = warp - 4;
+    // (Measured against announcing each stage after cp.async.wait_group, with or without an
+    // early flush when the next slot is busy: this is the faster of the two on B200.)
+    const int pw = warp - kFirstProducerWarp;
     uint32_t g = 0;
     bool ok = true;
     for (int64_t u = cid; ok && u < nunits; u += ncl) {
@@ -363,9 +388,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       if (did) {
         idle_since = 0;
       } else {
-        // back off briefly: this warp shares an SM sub-partition with a softmax warp, and a
-        // tight polling loop would take issue slots from it
-        __nanosleep(64);
         const uint64_t now = global_timer_ns();
         if (idle_since == 0) idle_since = now;
         else if (now - idle_since > kWaitLimitNs) {
@@ -376,37 +398,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
     }
     if (!ok && lane == 0) record_device_error(DSA_ERR_TIMEOUT);
   } else {
-    // ================= softmax / exchange / epilogue (warps 0-3) =================
-    const int h = tid;  // head row == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    // ================= softmax / exchange / epilogue (warps 0-7) =================
+    // Warps w and w+4 own the same TMEM lanes (head rows 32(w%4)..+31); warp w takes keys 0-31
+    // of every chunk and O columns 0-127, warp w+4 keys 32-63 and O columns 128-255.  The two
+    // share the row maximum through shared memory, so both halves use one reference per row.
+    const int q4 = warp & 3, hf = warp >> 2;
+    const int h = 32 * q4 + lane;  // head row == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const uint32_t x_peer = map_to_rank(smem_addr(sX), peer);
     uint32_t xbar_full_peer[2], xbar_empty_peer[2];
     for (int i = 0; i < 2; ++i) {
       xbar_full_peer[i] = map_to_rank(smem_addr(&bar_xfull[i]), peer);
       xbar_empty_peer[i] = map_to_rank(smem_addr(&bar_xempty[i]), peer);
     }
-    // Q rows of this rank's dims into TMEM columns [kColQ, kColQ + 144): three batches of
-    // twelve 16-byte loads, so the row costs three memory round trips rather than nine.
+    // Q rows of this rank's dims into TMEM columns [kColQ, kColQ + 144), in 16-column groups:
+    // half 0 stores groups 0-4, half 1 groups 5-8, each in batches of up to three groups whose
+    // loads are all in flight together.
     auto load_q = [&](int64_t qrow) {
       const __nv_bfloat16* qr = p.q + (qrow * p.H + h) * 576;
       const bool real = h < p.H;
-#pragma unroll
-      for (int c0 = 0; c0 < 144; c0 += 48) {
+      const int gbeg = hf == 0 ? 0 : 5, gend = hf == 0 ? 5 : 9;
+#pragma unroll 1
+      for (int gb = gbeg; gb < gend; gb += 3) {
         uint32_t v[48];
 #pragma unroll
-        for (int j = 0; j < 48; j += 4) {
-          const int col = c0 + j;  // packed column: dims 2col, 2col+1 of D_r
+        for (int j = 0; j < 12; ++j) {  // 12 x 16 bytes = three groups
+          const int col = 16 * gb + 4 * j;  // packed column: dims 2col, 2col+1 of D_r
           const int d = 2 * col < 256 ? 256 * static_cast<int>(rank) + 2 * col
                                       : 512 + 32 * static_cast<int>(rank) + (2 * col - 256);
           uint4 w = make_uint4(0u, 0u, 0u, 0u);
-          if (real) w = __ldg(reinterpret_cast<const uint4*>(qr + d));
-          v[j] = w.x;
-          v[j + 1] = w.y;
-          v[j + 2] = w.z;
-          v[j + 3] = w.w;
+          if (real && gb + j / 4 < gend) w = __ldg(reinterpret_cast<const uint4*>(qr + d));
+          v[4 * j] = w.x;
+          v[4 * j + 1] = w.y;
+          v[4 * j + 2] = w.z;
+          v[4 * j + 3] = w.w;
         }
 #pragma unroll
-        for (int c = 0; c < 48; c += 16) tmem_st16(lane_base + kColQ + c0 + c, *reinterpret_cast<uint32_t(*)[16]>(v + c));
+        for (int j = 0; j < 3; ++j)
+          if (gb + j < gend) tmem_st16(lane_base + kColQ + 16 * (gb + j), *reinterpret_cast<uint32_t(*)[16]>(v + 16 * j));
       }
       tmem_wait_st();
       tc_fence_before();
@@ -421,17 +450,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       unit_info(cid, qrow, kbeg, kend, seq, ss, sl);
       load_q(qrow);
     }
-    // Stage A of chunk gg: read the partial logits, form this rank's factor
+    // Stage A of chunk gg: read this half's partial logits, form this rank's factor
     // P_own = 2^(x*S_r - m_own) as bf16 and send it with m_own to the peer.
-    auto stage_a = [&](uint32_t gg, bool last_of_unit, int64_t next_unit, float& m_own, uint32_t(&pown)[32],
+    auto stage_a = [&](uint32_t gg, bool last_of_unit, int64_t next_unit, float& m_own, uint32_t(&pown)[16],
                        float& m_sent) -> bool {
       const int stage = static_cast<int>(gg % kStages);
       bool ok = mbar_wait(&bar_sfull, gg & 1u);
       if (sm_any(!ok)) return false;
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(lane_base + kColS, *reinterpret_cast<uint32_t(*)[32]>(sr));
-      tmem_ld32(lane_base + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+      uint32_t sr[32];
+      tmem_ld32(lane_base + kColS + 32 * hf, sr);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -442,44 +470,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
         unit_info(next_unit, nq, a, bb, cc, dd, ee);
         load_q(nq);
       }
-      // the validity mask was written by the producer before it armed this stage's barrier
+      // the validity mask was written by the producer before it arrived on this stage's barrier;
+      // producer warp hf gathered exactly this half's keys
       ok = mbar_wait(&bar_kvfull[stage], (gg / kStages) & 1u);
       if (sm_any(!ok)) return false;
-      const uint64_t vmask = s_vmask[stage];
-      const bool full = vmask == ~0ull;
-      float smax = -INFINITY;
+      const uint32_t vmask = reinterpret_cast<const uint32_t*>(&s_vmask[stage])[hf];
+      const bool full = vmask == ~0u;
+      // row maximum over this half as 8 independent chains, then with the partner half
+      float mx[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mx[j] = -INFINITY;
       if (full) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) smax = fmaxf(smax, __uint_as_float(sr[i]));
+        for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[i]));
       } else {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if ((vmask >> i) & 1ull) smax = fmaxf(smax, __uint_as_float(sr[i]));
+        for (int i = 0; i < 32; ++i)
+          if ((vmask >> i) & 1u) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[i]));
       }
+      const float hmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      s_rmax[hf][h] = hmax;
+      pair_sync(q4);
+      const float smax = fmaxf(hmax, s_rmax[hf ^ 1][h]);
       const float cmax = smax * p.scale_log2;  // scale > 0
       if (cmax > m_own + kTau || (m_own == -INFINITY && cmax > -INFINITY)) m_own = cmax;
       const float neg_m = -m_own;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        float a = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), p.scale_log2, neg_m));
-        float bq = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), p.scale_log2, neg_m));
+      for (int i = 0; i < 16; ++i) {
+        const float xa = fmaf(__uint_as_float(sr[2 * i]), p.scale_log2, neg_m);
+        const float xb = fmaf(__uint_as_float(sr[2 * i + 1]), p.scale_log2, neg_m);
+        float a, bq;
+        if ((i & 3) < kPolyPairsOf4) {  // this share of the pairs on the FMA pipe
+          a = exp2_poly(xa);
+          bq = exp2_poly(xb);
+        } else {
+          a = ex2_approx(xa);
+          bq = ex2_approx(xb);
+        }
         if (!full) {
-          a = ((vmask >> (2 * i)) & 1ull) ? a : 0.f;
-          bq = ((vmask >> (2 * i + 1)) & 1ull) ? bq : 0.f;
+          a = ((vmask >> (2 * i)) & 1u) ? a : 0.f;
+          bq = ((vmask >> (2 * i + 1)) & 1u) ? bq : 0.f;
         }
         pown[i] = pack_bf16x2(a, bq);
       }
       // The peer has read the block of chunk gg-2 (so that copy, which read this staging
-      // buffer, is complete): stage this chunk's rows locally and let the TMA engine push the
-      // whole block to the peer, keeping the load/store path free.
+      // buffer, is complete): stage this half of the row locally and let the TMA engine push
+      // the whole block to the peer, keeping the load/store path free.
       const int xb = static_cast<int>(gg & 1u);
       ok = mbar_wait_cluster(&bar_xempty[xb], ((gg >> 1) & 1u) ^ 1u);
       if (sm_any(!ok)) return false;
       uint8_t* row = sXout + xb * kXBufBytes + h * kXRowBytes;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        *reinterpret_cast<uint4*>(row + 16 * i) = make_uint4(pown[4 * i], pown[4 * i + 1], pown[4 * i + 2], pown[4 * i + 3]);
-      *reinterpret_cast<float*>(row + 128) = m_own;
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<uint4*>(row + 64 * hf + 16 * i) =
+            make_uint4(pown[4 * i], pown[4 * i + 1], pown[4 * i + 2], pown[4 * i + 3]);
+      if (hf == 0) *reinterpret_cast<float*>(row + 128) = m_own;
       fence_proxy_async_smem();
       sm_sync();
       if (tid == 0)
@@ -488,18 +533,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       return true;
     };
     // Stage B of chunk gg: receive the peer's factor, form P = P_own * P_peer relative to
-    // M = m_own + m_peer (identical in both ranks), rescale O_r and the row sums if M moved,
-    // and hand P to the tensor cores.
-    auto stage_b = [&](uint32_t gg, bool first_of_unit, const uint32_t(&pown)[32], float m_sent, float& M) -> bool {
+    // M = m_own + m_peer (identical in both ranks and both halves), rescale this half's O
+    // columns (and the row sums) if M moved, and hand this half of P to the tensor cores.
+    auto stage_b = [&](uint32_t gg, bool first_of_unit, const uint32_t(&pown)[16], float m_sent, float& M) -> bool {
       const int xb = static_cast<int>(gg & 1u);
       if (tid == 0) mbar_arrive_expect_tx(&bar_xfull[xb], kXBytesPerChunk);  // may land before or after the data
       bool ok = mbar_wait_cluster(&bar_xfull[xb], (gg >> 1) & 1u);
       if (sm_any(!ok)) return false;
       const uint8_t* src = sX + xb * kXBufBytes + h * kXRowBytes;
-      uint32_t pp[32];
+      uint32_t pp[16];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint4 w = *reinterpret_cast<const uint4*>(src + 16 * i);
+      for (int i = 0; i < 4; ++i) {
+        const uint4 w = *reinterpret_cast<const uint4*>(src + 64 * hf + 16 * i);
         pp[4 * i] = bf16x2_mul(pown[4 * i], w.x);
         pp[4 * i + 1] = bf16x2_mul(pown[4 * i + 1], w.y);
         pp[4 * i + 2] = bf16x2_mul(pown[4 * i + 2], w.z);
@@ -514,7 +559,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       } else {
         sm_sync();
       }
-      // every thread has read its row of the peer's block (the barrier above): release it.
+      // every thread has read its part of the peer's block (the barrier above): release it.
       // (Not thread 0: its cluster-scope release would also wait for the bulk copy it issued.)
       if (tid == 32) mbar_arrive_remote(xbar_empty_peer[xb]);
       // tcgen05.ld/st are warp-collective: the whole warp runs the rescale if any row needs it
@@ -522,23 +567,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       if (__any_sync(0xffffffffu, need_rescale)) {
         const float alpha = need_rescale ? exp2f(M - Mn) : 1.f;
 #pragma unroll 1
-        for (int c32 = 0; c32 < 256; c32 += 32) {
+        for (int c32 = 0; c32 < 128; c32 += 32) {
           uint32_t o[32];
-          tmem_ld32(lane_base + kColO + c32, o);
+          tmem_ld32(lane_base + kColO + 128 * hf + c32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(lane_base + kColO + c32, o);
+          tmem_st32(lane_base + kColO + 128 * hf + c32, o);
         }
-        uint32_t lv[16];
-        tmem_ld16(lane_base + kColL, lv);
-        tmem_wait_ld();
+        if (hf == 0) {
+          uint32_t lv[16];
+          tmem_ld16(lane_base + kColL, lv);
+          tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) lv[i] = __float_as_uint(__uint_as_float(lv[i]) * alpha);
-        tmem_st16(lane_base + kColL, lv);
+          for (int i = 0; i < 16; ++i) lv[i] = __float_as_uint(__uint_as_float(lv[i]) * alpha);
+          tmem_st16(lane_base + kColL, lv);
+        }
       }
       M = Mn;
-      tmem_st32(lane_base + kColP, pp);
+      tmem_st16(lane_base + kColP + 16 * hf, pp);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -556,12 +603,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
         int a, bb, cc, dd, ee;
         unit_info(u + ncl, nq, a, bb, cc, dd, ee);
         const char* qn = reinterpret_cast<const char*>(p.q + (nq * p.H + h) * 576);
+        if (hf == 0) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) prefetch_l2(qn + 512 * rank + 128 * i);
-        prefetch_l2(qn + 1024 + 64 * rank);
+          for (int i = 0; i < 4; ++i) prefetch_l2(qn + 512 * rank + 128 * i);
+        } else {
+          prefetch_l2(qn + 1024 + 64 * rank);
+        }
       }
       float m_own = -INFINITY, M = -INFINITY, m_cur = -INFINITY, m_next = -INFINITY;
-      uint32_t p_cur[32], p_next[32];
+      uint32_t p_cur[16], p_next[16];
       if (!stage_a(g, c0 == c1 - 1, u + ncl, m_own, p_cur, m_cur)) {
         aborted = true;
         break;
@@ -576,11 +626,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
           break;
         }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) p_cur[i] = p_next[i];
+        for (int i = 0; i < 16; ++i) p_cur[i] = p_next[i];
         m_cur = m_next;
       }
       if (aborted) break;
-      // epilogue of the unit: O_r / l
+      // epilogue of the unit: this half's O columns / l
       bool ok = mbar_wait(&bar_pvdone, (g - 1) & 1u);
       if (sm_any(!ok)) {
         aborted = true;
@@ -593,11 +643,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       const float l = __uint_as_float(lv[0]);
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       if constexpr (!DECODE) {
-        __nv_bfloat16* orow = p.out + (qrow * p.H + h) * 512 + 256 * rank;
+        __nv_bfloat16* orow = p.out + (qrow * p.H + h) * 512 + 256 * rank + 128 * hf;
 #pragma unroll 1
-        for (int c32 = 0; c32 < 256; c32 += 32) {
+        for (int c32 = 0; c32 < 128; c32 += 32) {
           uint32_t o[32];
-          tmem_ld32(lane_base + kColO + c32, o);
+          tmem_ld32(lane_base + kColO + 128 * hf + c32, o);
           tmem_wait_ld();
           if (h < p.H) {
             uint32_t pk[16];
@@ -609,15 +659,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
               *reinterpret_cast<uint4*>(orow + c32 + 8 * i) = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
         }
-        if (rank == 0 && p.lse != nullptr && h < p.H)
+        if (rank == 0 && hf == 0 && p.lse != nullptr && h < p.H)
           p.lse[qrow * p.H + h] = l > 0.f ? (M + log2f(l)) * 0.69314718055994531f : -INFINITY;
       } else {
         const int sp = static_cast<int>(u % p.splits);
-        float* po = p.part_o + ((static_cast<int64_t>(seq) * p.splits + sp) * p.H + h) * 512 + 256 * rank;
+        float* po = p.part_o + ((static_cast<int64_t>(seq) * p.splits + sp) * p.H + h) * 512 + 256 * rank + 128 * hf;
 #pragma unroll 1
-        for (int c32 = 0; c32 < 256; c32 += 32) {
+        for (int c32 = 0; c32 < 128; c32 += 32) {
           uint32_t o[32];
-          tmem_ld32(lane_base + kColO + c32, o);
+          tmem_ld32(lane_base + kColO + 128 * hf + c32, o);
           tmem_wait_ld();
           if (h < p.H) {
 #pragma unroll
@@ -625,7 +675,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
               *reinterpret_cast<uint4*>(po + c32 + 4 * i) = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
           }
         }
-        if (rank == 0 && h < p.H) {
+        if (rank == 0 && hf == 0 && h < p.H) {
           float* ml = p.part_ml + ((static_cast<int64_t>(seq) * p.splits + sp) * p.H + h) * 2;
           ml[0] = M;
           ml[1] = l;
