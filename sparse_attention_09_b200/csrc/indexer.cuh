@@ -287,7 +287,9 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
       }
       const bool ok = mbar_wait(&bar_accfull[acc], aph);
       if (!ok) record_device_error(DSA_ERR_TIMEOUT);
-      if (sel::gany(G, !ok)) {
+      // top-k mode takes the abort decision at its per-tile group vote below (one barrier per
+      // tile); reading a stale accumulator before it is harmless
+      if (MODE == kIdxScores && sel::gany(G, !ok)) {
         aborted = true;
         break;
       }
@@ -295,12 +297,17 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
       float part[TPG][2];
 #pragma unroll
       for (int tt = 0; tt < TPG; ++tt) part[tt][0] = part[tt][1] = 0.f;
-      constexpr int CH = NG >= 32 ? 32 : NG;
+      // columns in slices of up to 64 (two loads, one wait: the TMEM load latency is paid
+      // once per 64 columns)
+      constexpr int CH = NG >= 64 ? 64 : (NG >= 32 ? 32 : NG);
 #pragma unroll
       for (int c0 = 0; c0 < NG; c0 += CH) {
-        uint32_t r[32];
-        if constexpr (CH == 32) {
-          tmem_ld32(lane_base + acc * N + c0, r);
+        uint32_t r[CH >= 32 ? CH : 32];
+        if constexpr (CH == 64) {
+          tmem_ld32(lane_base + acc * N + c0, *reinterpret_cast<uint32_t(*)[32]>(r));
+          tmem_ld32(lane_base + acc * N + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        } else if constexpr (CH == 32) {
+          tmem_ld32(lane_base + acc * N + c0, *reinterpret_cast<uint32_t(*)[32]>(r));
         } else if constexpr (CH == 16) {
           tmem_ld16(lane_base + acc * N + c0, *reinterpret_cast<uint32_t(*)[16]>(r));
         } else {
@@ -364,7 +371,11 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
           wcnt[tt] += __popc(m);
           need_cut |= wcnt[tt] > Q - 32;  // the next tile could add 32 more to this region
         }
-        if (sel::gany(G, need_cut)) {
+        if (sel::gany(G, need_cut || !ok)) {
+          if (sel::gany(G, !ok)) {
+            aborted = true;
+            break;
+          }
           if (lane == 0) {
 #pragma unroll
             for (int tt = 0; tt < TPG; ++tt) s_cnt[tg0 + tt][q] = wcnt[tt];

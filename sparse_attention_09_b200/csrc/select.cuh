@@ -73,12 +73,10 @@ struct Cands {
 
 __device__ __forceinline__ int total_count(const Cands& C) { return C.cnt[0] + C.cnt[1] + C.cnt[2] + C.cnt[3]; }
 
-// Histogram increment aggregated over the lanes of a warp that hit the same bin.  Every lane
-// of the warp must call it.
+// Histogram increment (a shared-memory reduction; lanes hitting one bin are combined by the
+// memory unit).
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool valid) {
-  const uint32_t tag = valid ? bin : 0xFFFFFFFFu;
-  const uint32_t peers = __match_any_sync(0xffffffffu, tag);
-  if (valid && static_cast<int>(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+  if (valid) atomicAdd(&hist[bin], 1u);
 }
 
 // Calls f(key, idx, valid) for every entry of this warp's region, 32 at a time, with every
@@ -127,7 +125,9 @@ __device__ __forceinline__ void group_minmax(const Group& G, Scratch& S, uint32_
 
 // Keeps the entries with keep(key, idx), spreads them round-robin over the 4 regions and
 // returns the smallest kept key.  Every entry of the warp's region is read into registers
-// before the barrier that precedes the first write, so no entry is overwritten unread.
+// before the barrier that precedes the first write, so no entry is overwritten unread.  Output
+// positions come from per-warp ballots and one group scan (no shared-memory atomics, which
+// would serialise the rounds).
 template <class Keep>
 __device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S, Keep keep) {
   constexpr int kMaxRounds = 32;  // Q <= 1024 = 32 lanes x 32 rounds
@@ -135,6 +135,7 @@ __device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S
   const int c = C.cnt[w];
   uint32_t key[kMaxRounds];
   int32_t id[kMaxRounds];
+  uint32_t keepbits = 0u;  // bit r: this lane keeps its entry of round r
 #pragma unroll
   for (int r = 0; r < kMaxRounds; ++r) {
     const int i = r * 32 + lane;
@@ -143,40 +144,35 @@ __device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S
     if (i < c) {
       key[r] = C.key[w * C.Q + i];
       id[r] = C.idx[w * C.Q + i];
+      if (keep(key[r], id[r])) keepbits |= 1u << r;
     }
   }
-  if (G.tid == 0) {
-    S.cursor = 0u;
-    S.kmin = 0xFFFFFFFFu;
-  }
-  gsync(G);
+  const int wcount = __reduce_add_sync(0xffffffffu, __popc(keepbits));
+  int total;
+  int base = gscan(G, lane == 0 ? wcount : 0, S.scan, total);  // its barriers order reads before writes
+  base = __shfl_sync(0xffffffffu, base, 0);
   uint32_t mn = 0xFFFFFFFFu;
+  const uint32_t below = (1u << lane) - 1u;
 #pragma unroll
   for (int r = 0; r < kMaxRounds; ++r) {
     if (r * 32 >= c) break;
-    const bool k = (r * 32 + lane < c) && keep(key[r], id[r]);
+    const bool k = (keepbits >> r) & 1u;
     const uint32_t m = __ballot_sync(0xffffffffu, k);
-    if (m != 0u) {
-      const int leader = __ffs(m) - 1;
-      uint32_t base = 0;
-      if (lane == leader) base = atomicAdd(&S.cursor, static_cast<uint32_t>(__popc(m)));
-      base = __shfl_sync(0xffffffffu, base, leader);
-      if (k) {
-        const uint32_t p = base + static_cast<uint32_t>(__popc(m & ((1u << lane) - 1u)));
-        const int slot = static_cast<int>(p & 3u) * C.Q + static_cast<int>(p >> 2);
-        C.key[slot] = key[r];
-        C.idx[slot] = id[r];
-        mn = min(mn, key[r]);
-      }
+    if (k) {
+      const uint32_t p = static_cast<uint32_t>(base) + static_cast<uint32_t>(__popc(m & below));
+      const int slot = static_cast<int>(p & 3u) * C.Q + static_cast<int>(p >> 2);
+      C.key[slot] = key[r];
+      C.idx[slot] = id[r];
+      mn = min(mn, key[r]);
     }
+    base += __popc(m);
   }
   mn = __reduce_min_sync(0xffffffffu, mn);
-  if (lane == 0) atomicMin(&S.kmin, mn);
+  if (lane == 0) S.tmp_key[w] = mn;  // tmp_key is free here (cut_final is done with it)
   gsync(G);
-  const int total = static_cast<int>(S.cursor);
-  const uint32_t kmin = S.kmin;
+  const uint32_t kmin = min(min(S.tmp_key[0], S.tmp_key[1]), min(S.tmp_key[2], S.tmp_key[3]));
   if (G.tid < 4) C.cnt[G.tid] = total / 4 + (G.tid < total % 4 ? 1 : 0);
-  gsync(G);
+  gsync(G);  // every thread has read tmp_key and C.cnt is published before anyone moves on
   return kmin;
 }
 
