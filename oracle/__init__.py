@@ -35,6 +35,9 @@ Parity status per function (what pins it, in ``tests/test_oracle_*.py``):
   library routine; single-row, equal-rows and uniform-logit closed forms; permutation
   invariance).
 * ``paged_gather`` / decode functions: pinned (paged layout equals the contiguous result).
+* ``encode_e4m3`` / ``quantize_fp8_rows``: pinned (every finite code round-trips; midpoints
+  between neighbouring values go to the even code; saturation and NaN; agreement with torch's
+  float8_e4m3fn cast on random values; the per-row scale rule and its error bound).
 * Agreement with DeepSeek's trained model: parity unpinned (no weights, no printed values).
 """
 
@@ -42,6 +45,8 @@ from .dsa_oracle import (  # noqa: F401
     E4M3_MAX,
     e4m3_table,
     decode_e4m3,
+    encode_e4m3,
+    quantize_fp8_rows,
     indexer_scores_query,
     indexer_scores,
     indexer_magnitude_query,

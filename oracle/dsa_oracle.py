@@ -57,6 +57,47 @@ def decode_e4m3(codes: np.ndarray) -> np.ndarray:
     return _E4M3[np.asarray(codes, dtype=np.uint8)]
 
 
+def encode_e4m3(y: np.ndarray) -> np.ndarray:
+    """e4m3 bytes of the values y: nearest representable value, ties to the even mantissa
+    (round to nearest even), magnitudes >= 448 saturate to 448, NaN -> 0x7F with its sign
+    bit; the sign of zero is kept.
+
+    Written from the format definition: the 127 non-negative finite values (codes 0..126)
+    increase with the code, so a magnitude is bracketed by two consecutive codes and the
+    nearer one (the even one on a tie) is taken.
+    """
+    y = np.asarray(y, dtype=np.float64)
+    mag = np.abs(y)
+    pos = _E4M3[:127]                                   # codes 0..126, increasing
+    lo = np.clip(np.searchsorted(pos, mag, side="right") - 1, 0, 126)
+    hi = np.minimum(lo + 1, 126)
+    dlo = mag - pos[lo]
+    dhi = pos[hi] - mag
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (lo % 2 == 1))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(mag >= E4M3_MAX, 126, code)         # saturation (and +-inf)
+    code = np.where(np.isnan(y), 0x7F, code)
+    sign = np.where(np.signbit(y), 0x80, 0)
+    return (code | sign).astype(np.uint8)
+
+
+def quantize_fp8_rows(x: np.ndarray):
+    """Per-token FP8 quantiser ([MZ] "工作原理": the indexer runs in FP8 with per-token
+    scales): for each row, scale = amax|x| / 448 in IEEE float32 (1 for an all-zero row) and
+    codes = e4m3(x / scale) with the quotient in IEEE float32.  NaN elements take no part in
+    the maximum.  x: [rows, cols] values exactly representable in float32 (bf16 inputs are).
+    Returns (codes uint8 [rows, cols], scale float32 [rows]).
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    a = np.abs(x32)
+    a = np.where(np.isnan(a), np.float32(0.0), a)
+    amax = a.max(axis=1) if x32.shape[1] else np.zeros(x32.shape[0], np.float32)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        y = (x32 / scale[:, None]).astype(np.float32)
+    return encode_e4m3(y), scale
+
+
 # ---------------------------------------------------------------------------------------------
 # Lightning indexer ([MZ] "工作原理"; [36] "第一步：Lightning Indexer"; [DP] 二)
 # ---------------------------------------------------------------------------------------------
