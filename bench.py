@@ -271,6 +271,7 @@ def run_ours(args, world, rank, local):
 
     # ---- decode chain, same process ----
     decode = run_decode(args, dsa, sm) if (rank == 0 and not args.no_decode) else None
+    next_rows = {"f1_quantize_fp8": run_quantizer(dsa, peaks)} if (rank == 0 and not args.no_decode) else None
 
     # ---- end to end through dsa_forward with host buffers ----
     e2e = run_e2e(args, dsa, inp, cfg, sm) if (rank == 0 and not args.no_e2e) else None
@@ -295,10 +296,41 @@ def run_ours(args, world, rank, local):
                        "global_batch": world * len(cfg["seqlens"]), "seq_len": L, "k": k,
                        "parallelism": f"independent problems x{world}",
                        "l2": "inputs (~40 GB/step) larger than L2; no flush"},
-            "roofline": roofline, "kernels": kernels, "decode": decode, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "kernels": kernels, "decode": decode, "next_rows": next_rows,
+            "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk, "gpu_launches": 2 * args.steps,
         }
         print(json.dumps(line), flush=True)
+
+
+def run_quantizer(dsa, peaks):
+    """NEXT row f1: the per-token FP8 quantiser on the q_I of the L=131072 prefill
+    ([131072, 64 x 128] bf16 -> e4m3 + one scale per token) and on its k_I ([131072, 128]).
+    HBM-bound; algorithmic bytes per row = 2*cols read + cols written + 4 (scale)."""
+    out = {}
+    for name, rows, cols in (("q_index", 131072, 64 * 128), ("k_index", 131072, 128)):
+        x = torch.randn((rows, cols), dtype=torch.bfloat16, device="cuda")
+        codes = torch.empty((rows, cols), dtype=torch.uint8, device="cuda")
+        scale = torch.empty((rows,), dtype=torch.float32, device="cuda")
+        for _ in range(3):
+            dsa.dsa_quantize_fp8(x, codes, scale)
+        torch.cuda.synchronize()
+        n = 20
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            dsa.dsa_quantize_fp8(x, codes, scale)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / n
+        nbytes = rows * (3 * cols + 4)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"rows": rows, "cols": cols, "ms": ms, "gbs": gbs, "bytes": nbytes,
+                     "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                     "l2": "input larger than L2" if rows * cols * 2 > 126e6 else "input fits in L2 (hot)"}
+        del x, codes, scale
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_decode(args, dsa, sm):

@@ -186,6 +186,23 @@ const char* dsa_status_string(int32_t status);
  */
 dsa_status dsa_device_error(int32_t* code, void* stream);
 
+/*
+ * Per-token FP8 quantiser for the indexer operands (the step that produces a2's input
+ * contract; DeepSeek-V3.2-Exp, "Lightning Indexer": the indexer runs in FP8).  For each row r
+ * of x [rows, cols] bf16 (row-major, contiguous; one token: all of its indexer heads for
+ * q_I, its key for k_I):
+ *   scale[r] = amax_c |x[r,c]| / 448 in IEEE fp32 (1 for an all-zero row),
+ *   codes[r*cols + c] = e4m3(x[r,c] / scale[r]), the quotient in IEEE fp32 rounded to the
+ *   nearest e4m3 value (ties to even), saturating at +-448.  NaN elements take no part in
+ *   the maximum and encode as NaN.
+ * Device pointers; x 16-byte aligned, codes 8-byte aligned, cols a positive multiple of 8.
+ * rows == 0 is a no-op.  Outputs are caller-owned; nothing is allocated.
+ * Errors: DSA_ERR_INVALID_ARGUMENT for null/misaligned pointers or a bad cols; the call is
+ * asynchronous on `stream` (launch errors are returned, execution errors surface later).
+ */
+dsa_status dsa_quantize_fp8(const void* x_bf16, int64_t rows, int32_t cols, uint8_t* codes, float* scale,
+                            void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,7 @@ DSA_MODE_DECODE = 1
 
 EXPORTED = ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_mla_prefill", "dsa_sparse_mla_decode",
             "dsa_forward", "dsa_workspace_size", "dsa_status_string", "dsa_device_error",
-            "dsa_sparse_mla_decode_noalloc")
+            "dsa_sparse_mla_decode_noalloc", "dsa_quantize_fp8")
 
 
 class KVDesc(ctypes.Structure):
@@ -78,6 +78,8 @@ _lib.dsa_indexer_topk.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I32, _P,
 _lib.dsa_indexer_topk.restype = _I32
 _lib.dsa_sparse_mla_decode_noalloc.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P]
 _lib.dsa_sparse_mla_decode_noalloc.restype = _I32
+_lib.dsa_quantize_fp8.argtypes = [_P, _I64, _I32, _P, _P, _P]
+_lib.dsa_quantize_fp8.restype = _I32
 _lib.dsa_workspace_size.argtypes = [_I32, _I32, _I64, _I32, _I32, _I32, _I32]
 _lib.dsa_workspace_size.restype = _SZ
 
@@ -138,6 +140,14 @@ def paged_desc(data, block_table, context_lens, max_ctx, scale=None) -> Desc:
                total_tokens=0, max_seqlen=int(max_ctx), num_blocks=int(data.shape[0]),
                block_size=int(data.shape[1]), max_blocks_per_seq=int(block_table.shape[1]))
     return Desc(s, (data, scale, block_table, context_lens))
+
+
+def dsa_quantize_fp8(x, codes, scale, stream=None):
+    """codes[r, :] = e4m3(x[r, :] / scale[r]) with scale[r] = amax|x[r, :]| / 448 (per token)."""
+    rows = x.shape[0]
+    cols = x.numel() // rows if rows else 0
+    _check(_lib.dsa_quantize_fp8(_ptr(x), rows, cols, _ptr(codes), _ptr(scale), _stream(stream)), "dsa_quantize_fp8")
+    return codes, scale
 
 
 def dsa_topk(scores, row_len, k, idx, stream=None):

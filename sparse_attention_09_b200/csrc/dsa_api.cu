@@ -12,6 +12,7 @@
 #include "../../include/dsa.h"
 #include "common.cuh"
 #include "indexer.cuh"
+#include "quantize.cuh"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
 
@@ -219,6 +220,20 @@ dsa_status dsa_device_error(int32_t* code, void* stream) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return DSA_ERR_CUDA;
   *code = v;
   return DSA_OK;
+}
+
+dsa_status dsa_quantize_fp8(const void* x_bf16, int64_t rows, int32_t cols, uint8_t* codes, float* scale,
+                            void* stream) {
+  if (rows < 0) return DSA_ERR_INVALID_ARGUMENT;
+  if (rows == 0) return DSA_OK;
+  if (cols <= 0 || (cols % 8) != 0) return DSA_ERR_INVALID_ARGUMENT;
+  if (x_bf16 == nullptr || codes == nullptr || scale == nullptr || !aligned(x_bf16, 16) || !aligned(codes, 8))
+    return DSA_ERR_INVALID_ARGUMENT;
+  const int64_t blocks = (rows + quant::kWarps - 1) / quant::kWarps;
+  if (blocks > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+  quantize_fp8_rows_kernel<<<static_cast<unsigned>(blocks), quant::kWarps * 32, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x_bf16), rows, cols, codes, scale);
+  return launch_status();
 }
 
 dsa_status dsa_topk(const float* scores, int64_t ld_scores, int64_t rows, const int32_t* row_len, int32_t k,

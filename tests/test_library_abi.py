@@ -46,3 +46,17 @@ def test_host_validation_rejects_bad_arguments_before_launch():
         dsa.DSA_ERR_INVALID_ARGUMENT
     # zero rows is a no-op
     assert lib.dsa_topk(null, 8, 0, null, 4, null, null) == dsa.DSA_OK
+
+
+def test_quantiser_host_validation():
+    import sparse_attention_09_b200 as dsa
+    lib = dsa._lib
+    null = ctypes.c_void_p(0)
+    a = ctypes.c_void_p(4096)
+    assert lib.dsa_quantize_fp8(null, 0, 0, null, null, null) == dsa.DSA_OK            # zero rows: no-op
+    assert lib.dsa_quantize_fp8(a, -1, 8, a, a, null) == dsa.DSA_ERR_INVALID_ARGUMENT
+    assert lib.dsa_quantize_fp8(a, 4, 12, a, a, null) == dsa.DSA_ERR_INVALID_ARGUMENT   # cols % 8
+    assert lib.dsa_quantize_fp8(a, 4, 0, a, a, null) == dsa.DSA_ERR_INVALID_ARGUMENT
+    assert lib.dsa_quantize_fp8(null, 4, 8, a, a, null) == dsa.DSA_ERR_INVALID_ARGUMENT
+    assert lib.dsa_quantize_fp8(ctypes.c_void_p(4104), 4, 8, a, a, null) == dsa.DSA_ERR_INVALID_ARGUMENT  # 16 B
+    assert lib.dsa_quantize_fp8(a, 4, 8, ctypes.c_void_p(4100), a, null) == dsa.DSA_ERR_INVALID_ARGUMENT  # 8 B
