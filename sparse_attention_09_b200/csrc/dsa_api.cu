@@ -229,6 +229,12 @@ dsa_status dsa_quantize_fp8(const void* x_bf16, int64_t rows, int32_t cols, uint
   if (cols <= 0 || (cols % 8) != 0) return DSA_ERR_INVALID_ARGUMENT;
   if (x_bf16 == nullptr || codes == nullptr || scale == nullptr || !aligned(x_bf16, 16) || !aligned(codes, 8))
     return DSA_ERR_INVALID_ARGUMENT;
+  if (cols >= 2048 && cols <= quant::kWideThreads * quant::kWideMaxChunks * 8) {
+    if (rows > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+    quantize_fp8_wide_kernel<<<static_cast<unsigned>(rows), quant::kWideThreads, 0, as_stream(stream)>>>(
+        static_cast<const __nv_bfloat16*>(x_bf16), cols, codes, scale);
+    return launch_status();
+  }
   const int64_t blocks = (rows + quant::kWarps - 1) / quant::kWarps;
   if (blocks > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
   quantize_fp8_rows_kernel<<<static_cast<unsigned>(blocks), quant::kWarps * 32, 0, as_stream(stream)>>>(

@@ -297,16 +297,48 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
       float part[TPG][2];
 #pragma unroll
       for (int tt = 0; tt < TPG; ++tt) part[tt][0] = part[tt][1] = 0.f;
-      // columns in slices of up to 64 (two loads, one wait: the TMEM load latency is paid
-      // once per 64 columns)
-      constexpr int CH = NG >= 64 ? 64 : (NG >= 32 ? 32 : NG);
+      const uint32_t abase = lane_base + acc * N;
+      // part[tt] += w * ReLU(acc) over the 32 columns c0.. held in r
+      auto accumulate32 = [&](const uint32_t(&r)[32], int c0) {
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          const float4 w4 = idx_detail::lds128(sWq + g * NG + c0 + c);
+          const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int col = c0 + c + u;  // column inside the group's slice
+            part[col / H_I][u & 1] = fmaf(wv[u], fmaxf(__uint_as_float(r[c + u]), 0.f), part[col / H_I][u & 1]);
+          }
+        }
+      };
+      if constexpr (NG >= 64 && NG % 64 == 0) {
+        // Software pipeline over 32-column slices: the TMEM load of the next slice is in
+        // flight while this one is summed (tcgen05.wait::ld waits for every load issued so
+        // far, so each wait comes one slice of work after its load).  reg_fence keeps the
+        // compiler from moving uses of the loaded registers above their wait.
+        uint32_t ra[32], rb[32];
+        tmem_ld32(abase, ra);
+        tmem_wait_ld();
+        reg_fence(ra);
+#pragma unroll
+        for (int c0 = 0; c0 < NG; c0 += 64) {
+          tmem_ld32(abase + c0 + 32, rb);
+          accumulate32(ra, c0);
+          tmem_wait_ld();
+          reg_fence(rb);
+          if (c0 + 64 < NG) tmem_ld32(abase + c0 + 64, ra);
+          accumulate32(rb, c0 + 32);
+          if (c0 + 64 < NG) {
+            tmem_wait_ld();
+            reg_fence(ra);
+          }
+        }
+      } else {
+      constexpr int CH = NG >= 32 ? 32 : NG;
 #pragma unroll
       for (int c0 = 0; c0 < NG; c0 += CH) {
-        uint32_t r[CH >= 32 ? CH : 32];
-        if constexpr (CH == 64) {
-          tmem_ld32(lane_base + acc * N + c0, *reinterpret_cast<uint32_t(*)[32]>(r));
-          tmem_ld32(lane_base + acc * N + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-        } else if constexpr (CH == 32) {
+        uint32_t r[32];
+        if constexpr (CH == 32) {
           tmem_ld32(lane_base + acc * N + c0, *reinterpret_cast<uint32_t(*)[32]>(r));
         } else if constexpr (CH == 16) {
           tmem_ld16(lane_base + acc * N + c0, *reinterpret_cast<uint32_t(*)[16]>(r));
@@ -331,6 +363,7 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
             part[col / H_I][u & 1] = fmaf(wv[u], fmaxf(__uint_as_float(r[c + u]), 0.f), part[col / H_I][u & 1]);
           }
         }
+      }
       }
       tc_fence_before();
       __syncwarp();

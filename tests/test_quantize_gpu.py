@@ -32,7 +32,8 @@ def _check(x_gpu, rows=None):
     assert np.array_equal(codes[sel], ref_codes), "codes differ"
 
 
-@pytest.mark.parametrize("rows,cols", [(1, 8), (3, 16), (37, 128), (64, 256), (300, 8192), (9, 136)])
+@pytest.mark.parametrize("rows,cols", [(1, 8), (3, 16), (37, 128), (64, 256), (300, 8192), (9, 136), (7, 2048),
+                                       (5, 4104), (3, 8184), (2, 8200)])
 def test_quantiser_random_rows(rows, cols):
     g = torch.Generator(device="cuda")
     g.manual_seed(rows * 1000 + cols)
