@@ -271,7 +271,8 @@ def run_ours(args, world, rank, local):
 
     # ---- decode chain, same process ----
     decode = run_decode(args, dsa, sm) if (rank == 0 and not args.no_decode) else None
-    next_rows = {"f1_quantize_fp8": run_quantizer(dsa, peaks)} if (rank == 0 and not args.no_decode) else None
+    next_rows = ({"f1_quantize_fp8": run_quantizer(dsa, peaks), "f2_masked_mla": run_masked(dsa, sm)}
+                 if (rank == 0 and not args.no_decode) else None)
 
     # ---- end to end through dsa_forward with host buffers ----
     e2e = run_e2e(args, dsa, inp, cfg, sm) if (rank == 0 and not args.no_e2e) else None
@@ -330,6 +331,40 @@ def run_quantizer(dsa, peaks):
                      "l2": "input larger than L2" if rows * cols * 2 > 126e6 else "input fits in L2 (hot)"}
         del x, codes, scale
     torch.cuda.empty_cache()
+    return out
+
+
+def run_masked(dsa, sm):
+    """NEXT row f2: the masked dense mode of sparse MLA against the sparse path on short
+    prefills (selection from the fused indexer top-k, k = 2048), same outputs."""
+    out = {}
+    for L in (1024, 2048, 4096):
+        cfg = dict(synth.WORKLOADS["prefill_8k"])
+        cfg["seqlens"] = [L]
+        inp = synth.prefill_inputs(device="cuda", **cfg)
+        k, H = cfg["k"], cfg["H"]
+        keys = dsa.contiguous_desc(inp["k8"], inp["cu_seqlens"], L, scale=inp["k_scale"])
+        lat = dsa.contiguous_desc(inp["latent"], inp["cu_seqlens"], L)
+        idx = torch.empty((L, k), dtype=torch.int32, device="cuda")
+        dsa.dsa_indexer_topk(inp["q8"], inp["q_scale"], inp["w"], keys, 1, cfg["H_I"], cfg["d_I"], k, idx)
+        o = torch.empty((L, H, 512), dtype=torch.bfloat16, device="cuda")
+        row = {}
+        for name, fn in (("masked", dsa.dsa_masked_mla_prefill), ("sparse", dsa.dsa_sparse_mla_prefill)):
+            for _ in range(3):
+                fn(inp["q"], lat, idx, 1, H, k, sm, o)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(10):
+                fn(inp["q"], lat, idx, 1, H, k, sm, o)
+            e1.record()
+            torch.cuda.synchronize()
+            row[name + "_ms"] = e0.elapsed_time(e1) / 10
+        pairs = sum(min(k, t + 1) for t in range(L))
+        row["sparse_tflops"] = pairs * 278528 / (row["sparse_ms"] * 1e-3) / 1e12
+        row["masked_tflops_selected"] = pairs * 278528 / (row["masked_ms"] * 1e-3) / 1e12
+        out[f"L{L}"] = row
+    assert dsa.dsa_device_error() == 0
     return out
 
 

@@ -125,6 +125,20 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, int64_t rows, const 
  * q [T, H, 576] bf16, out [T, H, 512] bf16, lse [T, H] fp32 natural log (may be NULL).
  * Every row must hold at least one valid index.
  */
+/*
+ * Masked dense mode of sparse MLA prefill, for short sequences (DeepSeek-V3.2-Exp, "等性能验证":
+ * for short prefill a masked MHA mode simulates DSA): the same out/lse as
+ * dsa_sparse_mla_prefill for the same arguments, computed by walking every causal 64-key chunk
+ * of the contiguous latent with TMA tiles and masking the keys idx does not select.  Cost grows
+ * with L^2 instead of L*k, so it pays only when most causal keys are selected (L up to ~2k).
+ * idx rows must be ascending with the -1 padding at the end (as the top-k entry points write
+ * them); entries outside [0, t] are ignored.  Same layouts, alignment and errors as
+ * dsa_sparse_mla_prefill; additionally DSA_ERR_INVALID_ARGUMENT if the latent cannot be
+ * described to the TMA unit.
+ */
+dsa_status dsa_masked_mla_prefill(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B,
+                                  int32_t H, int32_t k, float sm_scale, void* out, float* lse, void* stream);
+
 dsa_status dsa_sparse_mla_prefill(const void* q, const dsa_kv_desc* latent, const int32_t* idx,
                                   int32_t B, int32_t H, int32_t k, float sm_scale, void* out,
                                   float* lse, void* stream);

@@ -33,7 +33,7 @@ DSA_MODE_DECODE = 1
 
 EXPORTED = ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_mla_prefill", "dsa_sparse_mla_decode",
             "dsa_forward", "dsa_workspace_size", "dsa_status_string", "dsa_device_error",
-            "dsa_sparse_mla_decode_noalloc", "dsa_quantize_fp8")
+            "dsa_sparse_mla_decode_noalloc", "dsa_quantize_fp8", "dsa_masked_mla_prefill")
 
 
 class KVDesc(ctypes.Structure):
@@ -78,6 +78,8 @@ _lib.dsa_indexer_topk.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I32, _P,
 _lib.dsa_indexer_topk.restype = _I32
 _lib.dsa_sparse_mla_decode_noalloc.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P]
 _lib.dsa_sparse_mla_decode_noalloc.restype = _I32
+_lib.dsa_masked_mla_prefill.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P]
+_lib.dsa_masked_mla_prefill.restype = _I32
 _lib.dsa_quantize_fp8.argtypes = [_P, _I64, _I32, _P, _P, _P]
 _lib.dsa_quantize_fp8.restype = _I32
 _lib.dsa_workspace_size.argtypes = [_I32, _I32, _I64, _I32, _I32, _I32, _I32]
@@ -162,6 +164,13 @@ def dsa_indexer_scores(q_fp8, q_scale, w, keys: Desc, B, H_I, d_I, row_begin, ro
                                    int(row_begin), int(row_end), _ptr(scores), scores.stride(0), _stream(stream)),
            "dsa_indexer_scores")
     return scores
+
+
+def dsa_masked_mla_prefill(q, latent: Desc, idx, B, H, k, sm_scale, out, lse=None, stream=None):
+    """Same result as dsa_sparse_mla_prefill, computed densely over the causal prefix with a mask."""
+    _check(_lib.dsa_masked_mla_prefill(_ptr(q), latent.ref(), _ptr(idx), int(B), int(H), int(k), float(sm_scale),
+                                       _ptr(out), _ptr(lse), _stream(stream)), "dsa_masked_mla_prefill")
+    return out
 
 
 def dsa_sparse_mla_prefill(q, latent: Desc, idx, B, H, k, sm_scale, out, lse=None, stream=None):

@@ -151,14 +151,18 @@ size_t decode_partials_bytes(int B, int H, int splits) {
 
 int decode_splits(int k) { return k / 64 < kDecodeSplits ? k / 64 : kDecodeSplits; }
 
-template <bool DECODE>
-dsa_status launch_mla(const void* latent, const MlaParams& p, int64_t units, cudaStream_t s) {
-  auto kern = sparse_mla_kernel<DECODE>;
+template <bool DECODE, bool DENSE = false>
+dsa_status launch_mla(const void* latent, const MlaParams& p, int64_t units, cudaStream_t s,
+                      const CUtensorMap* nope_map = nullptr, const CUtensorMap* rope_map = nullptr) {
+  auto kern = sparse_mla_kernel<DECODE, DENSE>;
   const int smem = mla::kSmemBytes + 1024;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return DSA_ERR_CUDA;
+  CUtensorMap unused;
+  std::memset(&unused, 0, sizeof(unused));
   const int clusters = static_cast<int>(units < kMlaClusters ? units : kMlaClusters);
-  kern<<<2 * clusters, mla::kThreads, smem, s>>>(static_cast<const __nv_bfloat16*>(latent), p);
+  kern<<<2 * clusters, mla::kThreads, smem, s>>>(static_cast<const __nv_bfloat16*>(latent), p,
+                                                  nope_map ? *nope_map : unused, rope_map ? *rope_map : unused);
   return launch_status();
 }
 
@@ -325,6 +329,41 @@ dsa_status dsa_sparse_mla_prefill(const void* q, const dsa_kv_desc* latent, cons
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   return launch_mla<false>(latent->data, p, p.rows, as_stream(stream));
+}
+
+dsa_status dsa_masked_mla_prefill(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B, int32_t H,
+                                  int32_t k, float sm_scale, void* out, float* lse, void* stream) {
+  if (q == nullptr || latent == nullptr || latent->data == nullptr || idx == nullptr || out == nullptr || B <= 0)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (latent->kind != DSA_KV_CONTIGUOUS || latent->cu_seqlens == nullptr || latent->total_tokens <= 0)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(latent->data, 16) || !aligned(idx, 16) || !aligned(out, 16))
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (!mla_shape_ok(H, k)) return DSA_ERR_UNSUPPORTED;
+  if (latent->total_tokens > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+  // the contiguous latent [T, 576] bf16 as two tiled views: 64-dim nope blocks (128-byte
+  // swizzle) and the 32-dim rope halves (64-byte swizzle), 64 rows per tile
+  CUtensorMap nope_map, rope_map;
+  const uint64_t T = static_cast<uint64_t>(latent->total_tokens);
+  if (!make_map_2d(&nope_map, latent->data, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kLatentDim, T, kLatentDim * 2, 64, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&rope_map, latent->data, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kLatentDim, T, kLatentDim * 2, 32, 64,
+                   CU_TENSOR_MAP_SWIZZLE_64B))
+    return DSA_ERR_INVALID_ARGUMENT;
+  MlaParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.idx = idx;
+  p.cu_seqlens = latent->cu_seqlens;
+  p.B = B;
+  p.H = H;
+  p.k = k;
+  p.rows = latent->total_tokens;
+  p.splits = 1;
+  p.scale_log2 = sm_scale * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  return launch_mla<false, true>(latent->data, p, p.rows, as_stream(stream), &nope_map, &rope_map);
 }
 
 dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B, int32_t H,

@@ -38,6 +38,12 @@
 // The same kernel serves decode: a work item is then (sequence, split of its selection) over
 // a paged latent cache, and the unnormalised partial result (O, M, l) goes to a workspace
 // that a small kernel merges by log-sum-exp.
+//
+// And the masked dense mode for short prefill (DENSE): the same attention over the selected
+// rows, computed by walking every causal 64-key chunk of the contiguous latent (loaded with
+// TMA tiles instead of a gather) and masking the keys the selection does not hold, as the
+// pages describe for short sequences (dense attention with a mask simulating the sparse
+// pattern).  The selection rows must be ascending (as the top-k emits them).
 #pragma once
 
 #include "common.cuh"
@@ -145,9 +151,11 @@ constexpr int kMmaWarp = kSoftmaxWarps + kProducerWarps;
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 }  // namespace mla
 
-template <bool DECODE>
+template <bool DECODE, bool DENSE = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
-    sparse_mla_kernel(const __nv_bfloat16* __restrict__ latent, const MlaParams p) {
+    sparse_mla_kernel(const __nv_bfloat16* __restrict__ latent, const MlaParams p,
+                      const __grid_constant__ CUtensorMap nope_map, const __grid_constant__ CUtensorMap rope_map) {
+  static_assert(!(DECODE && DENSE), "the dense mode is a prefill mode");
   using namespace dev;
   using namespace mla;
   constexpr uint32_t IDESC_QK = idesc_bf16(128, kChunk, false, false);
@@ -175,7 +183,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&bar_kvfull[i], 32 * kProducerWarps);  // every producer thread (plus its copies in flight)
+      // every producer thread (plus its copies in flight); dense mode: one arrival + TMA bytes
+      mbar_init(&bar_kvfull[i], DENSE ? 1 : 32 * kProducerWarps);
       mbar_init(&bar_kvempty[i], 1);
     }
     mbar_init(&bar_qfull, kSoftmaxThreads);
@@ -230,15 +239,78 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       seq_len = p.cu_seqlens[lo + 1] - seq_start;
     }
   };
-  // chunks [c0, c1) of the selection row this unit processes
-  auto unit_chunks = [&](int64_t qrow, int kbeg, int kend, int& c0, int& c1) {
+  // chunks [c0, c1) of the selection row this unit processes (dense mode: every causal chunk
+  // of the token's sequence prefix)
+  auto unit_chunks = [&](int64_t qrow, int kbeg, int kend, int seq_start, int& c0, int& c1) {
+    if constexpr (DENSE) {
+      c0 = 0;
+      c1 = static_cast<int>(qrow - seq_start) / kChunk + 1;
+      return;
+    }
     const int act = active_chunks(p.idx + qrow * p.k, p.k);
     c0 = kbeg / kChunk;
     c1 = min(kend / kChunk, act);
     if (c1 <= c0) c1 = c0 + 1;  // always at least one chunk (all masked if empty)
   };
 
-  if (warp >= kFirstProducerWarp && warp < kMmaWarp) {
+  if (DENSE && warp >= kFirstProducerWarp && warp < kMmaWarp) {
+    // ================= dense-mode producer =================
+    // Producer warp 0: per chunk, the selection mask of its 64 keys from the (ascending)
+    // selection row, then five TMA tiles of the contiguous latent (4 x 64 nope dims with the
+    // 128-byte swizzle, 32 rope dims with the 64-byte swizzle) into the stage.
+    if (warp == kFirstProducerWarp) {
+      uint32_t g = 0;
+      bool ok = true;
+      if (lane == 0) {
+        tma_prefetch_desc(&nope_map);
+        tma_prefetch_desc(&rope_map);
+      }
+      for (int64_t u = cid; ok && u < nunits; u += ncl) {
+        int64_t qrow;
+        int kbeg, kend, seq, seq_start, seq_len, c0, c1;
+        unit_info(u, qrow, kbeg, kend, seq, seq_start, seq_len);
+        unit_chunks(qrow, kbeg, kend, seq_start, c0, c1);
+        const int t = static_cast<int>(qrow - seq_start);
+        const int32_t* row = p.idx + qrow * p.k;
+        int pos = 0;  // entries of the row consumed by earlier chunks
+        for (int c = c0; c < c1; ++c, ++g) {
+          const int stage = static_cast<int>(g % kStages);
+          if (!mbar_wait(&bar_kvempty[stage], ((g / kStages) & 1u) ^ 1u)) {
+            record_device_error(DSA_ERR_TIMEOUT);
+            ok = false;
+            break;
+          }
+          // the row's entries in [64c, 64c + 64) form one run starting at pos
+          uint32_t lo = 0u, hi = 0u;
+          while (true) {
+            const int v = pos + lane < p.k ? row[pos + lane] : -1;
+            const bool in = v >= kChunk * c && v < kChunk * (c + 1) && v <= t;
+            const int n = __popc(__ballot_sync(0xffffffffu, in));
+            if (in) {
+              const int bit = v - kChunk * c;
+              if (bit < 32) lo |= 1u << bit;
+              else hi |= 1u << (bit - 32);
+            }
+            pos += n;
+            if (n < 32) break;
+          }
+          lo = __reduce_or_sync(0xffffffffu, lo);
+          hi = __reduce_or_sync(0xffffffffu, hi);
+          if (lane == 0) {
+            s_vmask[stage] = (static_cast<uint64_t>(hi) << 32) | lo;
+            uint8_t* st = sKV + stage * kStageBytes;
+            const int32_t y = seq_start + kChunk * c;
+            mbar_arrive_expect_tx(&bar_kvfull[stage], kStageBytes);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tma_load_2d(st + j * kNopeBlockBytes, &nope_map, &bar_kvfull[stage], 256 * static_cast<int>(rank) + 64 * j, y);
+            tma_load_2d(st + 4 * kNopeBlockBytes, &rope_map, &bar_kvfull[stage], 512 + 32 * static_cast<int>(rank), y);
+          }
+          __syncwarp();
+        }
+      }
+    }
+  } else if (!DENSE && warp >= kFirstProducerWarp && warp < kMmaWarp) {
     // ================= gather producers =================
     // Warp pw copies keys [32 pw, 32 pw + 32) of each 64-key chunk: one warp instruction per key
     // for its 512-byte nope segment (lane l -> 16-byte chunk l, written at its 128-byte-swizzle
@@ -254,7 +326,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       int64_t qrow;
       int kbeg, kend, seq, seq_start, seq_len, c0, c1;
       unit_info(u, qrow, kbeg, kend, seq, seq_start, seq_len);
-      unit_chunks(qrow, kbeg, kend, c0, c1);
+      unit_chunks(qrow, kbeg, kend, seq_start, c0, c1);
       const int32_t* row = p.idx + qrow * p.k;
       const int32_t* bt = DECODE ? p.block_table + static_cast<int64_t>(seq) * p.max_blocks_per_seq : nullptr;
       for (int c = c0; c < c1; ++c, ++g) {
@@ -312,7 +384,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       int64_t qrow;
       int kbeg, kend, seq, seq_start, seq_len;
       unit_info(cu.u, qrow, kbeg, kend, seq, seq_start, seq_len);
-      unit_chunks(qrow, kbeg, kend, cu.c0, cu.c1);
+      unit_chunks(qrow, kbeg, kend, seq_start, cu.c0, cu.c1);
       cu.c = cu.c0;
     };
     auto advance = [&](Cursor& cu) {
@@ -597,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       int64_t qrow;
       int kbeg, kend, seq, seq_start, seq_len, c0, c1;
       unit_info(u, qrow, kbeg, kend, seq, seq_start, seq_len);
-      unit_chunks(qrow, kbeg, kend, c0, c1);
+      unit_chunks(qrow, kbeg, kend, seq_start, c0, c1);
       if (u + ncl < nunits && h < p.H) {  // warm L2 with the next unit's Q row (loaded near this unit's end)
         int64_t nq;
         int a, bb, cc, dd, ee;

@@ -80,6 +80,16 @@ def sparse_mla_prefill(inp, idx, k, sm_scale, with_lse=True):
     return out, lse
 
 
+def masked_mla_prefill(inp, idx, k, sm_scale, with_lse=True):
+    dsa = lib()
+    T, H = inp["q"].shape[0], inp["q"].shape[1]
+    out = torch.full((T, H, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((T, H), float("nan"), device="cuda") if with_lse else None
+    dsa.dsa_masked_mla_prefill(inp["q"], latent_desc(inp), idx, len(inp["seqlens"]), H, k, sm_scale, out, lse)
+    assert dsa.dsa_device_error() == 0
+    return out, lse
+
+
 def assert_attention_close(got, ref, what=""):
     """The stated bar (max-abs 2e-2, mean-abs 2e-3 after bf16 rounding) plus a relative bar
     (1e-2 of the reference norm), since the synthetic outputs are only ~1e-2 in size."""
