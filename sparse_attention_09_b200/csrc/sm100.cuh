@@ -1,5 +1,5 @@
-// Device primitives for sm_100a (B200): mbarriers with bounded waits, TMA tiled and gather4
-// loads, tcgen05 tensor-memory allocation / MMA / load / store, UMMA shared-memory and
+// Device primitives for sm_100a (B200): mbarriers with bounded waits, TMA tiled loads,
+// cp.async, tcgen05 tensor-memory allocation / MMA / load / store, UMMA shared-memory and
 // instruction descriptors, and cluster (distributed shared memory) helpers.
 //
 // Every wait in this file is bounded: a wait that does not complete within the time limit
@@ -247,17 +247,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
       "[%5];" ::"r"(smem_addr(dst)),
       "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
-      : "memory");
-}
-
-// Loads four arbitrary rows (r0..r3) of a 2-D tensor, columns [col, col + box width), into
-// four consecutive rows of the shared-memory tile at dst (the map's box is one row high).
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t col,
-                                            int32_t r0, int32_t r1, int32_t r2, int32_t r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3, %4, %5, %6}], [%7];" ::"r"(smem_addr(dst)),
-      "l"(map), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_addr(bar))
       : "memory");
 }
 

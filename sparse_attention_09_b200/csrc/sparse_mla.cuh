@@ -8,7 +8,7 @@
 // Split over the pair (rank r = 0, 1), with no duplicated tensor-core work:
 //   * rank r owns the latent dims D_r = [256r, 256r+256) u [512+32r, 512+32r+32): it holds
 //     q[t, :, D_r] in TMEM (the A operand of Q.K^T), gathers only those 288 dims of each
-//     selected row (TMA gather4, 128- and 64-byte swizzle), and computes the PARTIAL logits
+//     selected row (into 128- and 64-byte-swizzled SMEM tiles), and computes the PARTIAL logits
 //     S_r = q[:, D_r] . c[:, D_r];
 //   * rank r owns the output half O_r = out[:, 256r : 256r+256] (the value dims it already
 //     gathered) as a [128 x 256] fp32 accumulator in TMEM.

@@ -1,4 +1,4 @@
-"""Sparse MLA (2-CTA cluster, tcgen05 BF16, TMA gather) against the oracle on the GPU's own
+"""Sparse MLA (2-CTA cluster, tcgen05 BF16, cp.async row gather) against the oracle on the GPU's own
 index set: max-abs <= 2e-2 and mean-abs <= 2e-3 after bf16 rounding (the stated bar), plus
 relative error <= 1e-2 (outputs here are ~1e-2, so the absolute bar alone would be loose).
 
