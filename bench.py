@@ -197,6 +197,104 @@ def prefill_work(cfg):
     return L, idx_flops, mla_flops, sel_pairs
 
 
+# ------------------------------------------------------------------------------------------
+# strong scaling: one sequence sharded by query rows (NEXT row f4)
+# ------------------------------------------------------------------------------------------
+def balanced_row_blocks(L, k, world, w_index=137.0, w_mla=145.0):
+    """Boundaries b[0] = 0 < ... < b[world] = L of query-row blocks of equal estimated cost.
+    A row t costs w_index * (t + 1) / sum(t + 1) (the indexer scans its causal prefix) plus
+    w_mla * min(t + 1, k) / sum(min(t + 1, k)) (sparse MLA over its selection); the weights
+    are the two kernels' measured shares of one step."""
+    t = np.arange(L, dtype=np.float64) + 1.0
+    ci = t / t.sum()
+    cm = np.minimum(t, k)
+    cm /= cm.sum()
+    cum = np.cumsum(w_index * ci + w_mla * cm)
+    targets = cum[-1] * np.arange(1, world) / world
+    inner = np.searchsorted(cum, targets, side="left") + 1
+    b = [0] + [int(x) for x in inner] + [L]
+    for i in range(1, len(b)):  # keep the blocks non-empty and ordered
+        b[i] = max(b[i], min(L, b[i - 1] + 1)) if i < len(b) - 1 else L
+    return b
+
+
+def even_row_blocks(L, world):
+    """Equal row blocks (how the key / latent rows are spread before the all-gather)."""
+    return [L * r // world for r in range(world + 1)]
+
+
+def gather_rows(local, full, world):
+    """All-gather of equal row blocks of `full` (block r comes from rank r) into `full`."""
+    if world == 1:
+        full.copy_(local)
+        return full
+    import torch.distributed as dist
+    if dist.get_backend() == "nccl":
+        dist.all_gather_into_tensor(full, local.contiguous())
+    else:
+        parts = list(full.chunk(world, 0))
+        dist.all_gather(parts, local.contiguous())
+        full.copy_(torch.cat(parts, 0))
+    return full
+
+
+def run_strong(args, world, rank, local):
+    """One L=131072 prefill sharded over the ranks by query-row blocks: every step all-gathers
+    the key (k_I, k_scale) and latent rows each rank holds, then runs the fused indexer top-k
+    and sparse MLA on the rank's own rows.  value = L tokens per (slowest rank's) step."""
+    import sparse_attention_09_b200 as dsa
+    cfg = dict(synth.WORKLOADS[args.workload])
+    k, sm, H, H_I, d_I = cfg["k"], 1.0 / math.sqrt(576), cfg["H"], cfg["H_I"], cfg["d_I"]
+    inp = synth.prefill_inputs(device="cuda", **cfg)  # same seed on every rank: rank r keeps its blocks
+    L = inp["q"].shape[0]
+    rb = balanced_row_blocks(L, k, world)
+    q0, q1 = rb[rank], rb[rank + 1]
+    kb = even_row_blocks(L, world)
+    k0, k1 = kb[rank], kb[rank + 1]
+    my_k8, my_ks, my_lat = inp["k8"][k0:k1].clone(), inp["k_scale"][k0:k1].clone(), inp["latent"][k0:k1].clone()
+    keys = dsa.contiguous_desc(inp["k8"], inp["cu_seqlens"], L, scale=inp["k_scale"])
+    lat = dsa.contiguous_desc(inp["latent"], inp["cu_seqlens"], L)
+    R = q1 - q0
+    idx = torch.empty((R, k), dtype=torch.int32, device="cuda")
+    out = torch.empty((R, H, 512), dtype=torch.bfloat16, device="cuda")
+    qb = (inp["q8"][q0:q1], inp["q_scale"][q0:q1], inp["w"][q0:q1], inp["q"][q0:q1])
+
+    def step():
+        gather_rows(my_k8, inp["k8"], world)
+        gather_rows(my_ks, inp["k_scale"], world)
+        gather_rows(my_lat, inp["latent"], world)
+        dsa.dsa_indexer_topk_rows(qb[0], qb[1], qb[2], keys, H_I, d_I, k, q0, q1, idx)
+        dsa.dsa_sparse_mla_prefill_rows(qb[3], lat, idx, H, k, sm, q0, q1, out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert dsa.dsa_device_error() == 0, "device error during warm-up"
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms_per_step = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    assert dsa.dsa_device_error() == 0
+    if rank == 0:
+        line = {"metric": METRIC, "value": L / (ms_per_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
+                "config": {"workload": f"{args.workload}: one sequence sharded by query-row blocks {rb}, "
+                                       "keys and latent all-gathered every step",
+                           "global_batch": 1, "seq_len": L, "k": k, "parallelism": f"row-sharded x{world}",
+                           "l2": "inputs larger than L2; no flush"},
+                "clocks": clk, "gpu_launches": 2 * args.steps}
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, world, rank, local):
     import sparse_attention_09_b200 as dsa
 
@@ -497,6 +595,8 @@ def main():
     ap.add_argument("--workload", default=PREFILL, choices=[w for w, c in synth.WORKLOADS.items() if c["kind"] == "prefill"],
                     help="prefill workload of the timed step (the headline is prefill_128k; smaller ones are for profiling)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--strong", action="store_true",
+                    help="shard ONE sequence over the ranks by query rows (strong scaling) instead of one problem per rank")
     args = ap.parse_args()
     if args.warmup < 3:
         log("warm-up raised to the minimum of 3 steps")
@@ -505,7 +605,10 @@ def main():
         run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
         return
     world, rank, local = dist_setup(args)
-    run_ours(args, world, rank, local)
+    if args.strong:
+        run_strong(args, world, rank, local)
+    else:
+        run_ours(args, world, rank, local)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

@@ -126,6 +126,25 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, int64_t rows, const 
  * Every row must hold at least one valid index.
  */
 /*
+ * Row blocks of one sequence, for sharding a long prefill over GPUs by query rows (each GPU
+ * holds every key and latent row -- gathered from the others -- and its own block of query
+ * rows).  keys / latent describe ONE contiguous sequence (cu_seqlens = {0, L}).
+ *   dsa_indexer_topk_rows: like dsa_indexer_topk for query rows [row_begin, row_end) only;
+ *     q_fp8 [R, H_I, d_I], q_scale [R], w [R, H_I] and idx_out [R, k] hold just those
+ *     R = row_end - row_begin rows (row 0 = query row_begin).
+ *   dsa_sparse_mla_prefill_rows: like dsa_sparse_mla_prefill for rows [row_begin, row_end);
+ *     q [R, H, 576], idx [R, k], out [R, H, 512], lse [R, H] hold just those rows.
+ * Each block's results equal the corresponding rows of the whole-sequence call.  row_begin ==
+ * row_end is a no-op; 0 <= row_begin <= row_end <= L, else DSA_ERR_INVALID_ARGUMENT.
+ */
+dsa_status dsa_indexer_topk_rows(const uint8_t* q_fp8, const float* q_scale, const float* w,
+                                 const dsa_kv_desc* keys, int32_t H_I, int32_t d_I, int32_t k,
+                                 int64_t row_begin, int64_t row_end, int32_t* idx_out, void* stream);
+dsa_status dsa_sparse_mla_prefill_rows(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t H,
+                                       int32_t k, float sm_scale, int64_t row_begin, int64_t row_end, void* out,
+                                       float* lse, void* stream);
+
+/*
  * Masked dense mode of sparse MLA prefill, for short sequences (DeepSeek-V3.2-Exp, "等性能验证":
  * for short prefill a masked MHA mode simulates DSA): the same out/lse as
  * dsa_sparse_mla_prefill for the same arguments, computed by walking every causal 64-key chunk

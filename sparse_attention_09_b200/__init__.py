@@ -33,7 +33,8 @@ DSA_MODE_DECODE = 1
 
 EXPORTED = ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_mla_prefill", "dsa_sparse_mla_decode",
             "dsa_forward", "dsa_workspace_size", "dsa_status_string", "dsa_device_error",
-            "dsa_sparse_mla_decode_noalloc", "dsa_quantize_fp8", "dsa_masked_mla_prefill")
+            "dsa_sparse_mla_decode_noalloc", "dsa_quantize_fp8", "dsa_masked_mla_prefill",
+            "dsa_indexer_topk_rows", "dsa_sparse_mla_prefill_rows")
 
 
 class KVDesc(ctypes.Structure):
@@ -78,6 +79,10 @@ _lib.dsa_indexer_topk.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I32, _P,
 _lib.dsa_indexer_topk.restype = _I32
 _lib.dsa_sparse_mla_decode_noalloc.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P]
 _lib.dsa_sparse_mla_decode_noalloc.restype = _I32
+_lib.dsa_indexer_topk_rows.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I64, _I64, _P, _P]
+_lib.dsa_indexer_topk_rows.restype = _I32
+_lib.dsa_sparse_mla_prefill_rows.argtypes = [_P, _DESC, _P, _I32, _I32, _F32, _I64, _I64, _P, _P, _P]
+_lib.dsa_sparse_mla_prefill_rows.restype = _I32
 _lib.dsa_masked_mla_prefill.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P]
 _lib.dsa_masked_mla_prefill.restype = _I32
 _lib.dsa_quantize_fp8.argtypes = [_P, _I64, _I32, _P, _P, _P]
@@ -164,6 +169,22 @@ def dsa_indexer_scores(q_fp8, q_scale, w, keys: Desc, B, H_I, d_I, row_begin, ro
                                    int(row_begin), int(row_end), _ptr(scores), scores.stride(0), _stream(stream)),
            "dsa_indexer_scores")
     return scores
+
+
+def dsa_indexer_topk_rows(q_fp8, q_scale, w, keys: Desc, H_I, d_I, k, row_begin, row_end, idx, stream=None):
+    """Fused indexer + top-k for query rows [row_begin, row_end) of one sequence; the query
+    arrays and idx hold just those rows."""
+    _check(_lib.dsa_indexer_topk_rows(_ptr(q_fp8), _ptr(q_scale), _ptr(w), keys.ref(), int(H_I), int(d_I), int(k),
+                                      int(row_begin), int(row_end), _ptr(idx), _stream(stream)), "dsa_indexer_topk_rows")
+    return idx
+
+
+def dsa_sparse_mla_prefill_rows(q, latent: Desc, idx, H, k, sm_scale, row_begin, row_end, out, lse=None, stream=None):
+    """Sparse MLA prefill for query rows [row_begin, row_end) of one sequence."""
+    _check(_lib.dsa_sparse_mla_prefill_rows(_ptr(q), latent.ref(), _ptr(idx), int(H), int(k), float(sm_scale),
+                                            int(row_begin), int(row_end), _ptr(out), _ptr(lse), _stream(stream)),
+           "dsa_sparse_mla_prefill_rows")
+    return out
 
 
 def dsa_masked_mla_prefill(q, latent: Desc, idx, B, H, k, sm_scale, out, lse=None, stream=None):

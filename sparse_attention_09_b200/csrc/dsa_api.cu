@@ -94,9 +94,10 @@ dsa_status launch_indexer(int d_I, int H_I, const CUtensorMap& qm, const CUtenso
 bool indexer_shape_ok(int H_I, int d_I) { return (H_I == 4 || H_I == 64) && (d_I == 64 || d_I == 128); }
 
 // Validates the common indexer arguments and builds the Q / K tensor maps.
+// q_rows: rows held by the query arrays (prefill: the packed tokens they cover; 0 = all of them)
 dsa_status indexer_common(const uint8_t* q_fp8, const float* q_scale, const float* w, const dsa_kv_desc* keys,
                           int32_t B, int32_t H_I, int32_t d_I, CUtensorMap* qm, CUtensorMap* km,
-                          IndexerParams* p) {
+                          IndexerParams* p, int64_t q_rows = 0) {
   if (q_fp8 == nullptr || q_scale == nullptr || w == nullptr || keys == nullptr || keys->data == nullptr ||
       keys->scale == nullptr || B <= 0)
     return DSA_ERR_INVALID_ARGUMENT;
@@ -104,6 +105,9 @@ dsa_status indexer_common(const uint8_t* q_fp8, const float* q_scale, const floa
   if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED;
   const CUtensorMapSwizzle sw = d_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   std::memset(p, 0, sizeof(*p));
+  p->tok_begin = 0;
+  p->tok_end = 0x7FFFFFFF;
+  p->q_row0 = 0;
   p->q_scale = q_scale;
   p->w = w;
   p->k_scale = keys->scale;
@@ -111,7 +115,8 @@ dsa_status indexer_common(const uint8_t* q_fp8, const float* q_scale, const floa
     if (keys->cu_seqlens == nullptr || keys->total_tokens <= 0 || keys->max_seqlen <= 0) return DSA_ERR_INVALID_ARGUMENT;
     if (keys->total_tokens * H_I > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
     const uint64_t T = static_cast<uint64_t>(keys->total_tokens);
-    if (!make_map_2d(qm, q_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, d_I, T * H_I, d_I, d_I, kIdxTok * H_I, sw) ||
+    const uint64_t TQ = q_rows > 0 ? static_cast<uint64_t>(q_rows) : T;
+    if (!make_map_2d(qm, q_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, d_I, TQ * H_I, d_I, d_I, kIdxTok * H_I, sw) ||
         !make_map_2d(km, keys->data, CU_TENSOR_MAP_DATA_TYPE_UINT8, d_I, T, d_I, d_I, 128, sw))
       return DSA_ERR_INVALID_ARGUMENT;
     p->cu_seqlens = keys->cu_seqlens;
@@ -303,6 +308,63 @@ dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, const fl
   if (p.cap > kIdxCapMax) p.cap = kIdxCapMax;
   dim3 grid((keys->max_seqlen + kIdxTok - 1) / kIdxTok, B);
   return launch_indexer<kIdxTopk, false>(d_I, H_I, qm, km, p, grid, as_stream(stream));
+}
+
+dsa_status dsa_indexer_topk_rows(const uint8_t* q_fp8, const float* q_scale, const float* w, const dsa_kv_desc* keys,
+                                 int32_t H_I, int32_t d_I, int32_t k, int64_t row_begin, int64_t row_end,
+                                 int32_t* idx_out, void* stream) {
+  if (keys == nullptr || k <= 0 || row_begin < 0 || row_end < row_begin) return DSA_ERR_INVALID_ARGUMENT;
+  if (keys->kind != DSA_KV_CONTIGUOUS) return DSA_ERR_UNSUPPORTED;
+  if (k > 2048) return DSA_ERR_UNSUPPORTED;
+  if (row_end > keys->total_tokens) return DSA_ERR_INVALID_ARGUMENT;
+  if (row_end == row_begin) return DSA_OK;  // an empty block: nothing to read or write
+  if (idx_out == nullptr) return DSA_ERR_INVALID_ARGUMENT;
+  CUtensorMap qm, km;
+  IndexerParams p;
+  dsa_status st = indexer_common(q_fp8, q_scale, w, keys, 1, H_I, d_I, &qm, &km, &p, row_end - row_begin);
+  if (st != DSA_OK) return st;
+  const int64_t bitmap_bytes = (static_cast<int64_t>(keys->max_seqlen) + 31) / 32 * 4;
+  if (bitmap_bytes > static_cast<int64_t>(kIdxStagesTopk) * 128 * d_I / 2 || keys->max_seqlen > (1 << 24))
+    return DSA_ERR_UNSUPPORTED;
+  p.idx_out = idx_out;
+  p.k = k;
+  p.cap = k + 1024 < 2 * k ? 2 * k : k + 1024;
+  if (p.cap > kIdxCapMax) p.cap = kIdxCapMax;
+  p.tok_begin = static_cast<int32_t>(row_begin);
+  p.tok_end = static_cast<int32_t>(row_end);
+  p.q_row0 = row_begin;
+  dim3 grid(static_cast<unsigned>((row_end - row_begin + kIdxTok - 1) / kIdxTok), 1);
+  return launch_indexer<kIdxTopk, false>(d_I, H_I, qm, km, p, grid, as_stream(stream));
+}
+
+dsa_status dsa_sparse_mla_prefill_rows(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t H,
+                                       int32_t k, float sm_scale, int64_t row_begin, int64_t row_end, void* out,
+                                       float* lse, void* stream) {
+  if (latent == nullptr || latent->kind != DSA_KV_CONTIGUOUS || latent->cu_seqlens == nullptr ||
+      latent->total_tokens <= 0)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (row_begin < 0 || row_end < row_begin || row_end > latent->total_tokens) return DSA_ERR_INVALID_ARGUMENT;
+  if (row_end == row_begin) return DSA_OK;  // an empty block: nothing to read or write
+  if (q == nullptr || latent->data == nullptr || idx == nullptr || out == nullptr) return DSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(latent->data, 16) || !aligned(idx, 16) || !aligned(out, 16))
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (!mla_shape_ok(H, k)) return DSA_ERR_UNSUPPORTED;
+  if (latent->total_tokens > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+  MlaParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.idx = idx;
+  p.cu_seqlens = latent->cu_seqlens;
+  p.B = 1;
+  p.H = H;
+  p.k = k;
+  p.rows = row_end - row_begin;
+  p.unit0 = row_begin;
+  p.splits = 1;
+  p.scale_log2 = sm_scale * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  return launch_mla<false>(latent->data, p, p.rows, as_stream(stream));
 }
 
 dsa_status dsa_sparse_mla_prefill(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B, int32_t H,

@@ -48,6 +48,8 @@ struct IndexerParams {
   int64_t ld;
   int64_t row_begin, row_end;
   int32_t* idx_out;           // kIdxTopk output [T, k]
+  int32_t tok_begin, tok_end; // top-k prefill: token positions [tok_begin, tok_end) of each sequence
+  int64_t q_row0;             // prefill: packed row held by row 0 of q / q_scale / w / idx_out
   int32_t k;
   int32_t cap;                // candidate capacity per token (kIdxTopk)
 };
@@ -127,11 +129,12 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
   if constexpr (!PAGED) {
     const int seq_start = p.cu_seqlens[b];
     len = p.cu_seqlens[b + 1] - seq_start;
-    const int nblk = (len + TOK - 1) / TOK;
-    const int tb = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);  // heavy blocks first
-    if (tb >= nblk) return;
-    t0 = tb * TOK;
-    ntok = min(TOK, len - t0);
+    // tokens [tok_begin, min(len, tok_end)) of the sequence, TOK per CTA, heavy blocks first
+    const int tend = min(len, p.tok_end);
+    const int tb = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);
+    t0 = p.tok_begin + tb * TOK;
+    if (t0 >= tend) return;
+    ntok = min(TOK, tend - t0);
     if (MODE == kIdxScores) {
       const int64_t g0 = seq_start + t0, g1 = g0 + ntok;
       if (g1 <= p.row_begin || g0 >= p.row_end) return;
@@ -139,7 +142,7 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
     tile0 = 0;
     ntiles = (t0 + ntok - 1) / 128 + 1;
     key_row0 = seq_start;
-    q_row = static_cast<int64_t>(seq_start + t0) * H_I;
+    q_row = (static_cast<int64_t>(seq_start + t0) - p.q_row0) * H_I;
   } else {
     if (b < p.row_begin || b >= p.row_end) return;
     len = min(p.context_lens[b], p.max_blocks_per_seq * 64);  // never read past the block table row
@@ -175,7 +178,7 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
     const int tt = i / H_I, j = i % H_I;
     float v = 0.f;
     if (tt < ntok) {
-      const int64_t row = PAGED ? b : (p.cu_seqlens[b] + t0 + tt);
+      const int64_t row = PAGED ? b : (p.cu_seqlens[b] + t0 + tt - p.q_row0);
       v = p.w[row * H_I + j] * p.q_scale[row];
     }
     sWq[i] = v;
@@ -466,7 +469,7 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
           if (thr[tt] >= 0) lo = min(lo, static_cast<uint32_t>(thr[tt]));  // the smallest kept key
           sel::Cands C{sCandKey + tok * p.cap, sCandIdx + tok * p.cap, &s_cnt[tok][0], Q};
           sel::cut_final(G, C, s_sel[g], min(p.k, t + 1), lo, hi);
-          sel::emit_sorted(G, C, s_sel[g], bitmap, t + 1, p.idx_out + static_cast<int64_t>(seq_start + t) * p.k, p.k);
+          sel::emit_sorted(G, C, s_sel[g], bitmap, t + 1, p.idx_out + (static_cast<int64_t>(seq_start + t) - p.q_row0) * p.k, p.k);
         }
       }
     }

@@ -61,7 +61,8 @@ struct MlaParams {
   int32_t B;
   int32_t H;                  // query heads (<= 128; rows >= H are padding)
   int32_t k;                  // selected entries per row (multiple of 64)
-  int64_t rows;               // prefill: total tokens; decode: B
+  int64_t rows;               // prefill: tokens (units) to process; decode: B
+  int64_t unit0;              // prefill: packed token of unit 0 (row 0 of q, idx, out, lse)
   int32_t splits;             // decode: selection splits per sequence
   float scale_log2;           // sm_scale * log2(e)
   __nv_bfloat16* out;         // prefill: [rows, H, 512]
@@ -224,14 +225,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       seq_start = 0;
       seq_len = min(p.context_lens[seq], p.max_blocks_per_seq * 64);
     } else {
-      qrow = u;
+      qrow = u;  // row of q, idx, out and lse
       kbeg = 0;
       kend = p.k;
-      // sequence of token u: binary search in cu_seqlens
+      // sequence of packed token u + unit0: binary search in cu_seqlens
+      const int64_t gtok = u + p.unit0;
       int lo = 0, hi = p.B;
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (p.cu_seqlens[mid] <= u) lo = mid;
+        if (p.cu_seqlens[mid] <= gtok) lo = mid;
         else hi = mid;
       }
       seq = lo;
@@ -244,7 +246,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
   auto unit_chunks = [&](int64_t qrow, int kbeg, int kend, int seq_start, int& c0, int& c1) {
     if constexpr (DENSE) {
       c0 = 0;
-      c1 = static_cast<int>(qrow - seq_start) / kChunk + 1;
+      c1 = static_cast<int>(qrow + p.unit0 - seq_start) / kChunk + 1;
       return;
     }
     const int act = active_chunks(p.idx + qrow * p.k, p.k);
@@ -270,7 +272,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
         int kbeg, kend, seq, seq_start, seq_len, c0, c1;
         unit_info(u, qrow, kbeg, kend, seq, seq_start, seq_len);
         unit_chunks(qrow, kbeg, kend, seq_start, c0, c1);
-        const int t = static_cast<int>(qrow - seq_start);
+        const int t = static_cast<int>(qrow + p.unit0 - seq_start);
         const int32_t* row = p.idx + qrow * p.k;
         int pos = 0;  // entries of the row consumed by earlier chunks
         for (int c = c0; c < c1; ++c, ++g) {

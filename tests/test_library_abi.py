@@ -60,3 +60,21 @@ def test_quantiser_host_validation():
     assert lib.dsa_quantize_fp8(null, 4, 8, a, a, null) == dsa.DSA_ERR_INVALID_ARGUMENT
     assert lib.dsa_quantize_fp8(ctypes.c_void_p(4104), 4, 8, a, a, null) == dsa.DSA_ERR_INVALID_ARGUMENT  # 16 B
     assert lib.dsa_quantize_fp8(a, 4, 8, ctypes.c_void_p(4100), a, null) == dsa.DSA_ERR_INVALID_ARGUMENT  # 8 B
+
+
+def test_row_block_entries_host_validation():
+    import sparse_attention_09_b200 as dsa
+    lib = dsa._lib
+    null = ctypes.c_void_p(0)
+    cu = ctypes.c_void_p(4096)
+    d = dsa.KVDesc(dsa.DSA_KV_CONTIGUOUS, 4096, 4096, 4096, 0, 0, 100, 100, 0, 0, 0)
+    ref = ctypes.byref(d)
+    # empty blocks are no-ops even with NULL row arrays
+    assert lib.dsa_indexer_topk_rows(null, null, null, ref, 64, 128, 2048, 40, 40, null, null) == dsa.DSA_OK
+    assert lib.dsa_sparse_mla_prefill_rows(null, ref, null, 128, 2048, ctypes.c_float(0.04), 40, 40, null, null,
+                                           null) == dsa.DSA_OK
+    # bad ranges
+    assert lib.dsa_indexer_topk_rows(cu, cu, cu, ref, 64, 128, 2048, 50, 40, cu, null) == dsa.DSA_ERR_INVALID_ARGUMENT
+    assert lib.dsa_indexer_topk_rows(cu, cu, cu, ref, 64, 128, 2048, 0, 101, cu, null) == dsa.DSA_ERR_INVALID_ARGUMENT
+    assert lib.dsa_sparse_mla_prefill_rows(cu, ref, cu, 128, 2048, ctypes.c_float(0.04), -1, 4, cu, null,
+                                           null) == dsa.DSA_ERR_INVALID_ARGUMENT
