@@ -35,6 +35,10 @@ Parity status per function (what pins it, in ``tests/test_oracle_*.py``):
   library routine; single-row, equal-rows and uniform-logit closed forms; permutation
   invariance).
 * ``paged_gather`` / decode functions: pinned (paged layout equals the contiguous result).
+* ``attention_distribution_token`` / ``indexer_kl``: pinned (a distribution summing to 1, one
+  head = the softmax of its logits, equal logits = uniform, head-permutation invariance; KL >= 0,
+  0 exactly when the scores are log p plus a constant, the gradient sums to 0 and matches
+  central finite differences of the loss, and a two-point closed form).
 * ``encode_e4m3`` / ``quantize_fp8_rows``: pinned (every finite code round-trips; midpoints
   between neighbouring values go to the even code; saturation and NaN; agreement with torch's
   float8_e4m3fn cast on random values; the per-row scale rule and its error bound).
@@ -55,6 +59,8 @@ from .dsa_oracle import (  # noqa: F401
     topk_rows,
     sparse_mla_token,
     sparse_mla,
+    attention_distribution_token,
+    indexer_kl,
     paged_gather,
     decode_indexer_scores,
     dsa_prefill_rows,

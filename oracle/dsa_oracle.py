@@ -27,7 +27,7 @@ E4M3_MAX = 448.0
 
 
 # ---------------------------------------------------------------------------------------------
-# FP8 e4m3 ([MZ] "工作原理": the indexer "can run in FP8"; [JD] 2.1: "FP8低精度计算")
+# FP8 e4m3 ([MZ] "工作原理": the indexer may run in FP8; [JD] 2.1: low-precision FP8 compute)
 # ---------------------------------------------------------------------------------------------
 def e4m3_table() -> np.ndarray:
     """Value of every byte under OCP E4M3FN, written from the format definition.
@@ -197,6 +197,37 @@ def sparse_mla_token(q: np.ndarray, latent: np.ndarray, sel: np.ndarray, sm_scal
     out = (e / z) @ c[:, :dv]
     lse = mx[:, 0] + np.log(z[:, 0])
     return out, lse
+
+
+def attention_distribution_token(q: np.ndarray, latent: np.ndarray, sel: np.ndarray, sm_scale: float):
+    """The main attention's distribution over a token's selected rows, aggregated over heads:
+    p[i] = (1/H) sum_h softmax_i(sm_scale * q[h] . c[sel_i]) -- the target the indexer's
+    distribution is aligned to by the KL loss ([MZ] 二, the two training stages of the indexer:
+    a KL-divergence loss pulls the indexer's output distribution towards the main attention's;
+    in the sparse stage over the selected set).
+    Reading: "the main attention's distribution" of a query = its per-head attention
+    probabilities summed over heads and normalised to total 1 (= the mean over heads).
+    q: [H, D], latent: [n, D], sel: selected rows (no padding).  Returns float64 [len(sel)].
+    """
+    c = np.asarray(latent, np.float64)[np.asarray(sel, np.int64)]
+    logits = float(sm_scale) * (np.asarray(q, np.float64) @ c.T)     # [H, m]
+    mx = logits.max(axis=1, keepdims=True)
+    e = np.exp(logits - mx)
+    return (e / e.sum(axis=1, keepdims=True)).mean(axis=0)
+
+
+def indexer_kl(p: np.ndarray, scores: np.ndarray):
+    """KL alignment loss of one token and its gradient ([MZ] 二, training of the indexer):
+    q = softmax(scores) over the same rows as the target p;
+    loss = KL(p || q) = sum_i p_i (log p_i - log q_i) (terms with p_i = 0 contribute 0);
+    d loss / d scores_i = q_i - p_i.  Returns (loss float64, grad float64 [m])."""
+    p = np.asarray(p, np.float64)
+    s = np.asarray(scores, np.float64)
+    mx = s.max()
+    logq = s - mx - np.log(np.exp(s - mx).sum())
+    pos = p > 0
+    loss = float(np.sum(p[pos] * (np.log(p[pos]) - logq[pos])))
+    return loss, np.exp(logq) - p
 
 
 def sparse_mla(q: np.ndarray, latent: np.ndarray, idx: np.ndarray, sm_scale: float, rows=None,
