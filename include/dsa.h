@@ -145,8 +145,8 @@ dsa_status dsa_sparse_mla_prefill_rows(const void* q, const dsa_kv_desc* latent,
                                        float* lse, void* stream);
 
 /*
- * Masked dense mode of sparse MLA prefill, for short sequences (DeepSeek-V3.2-Exp, "等性能验证":
- * for short prefill a masked MHA mode simulates DSA): the same out/lse as
+ * Masked dense mode of sparse MLA prefill, for short sequences ("DeepSeek-V3.2 论文解读",
+ * section 二, subsection "等性能验证": for short prefill a masked MHA mode simulates DSA): the same out/lse as
  * dsa_sparse_mla_prefill for the same arguments, computed by walking every causal 64-key chunk
  * of the contiguous latent with TMA tiles and masking the keys idx does not select.  Cost grows
  * with L^2 instead of L*k, so it pays only when most causal keys are selected (L up to ~2k).
@@ -221,7 +221,7 @@ dsa_status dsa_device_error(int32_t* code, void* stream);
 
 /*
  * Per-token FP8 quantiser for the indexer operands (the step that produces a2's input
- * contract; DeepSeek-V3.2-Exp, "Lightning Indexer": the indexer runs in FP8).  For each row r
+ * contract; "DeepSeek-V3.2 论文解读", section 二, subsection "工作原理": the indexer runs in FP8).  For each row r
  * of x [rows, cols] bf16 (row-major, contiguous; one token: all of its indexer heads for
  * q_I, its key for k_I):
  *   scale[r] = amax_c |x[r,c]| / 448 in IEEE fp32 (1 for an all-zero row),

@@ -1,7 +1,7 @@
 // Per-token FP8 (e4m3) quantiser for the lightning indexer's operands.
 //
-// The indexer runs in FP8 with one fp32 scale per token (DeepSeek-V3.2-Exp, "Lightning
-// Indexer": the indexer may run in FP8).  For a token row x (all of its indexer heads for
+// The indexer runs in FP8 with one fp32 scale per token ("DeepSeek-V3.2 论文解读", section 二,
+// subsection "工作原理": the indexer may run in FP8).  For a token row x (all of its indexer heads for
 // q_I, its single key for k_I):
 //   scale = amax(|x|) / 448   (1 for an all-zero row),   codes = e4m3(x / scale)
 // with both divisions in IEEE fp32 and the e4m3 encoding rounding to nearest-even, saturating

@@ -41,9 +41,9 @@
 //
 // And the masked dense mode for short prefill (DENSE): the same attention over the selected
 // rows, computed by walking every causal 64-key chunk of the contiguous latent (loaded with
-// TMA tiles instead of a gather) and masking the keys the selection does not hold, as the
-// pages describe for short sequences (dense attention with a mask simulating the sparse
-// pattern).  The selection rows must be ascending (as the top-k emits them).
+// TMA tiles instead of a gather) and masking the keys the selection does not hold: the mode
+// "DeepSeek-V3.2 论文解读" (section 二, subsection "等性能验证") describes for short prefill
+// (dense attention with a mask that simulates the sparse pattern).  The selection rows must be ascending (as the top-k emits them).
 #pragma once
 
 #include "common.cuh"
