@@ -369,7 +369,8 @@ def run_ours(args, world, rank, local):
 
     # ---- decode chain, same process ----
     decode = run_decode(args, dsa, sm) if (rank == 0 and not args.no_decode) else None
-    next_rows = ({"f1_quantize_fp8": run_quantizer(dsa, peaks), "f2_masked_mla": run_masked(dsa, sm)}
+    next_rows = ({"f1_quantize_fp8": run_quantizer(dsa, peaks), "f2_masked_mla": run_masked(dsa, sm),
+                  "f3_indexer_kl": run_kl(dsa, inp, idx, cfg, sm)}
                  if (rank == 0 and not args.no_decode) else None)
 
     # ---- end to end through dsa_forward with host buffers ----
@@ -464,6 +465,45 @@ def run_masked(dsa, sm):
         out[f"L{L}"] = row
     assert dsa.dsa_device_error() == 0
     return out
+
+
+def run_kl(dsa, inp, idx, cfg, sm):
+    """NEXT row f3: the indexer's KL alignment on the full prefill: the head-averaged attention
+    distribution over each token's selection (from the forward's lse) and KL(p || softmax(I))
+    with its gradient.  The indexer scores at the selected rows are a synthetic stand-in here
+    (the loss kernel's cost does not depend on their values)."""
+    T, H, k = inp["q"].shape[0], cfg["H"], cfg["k"]
+    lat = dsa.contiguous_desc(inp["latent"], inp["cu_seqlens"], max(inp["seqlens"]))
+    nseq = len(cfg["seqlens"])
+    out = torch.empty((T, H, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((T, H), device="cuda")
+    dsa.dsa_sparse_mla_prefill(inp["q"], lat, idx, nseq, H, k, sm, out, lse)
+    del out
+    p = torch.empty((T, k), device="cuda")
+    scores = torch.randn((T, k), device="cuda")
+    loss = torch.empty((T,), device="cuda")
+    grad = torch.empty((T, k), device="cuda")
+    res = {}
+    for name, fn in (("attn_distribution", lambda: dsa.dsa_attn_distribution(inp["q"], lat, idx, lse, nseq, H, k, sm, p)),
+                     ("indexer_kl", lambda: dsa.dsa_indexer_kl(p, scores, idx, loss, grad))):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(3):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        res[name + "_ms"] = e0.elapsed_time(e1) / 3
+    pairs = sum(min(k, t + 1) for s in cfg["seqlens"] for t in range(s))
+    res["attn_distribution_tflops"] = pairs * 2 * H * 576 / (res["attn_distribution_ms"] * 1e-3) / 1e12
+    res["indexer_kl_gbs"] = T * k * 4 * 4 / (res["indexer_kl_ms"] * 1e-3) / 1e9  # p, scores, idx read; grad written
+    res["mean_row_sum_p"] = float(p.sum(dim=1).mean().item())
+    assert dsa.dsa_device_error() == 0
+    del p, scores, loss, grad, lse
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_decode(args, dsa, sm):

@@ -220,6 +220,26 @@ const char* dsa_status_string(int32_t status);
 dsa_status dsa_device_error(int32_t* code, void* stream);
 
 /*
+ * Indexer KL alignment (the training-side step next to the indexer; "DeepSeek-V3.2 论文解读",
+ * section 二: a KL loss aligns the indexer's distribution with the main attention's; in the
+ * sparse stage over each token's selected rows).
+ *   dsa_attn_distribution: p_out[t*k + i] = (1/H) sum_h exp(sm_scale * q[t,h,:] . c[idx[t,i],:]
+ *     - lse[t,h]) for valid entries (idx >= 0 and inside the sequence), 0 otherwise: the
+ *     head-averaged attention distribution over the selected rows.  q [T, H, 576] bf16, latent
+ *     contiguous [T, 576] bf16 with cu_seqlens, idx [T, k] (k a multiple of 64, <= 2048), lse
+ *     [T, H] fp32 natural log as dsa_sparse_mla_prefill writes it; p_out [T, k] fp32.
+ *   dsa_indexer_kl: per row r over the valid entries (idx >= 0): q = softmax(scores[r,:]),
+ *     loss[r] = sum_i p_i (log p_i - log q_i) (p_i = 0 adds nothing), grad[r*k + i] = q_i - p_i
+ *     (0 for invalid entries); a row without valid entries gets loss 0.  fp32 [rows, k] inputs.
+ * Device pointers, caller-owned outputs, asynchronous on `stream`; DSA_ERR_INVALID_ARGUMENT for
+ * NULL / misaligned pointers, DSA_ERR_UNSUPPORTED outside the stated shapes.
+ */
+dsa_status dsa_attn_distribution(const void* q, const dsa_kv_desc* latent, const int32_t* idx, const float* lse,
+                                 int32_t B, int32_t H, int32_t k, float sm_scale, float* p_out, void* stream);
+dsa_status dsa_indexer_kl(const float* p, const float* scores, const int32_t* idx, int64_t rows, int32_t k,
+                          float* loss, float* grad, void* stream);
+
+/*
  * Per-token FP8 quantiser for the indexer operands (the step that produces a2's input
  * contract; "DeepSeek-V3.2 论文解读", section 二, subsection "工作原理": the indexer runs in FP8).  For each row r
  * of x [rows, cols] bf16 (row-major, contiguous; one token: all of its indexer heads for

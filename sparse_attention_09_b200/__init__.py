@@ -34,7 +34,7 @@ DSA_MODE_DECODE = 1
 EXPORTED = ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_mla_prefill", "dsa_sparse_mla_decode",
             "dsa_forward", "dsa_workspace_size", "dsa_status_string", "dsa_device_error",
             "dsa_sparse_mla_decode_noalloc", "dsa_quantize_fp8", "dsa_masked_mla_prefill",
-            "dsa_indexer_topk_rows", "dsa_sparse_mla_prefill_rows")
+            "dsa_indexer_topk_rows", "dsa_sparse_mla_prefill_rows", "dsa_attn_distribution", "dsa_indexer_kl")
 
 
 class KVDesc(ctypes.Structure):
@@ -79,6 +79,10 @@ _lib.dsa_indexer_topk.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I32, _P,
 _lib.dsa_indexer_topk.restype = _I32
 _lib.dsa_sparse_mla_decode_noalloc.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P]
 _lib.dsa_sparse_mla_decode_noalloc.restype = _I32
+_lib.dsa_attn_distribution.argtypes = [_P, _DESC, _P, _P, _I32, _I32, _I32, _F32, _P, _P]
+_lib.dsa_attn_distribution.restype = _I32
+_lib.dsa_indexer_kl.argtypes = [_P, _P, _P, _I64, _I32, _P, _P, _P]
+_lib.dsa_indexer_kl.restype = _I32
 _lib.dsa_indexer_topk_rows.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I64, _I64, _P, _P]
 _lib.dsa_indexer_topk_rows.restype = _I32
 _lib.dsa_sparse_mla_prefill_rows.argtypes = [_P, _DESC, _P, _I32, _I32, _F32, _I64, _I64, _P, _P, _P]
@@ -169,6 +173,21 @@ def dsa_indexer_scores(q_fp8, q_scale, w, keys: Desc, B, H_I, d_I, row_begin, ro
                                    int(row_begin), int(row_end), _ptr(scores), scores.stride(0), _stream(stream)),
            "dsa_indexer_scores")
     return scores
+
+
+def dsa_attn_distribution(q, latent: Desc, idx, lse, B, H, k, sm_scale, p_out, stream=None):
+    """p_out[t, i] = head-averaged attention probability of the selected row idx[t, i]."""
+    _check(_lib.dsa_attn_distribution(_ptr(q), latent.ref(), _ptr(idx), _ptr(lse), int(B), int(H), int(k),
+                                      float(sm_scale), _ptr(p_out), _stream(stream)), "dsa_attn_distribution")
+    return p_out
+
+
+def dsa_indexer_kl(p, scores, idx, loss, grad, stream=None):
+    """loss[r] = KL(p[r] || softmax(scores[r])) over valid entries; grad = softmax(scores) - p."""
+    rows, k = p.shape
+    _check(_lib.dsa_indexer_kl(_ptr(p), _ptr(scores), _ptr(idx), int(rows), int(k), _ptr(loss), _ptr(grad),
+                               _stream(stream)), "dsa_indexer_kl")
+    return loss, grad
 
 
 def dsa_indexer_topk_rows(q_fp8, q_scale, w, keys: Desc, H_I, d_I, k, row_begin, row_end, idx, stream=None):

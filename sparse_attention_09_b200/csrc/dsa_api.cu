@@ -13,6 +13,8 @@
 #include "common.cuh"
 #include "indexer.cuh"
 #include "quantize.cuh"
+#include "attn_probs.cuh"
+#include "indexer_kl.cuh"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
 
@@ -229,6 +231,47 @@ dsa_status dsa_device_error(int32_t* code, void* stream) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return DSA_ERR_CUDA;
   *code = v;
   return DSA_OK;
+}
+
+dsa_status dsa_attn_distribution(const void* q, const dsa_kv_desc* latent, const int32_t* idx, const float* lse,
+                                 int32_t B, int32_t H, int32_t k, float sm_scale, float* p_out, void* stream) {
+  if (q == nullptr || latent == nullptr || latent->data == nullptr || idx == nullptr || lse == nullptr ||
+      p_out == nullptr || B <= 0)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (latent->kind != DSA_KV_CONTIGUOUS || latent->cu_seqlens == nullptr || latent->total_tokens <= 0)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(latent->data, 16)) return DSA_ERR_INVALID_ARGUMENT;
+  if (H < 1 || H > 128 || k < 64 || k > 2048 || k % 64 != 0) return DSA_ERR_UNSUPPORTED;
+  ProbsParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.idx = idx;
+  p.lse = lse;
+  p.cu_seqlens = latent->cu_seqlens;
+  p.B = B;
+  p.H = H;
+  p.k = k;
+  p.rows = latent->total_tokens;
+  p.scale_log2 = sm_scale * 1.4426950408889634f;
+  p.p = p_out;
+  const int smem = probs::kSmemBytes + 1024;
+  if (cudaFuncSetAttribute(attn_probs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  const int64_t grid = p.rows < 148 ? p.rows : 148;
+  attn_probs_kernel<<<static_cast<unsigned>(grid), probs::kThreads, smem, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(latent->data), p);
+  return launch_status();
+}
+
+dsa_status dsa_indexer_kl(const float* p, const float* scores, const int32_t* idx, int64_t rows, int32_t k,
+                          float* loss, float* grad, void* stream) {
+  if (rows < 0 || k <= 0) return DSA_ERR_INVALID_ARGUMENT;
+  if (rows == 0) return DSA_OK;
+  if (p == nullptr || scores == nullptr || idx == nullptr || loss == nullptr || grad == nullptr)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (rows > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+  indexer_kl_kernel<<<static_cast<unsigned>(rows), kl::kThreads, 0, as_stream(stream)>>>(p, scores, idx, k, loss, grad);
+  return launch_status();
 }
 
 dsa_status dsa_quantize_fp8(const void* x_bf16, int64_t rows, int32_t cols, uint8_t* codes, float* scale,
