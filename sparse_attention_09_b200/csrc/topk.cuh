@@ -4,7 +4,8 @@
 // scores (8 bits per pass, warp-private histograms) finds the key of the k-th largest entry
 // and how many entries equal to it are still needed; an emit pass then walks the row in
 // index order and writes the selected indices with a block-wide scan, so the output is
-// ascending and ties at the boundary go to the lowest indices.
+// ascending and ties at the boundary go to the lowest indices.  Each thread takes 16
+// consecutive scores per step (four 16-byte loads in flight), so a step covers 8192 scores.
 #pragma once
 
 #include "common.cuh"
@@ -13,7 +14,22 @@ namespace dsa {
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kTopkTile = 4 * kTopkThreads;  // one float4 per thread per step
+constexpr int kTopkVec = 4;                               // float4 loads per thread per step
+constexpr int kTopkTile = 4 * kTopkVec * kTopkThreads;    // scores per step
+
+// The 16 scores [i0, i0 + 16) of a row of length n (entries past n are not loaded; a row
+// buffer of ld >= n elements, ld % 4 == 0, holds every float4 that starts before n).
+__device__ __forceinline__ void topk_load16(const float* row, int i0, int n, float (&f)[16]) {
+#pragma unroll
+  for (int v = 0; v < kTopkVec; ++v) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i0 + 4 * v < n) x = *reinterpret_cast<const float4*>(row + i0 + 4 * v);
+    f[4 * v] = x.x;
+    f[4 * v + 1] = x.y;
+    f[4 * v + 2] = x.z;
+    f[4 * v + 3] = x.w;
+  }
+}
 
 __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const float* __restrict__ scores, int64_t ld,
                                                                  const int32_t* __restrict__ row_len, int32_t k,
@@ -42,12 +58,12 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const float* __
     __syncthreads();
 #pragma unroll 1
     for (int base = 0; base < n; base += kTopkTile) {
-      const int i0 = base + 4 * tid;
+      const int i0 = base + 16 * tid;
       if (i0 < n) {
-        const float4 v = *reinterpret_cast<const float4*>(row + i0);
-        const float f[4] = {v.x, v.y, v.z, v.w};
+        float f[16];
+        topk_load16(row, i0, n, f);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 16; ++j) {
           if (i0 + j < n) {
             if (pass == 0 && is_nan_bits(__float_as_uint(f[j]))) record_device_error(DSA_ERR_DEVICE_CHECK);
             const uint32_t key = order_key(f[j]);
@@ -100,38 +116,35 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const float* __
   int eq_taken = 0, out_pos = 0;
 #pragma unroll 1
   for (int base = 0; base < n && out_pos < k; base += kTopkTile) {
-    const int i0 = base + 4 * tid;
-    bool g[4] = {false, false, false, false}, e[4] = {false, false, false, false};
+    const int i0 = base + 16 * tid;
+    uint32_t gbits = 0u, ebits = 0u;  // bit j: score i0 + j is above / equal to the threshold
     if (i0 < n) {
-      const float4 v = *reinterpret_cast<const float4*>(row + i0);
-      const float f[4] = {v.x, v.y, v.z, v.w};
+      float f[16];
+      topk_load16(row, i0, n, f);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 16; ++j) {
         if (i0 + j < n) {
           const uint32_t key = order_key(f[j]);
-          g[j] = key > thr;
-          e[j] = key == thr;
+          gbits |= static_cast<uint32_t>(key > thr) << j;
+          ebits |= static_cast<uint32_t>(key == thr) << j;
         }
       }
     }
-    const int ne = int(e[0]) + int(e[1]) + int(e[2]) + int(e[3]);
     int tie_total;
-    int tie_rank = eq_taken + block_exclusive_scan<kTopkWarps>(ne, scan_scratch, tie_total);
-    bool sel[4];
+    int tie_rank = eq_taken + block_exclusive_scan<kTopkWarps>(__popc(ebits), scan_scratch, tie_total);
+    uint32_t sbits = gbits;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      sel[j] = g[j];
-      if (e[j]) {
-        sel[j] = tie_rank < need_eq;
+    for (int j = 0; j < 16; ++j) {
+      if ((ebits >> j) & 1u) {
+        if (tie_rank < need_eq) sbits |= 1u << j;
         ++tie_rank;
       }
     }
-    const int ns = int(sel[0]) + int(sel[1]) + int(sel[2]) + int(sel[3]);
     int sel_total;
-    int pos = out_pos + block_exclusive_scan<kTopkWarps>(ns, scan_scratch, sel_total);
+    int pos = out_pos + block_exclusive_scan<kTopkWarps>(__popc(sbits), scan_scratch, sel_total);
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (sel[j]) out[pos++] = i0 + j;
+    for (int j = 0; j < 16; ++j)
+      if ((sbits >> j) & 1u) out[pos++] = i0 + j;
     eq_taken += tie_total;
     out_pos += sel_total;
   }
