@@ -301,8 +301,9 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, int64_t rows, const 
   if (scores == nullptr || row_len == nullptr || idx == nullptr || !aligned(scores, 16))
     return DSA_ERR_INVALID_ARGUMENT;
   if (rows > 0x7FFFFFFFLL || ld_scores > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
-  topk_rows_kernel<<<static_cast<unsigned>(rows), kTopkThreads, 0, as_stream(stream)>>>(scores, ld_scores, row_len,
-                                                                                       k, idx);
+  if (rows * kTopkCluster > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+  topk_rows_cluster_kernel<<<static_cast<unsigned>(rows * kTopkCluster), kTopkThreads, 0, as_stream(stream)>>>(
+      scores, ld_scores, row_len, k, idx);
   return launch_status();
 }
 
