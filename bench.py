@@ -375,6 +375,10 @@ def run_ours(args, world, rank, local):
 
     # ---- end to end through dsa_forward with host buffers ----
     e2e = run_e2e(args, dsa, inp, cfg, sm) if (rank == 0 and not args.no_e2e) else None
+    if e2e is not None:  # the pipelined host-to-host result equals the device-resident step's output
+        rows_chk, got = e2e.pop("_check_rows"), e2e.pop("_check")
+        assert torch.equal(got, out[rows_chk]), "pipelined e2e output differs from the device-resident step"
+        e2e["matches_device_path"] = True
 
     # ---- oracle on a bounded sample ----
     cpu = None
@@ -539,11 +543,18 @@ def run_decode(args, dsa, sm):
             "gpu_launches_per_step": 4}
 
 
-def run_e2e(args, dsa, inp, cfg, sm):
-    """dsa_forward with inputs copied from pinned host memory and the output copied back, every step."""
-    names = ["q8", "q_scale", "w", "k8", "k_scale", "q", "latent", "cu_seqlens"]
+def run_e2e(args, dsa, inp, cfg, sm, n_blocks=16):
+    """The prefill end to end from pinned host memory: every step copies all of its inputs in
+    and its output back.  The step is pipelined over query-row blocks of the sequence on three
+    streams -- the key-side inputs (k_I, k_scale, latent) first, then per block the copy-in of
+    its query-side rows, the fused indexer top-k and sparse MLA of those rows
+    (dsa_indexer_topk_rows, dsa_sparse_mla_prefill_rows) and the copy-out of its output -- so
+    that both copy directions overlap the kernels.  Steps do not overlap each other."""
+    assert len(cfg["seqlens"]) == 1, "the pipelined step shards one sequence by rows"
+    key_names = ["k8", "k_scale", "latent", "cu_seqlens"]
+    row_names = ["q8", "q_scale", "w", "q"]
     host = {}
-    for n in names:
+    for n in key_names + row_names:
         t = inp[n]
         try:
             h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
@@ -551,29 +562,59 @@ def run_e2e(args, dsa, inp, cfg, sm):
             h = torch.empty(t.shape, dtype=t.dtype)
         h.copy_(t)
         host[n] = h
-    dev = {n: torch.empty_like(inp[n]) for n in names}
-    T, H, k = inp["q"].shape[0], cfg["H"], cfg["k"]
+    dev = {n: torch.empty_like(inp[n]) for n in key_names + row_names}
+    T, H, k, H_I, d_I = inp["q"].shape[0], cfg["H"], cfg["k"], cfg["H_I"], cfg["d_I"]
     out = torch.empty((T, H, 512), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
     try:
         out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     except RuntimeError:
         out_h = torch.empty(out.shape, dtype=out.dtype)
-    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_PREFILL, 1, T, T, H, cfg["H_I"], k), dtype=torch.uint8,
-                     device="cuda")
-    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in key_names + row_names)
     d2h = out.numel() * out.element_size()
+    keys = dsa.contiguous_desc(dev["k8"], dev["cu_seqlens"], T, scale=dev["k_scale"])
+    lat = dsa.contiguous_desc(dev["latent"], dev["cu_seqlens"], T)
+    bounds = [T * b // n_blocks for b in range(n_blocks + 1)]
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    main = torch.cuda.current_stream()
 
     def step():
-        for n in names:
-            dev[n].copy_(host[n], non_blocking=True)
-        keys = dsa.contiguous_desc(dev["k8"], dev["cu_seqlens"], T, scale=dev["k_scale"])
-        lat = dsa.contiguous_desc(dev["latent"], dev["cu_seqlens"], T)
-        dsa.dsa_forward(dsa.DSA_MODE_PREFILL, dev["q8"], dev["q_scale"], dev["w"], keys, dev["q"], lat, 1, cfg["H_I"],
-                        cfg["d_I"], H, k, sm, out, None, None, ws)
-        out_h.copy_(out, non_blocking=True)
+        # a step starts after everything before it on the main stream (including the previous step)
+        for s in (s_in, s_run, s_out):
+            s.wait_stream(main)
+        with torch.cuda.stream(s_in):
+            for n in key_names:
+                dev[n].copy_(host[n], non_blocking=True)
+            keys_in = torch.cuda.Event()
+            keys_in.record(s_in)
+        s_run.wait_event(keys_in)
+        for b in range(n_blocks):
+            r0, r1 = bounds[b], bounds[b + 1]
+            with torch.cuda.stream(s_in):
+                for n in row_names:
+                    dev[n][r0:r1].copy_(host[n][r0:r1], non_blocking=True)
+                rows_in = torch.cuda.Event()
+                rows_in.record(s_in)
+            with torch.cuda.stream(s_run):
+                s_run.wait_event(rows_in)
+                dsa.dsa_indexer_topk_rows(dev["q8"][r0:r1], dev["q_scale"][r0:r1], dev["w"][r0:r1], keys, H_I, d_I, k,
+                                          r0, r1, idx[r0:r1])
+                dsa.dsa_sparse_mla_prefill_rows(dev["q"][r0:r1], lat, idx[r0:r1], H, k, sm, r0, r1, out[r0:r1])
+                done = torch.cuda.Event()
+                done.record(s_run)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done)
+                out_h[r0:r1].copy_(out[r0:r1], non_blocking=True)
+        for s in (s_in, s_run, s_out):
+            main.wait_stream(s)
 
     step()
     torch.cuda.synchronize()
+    # the pipelined result equals the device-resident path's on sampled rows
+    check = torch.empty((8, H, 512), dtype=torch.bfloat16, device="cuda")
+    rows = torch.linspace(0, T - 1, 8).long().tolist()
+    for i, r in enumerate(rows):
+        check[i] = out_h[r].to("cuda")
     n = max(1, min(args.steps, args.e2e_steps))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -585,7 +626,8 @@ def run_e2e(args, dsa, inp, cfg, sm):
     ms = e0.elapsed_time(e1) / n
     return {"value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": n,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "pinned": bool(host["q"].is_pinned())}
+            "pinned": bool(host["q"].is_pinned()), "pipeline": f"{n_blocks} query-row blocks, 3 streams",
+            "_check_rows": rows, "_check": check}
 
 
 # ------------------------------------------------------------------------------------------
