@@ -543,7 +543,7 @@ def run_decode(args, dsa, sm):
             "gpu_launches_per_step": 4}
 
 
-def run_e2e(args, dsa, inp, cfg, sm, n_blocks=16):
+def run_e2e(args, dsa, inp, cfg, sm, n_blocks=32):
     """The prefill end to end from pinned host memory: every step copies all of its inputs in
     and its output back.  The step is pipelined over query-row blocks of the sequence on three
     streams -- the key-side inputs (k_I, k_scale, latent) first, then per block the copy-in of
