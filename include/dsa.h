@@ -240,6 +240,15 @@ dsa_status dsa_indexer_kl(const float* p, const float* scores, const int32_t* id
                           float* loss, float* grad, void* stream);
 
 /*
+ * Self-test of failure detection (no counterpart on the pages): launches a kernel that waits on
+ * a barrier nothing completes, with the same bounded-wait scheme as every pipeline wait of this
+ * library but a limit of limit_us microseconds (1 .. 2000000); the kernel then records
+ * DSA_ERR_TIMEOUT in the device error word and returns normally, so a following
+ * dsa_device_error reports 5 and the context stays usable.  Asynchronous on `stream`.
+ */
+dsa_status dsa_selftest_wait_timeout(int32_t limit_us, void* stream);
+
+/*
  * Per-token FP8 quantiser for the indexer operands (the step that produces a2's input
  * contract; "DeepSeek-V3.2 论文解读", section 二, subsection "工作原理": the indexer runs in FP8).  For each row r
  * of x [rows, cols] bf16 (row-major, contiguous; one token: all of its indexer heads for

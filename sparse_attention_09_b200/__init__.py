@@ -34,7 +34,8 @@ DSA_MODE_DECODE = 1
 EXPORTED = ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_mla_prefill", "dsa_sparse_mla_decode",
             "dsa_forward", "dsa_workspace_size", "dsa_status_string", "dsa_device_error",
             "dsa_sparse_mla_decode_noalloc", "dsa_quantize_fp8", "dsa_masked_mla_prefill",
-            "dsa_indexer_topk_rows", "dsa_sparse_mla_prefill_rows", "dsa_attn_distribution", "dsa_indexer_kl")
+            "dsa_indexer_topk_rows", "dsa_sparse_mla_prefill_rows", "dsa_attn_distribution", "dsa_indexer_kl",
+            "dsa_selftest_wait_timeout")
 
 
 class KVDesc(ctypes.Structure):
@@ -83,6 +84,8 @@ _lib.dsa_attn_distribution.argtypes = [_P, _DESC, _P, _P, _I32, _I32, _I32, _F32
 _lib.dsa_attn_distribution.restype = _I32
 _lib.dsa_indexer_kl.argtypes = [_P, _P, _P, _I64, _I32, _P, _P, _P]
 _lib.dsa_indexer_kl.restype = _I32
+_lib.dsa_selftest_wait_timeout.argtypes = [_I32, _P]
+_lib.dsa_selftest_wait_timeout.restype = _I32
 _lib.dsa_indexer_topk_rows.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I64, _I64, _P, _P]
 _lib.dsa_indexer_topk_rows.restype = _I32
 _lib.dsa_sparse_mla_prefill_rows.argtypes = [_P, _DESC, _P, _I32, _I32, _F32, _I64, _I64, _P, _P, _P]
@@ -188,6 +191,11 @@ def dsa_indexer_kl(p, scores, idx, loss, grad, stream=None):
     _check(_lib.dsa_indexer_kl(_ptr(p), _ptr(scores), _ptr(idx), int(rows), int(k), _ptr(loss), _ptr(grad),
                                _stream(stream)), "dsa_indexer_kl")
     return loss, grad
+
+
+def dsa_selftest_wait_timeout(limit_us, stream=None):
+    """Runs the bounded-wait self-test kernel (it records DSA_ERR_TIMEOUT and returns)."""
+    _check(_lib.dsa_selftest_wait_timeout(int(limit_us), _stream(stream)), "dsa_selftest_wait_timeout")
 
 
 def dsa_indexer_topk_rows(q_fp8, q_scale, w, keys: Desc, H_I, d_I, k, row_begin, row_end, idx, stream=None):

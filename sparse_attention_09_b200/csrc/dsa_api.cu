@@ -15,6 +15,7 @@
 #include "quantize.cuh"
 #include "attn_probs.cuh"
 #include "indexer_kl.cuh"
+#include "selftest.cuh"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
 
@@ -271,6 +272,12 @@ dsa_status dsa_indexer_kl(const float* p, const float* scores, const int32_t* id
     return DSA_ERR_INVALID_ARGUMENT;
   if (rows > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
   indexer_kl_kernel<<<static_cast<unsigned>(rows), kl::kThreads, 0, as_stream(stream)>>>(p, scores, idx, k, loss, grad);
+  return launch_status();
+}
+
+dsa_status dsa_selftest_wait_timeout(int32_t limit_us, void* stream) {
+  if (limit_us <= 0 || limit_us > 2000000) return DSA_ERR_INVALID_ARGUMENT;
+  wait_timeout_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(static_cast<uint64_t>(limit_us) * 1000u);
   return launch_status();
 }
 
