@@ -545,11 +545,13 @@ def run_decode(args, dsa, sm):
 
 def run_e2e(args, dsa, inp, cfg, sm, n_blocks=32):
     """The prefill end to end from pinned host memory: every step copies all of its inputs in
-    and its output back.  The step is pipelined over query-row blocks of the sequence on three
+    and its output back.  A step is pipelined over query-row blocks of the sequence on three
     streams -- the key-side inputs (k_I, k_scale, latent) first, then per block the copy-in of
     its query-side rows, the fused indexer top-k and sparse MLA of those rows
     (dsa_indexer_topk_rows, dsa_sparse_mla_prefill_rows) and the copy-out of its output -- so
-    that both copy directions overlap the kernels.  Steps do not overlap each other."""
+    that both copy directions overlap the kernels.  The device-side inputs and outputs are
+    double-buffered, so step i+1 starts copying in while step i still computes and copies out;
+    events keep each buffer's reuse behind the step that used it two steps before."""
     assert len(cfg["seqlens"]) == 1, "the pipelined step shards one sequence by rows"
     key_names = ["k8", "k_scale", "latent", "cu_seqlens"]
     row_names = ["q8", "q_scale", "w", "q"]
@@ -562,32 +564,41 @@ def run_e2e(args, dsa, inp, cfg, sm, n_blocks=32):
             h = torch.empty(t.shape, dtype=t.dtype)
         h.copy_(t)
         host[n] = h
-    dev = {n: torch.empty_like(inp[n]) for n in key_names + row_names}
     T, H, k, H_I, d_I = inp["q"].shape[0], cfg["H"], cfg["k"], cfg["H_I"], cfg["d_I"]
-    out = torch.empty((T, H, 512), dtype=torch.bfloat16, device="cuda")
-    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    bufs = []
+    for _ in range(2):
+        dev = {n: torch.empty_like(inp[n]) for n in key_names + row_names}
+        bufs.append({"dev": dev,
+                     "out": torch.empty((T, H, 512), dtype=torch.bfloat16, device="cuda"),
+                     "idx": torch.empty((T, k), dtype=torch.int32, device="cuda"),
+                     "keys": dsa.contiguous_desc(dev["k8"], dev["cu_seqlens"], T, scale=dev["k_scale"]),
+                     "lat": dsa.contiguous_desc(dev["latent"], dev["cu_seqlens"], T),
+                     "inputs_free": None, "out_free": None})
     try:
-        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        out_h = torch.empty((T, H, 512), dtype=torch.bfloat16, pin_memory=True)
     except RuntimeError:
-        out_h = torch.empty(out.shape, dtype=out.dtype)
+        out_h = torch.empty((T, H, 512), dtype=torch.bfloat16)
     h2d = sum(host[n].numel() * host[n].element_size() for n in key_names + row_names)
-    d2h = out.numel() * out.element_size()
-    keys = dsa.contiguous_desc(dev["k8"], dev["cu_seqlens"], T, scale=dev["k_scale"])
-    lat = dsa.contiguous_desc(dev["latent"], dev["cu_seqlens"], T)
+    d2h = out_h.numel() * out_h.element_size()
     bounds = [T * b // n_blocks for b in range(n_blocks + 1)]
     s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     main = torch.cuda.current_stream()
+    for s in (s_in, s_run, s_out):
+        s.wait_stream(main)
 
-    def step():
-        # a step starts after everything before it on the main stream (including the previous step)
-        for s in (s_in, s_run, s_out):
-            s.wait_stream(main)
+    def step(i):
+        B = bufs[i & 1]
+        dev, out, idx = B["dev"], B["out"], B["idx"]
         with torch.cuda.stream(s_in):
+            if B["inputs_free"] is not None:
+                s_in.wait_event(B["inputs_free"])      # the step two back has finished reading them
             for n in key_names:
                 dev[n].copy_(host[n], non_blocking=True)
             keys_in = torch.cuda.Event()
             keys_in.record(s_in)
         s_run.wait_event(keys_in)
+        if B["out_free"] is not None:
+            s_run.wait_event(B["out_free"])            # the step two back has copied its output out
         for b in range(n_blocks):
             r0, r1 = bounds[b], bounds[b + 1]
             with torch.cuda.stream(s_in):
@@ -597,36 +608,45 @@ def run_e2e(args, dsa, inp, cfg, sm, n_blocks=32):
                 rows_in.record(s_in)
             with torch.cuda.stream(s_run):
                 s_run.wait_event(rows_in)
-                dsa.dsa_indexer_topk_rows(dev["q8"][r0:r1], dev["q_scale"][r0:r1], dev["w"][r0:r1], keys, H_I, d_I, k,
-                                          r0, r1, idx[r0:r1])
-                dsa.dsa_sparse_mla_prefill_rows(dev["q"][r0:r1], lat, idx[r0:r1], H, k, sm, r0, r1, out[r0:r1])
+                dsa.dsa_indexer_topk_rows(dev["q8"][r0:r1], dev["q_scale"][r0:r1], dev["w"][r0:r1], B["keys"], H_I,
+                                          d_I, k, r0, r1, idx[r0:r1])
+                dsa.dsa_sparse_mla_prefill_rows(dev["q"][r0:r1], B["lat"], idx[r0:r1], H, k, sm, r0, r1, out[r0:r1])
                 done = torch.cuda.Event()
                 done.record(s_run)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(done)
                 out_h[r0:r1].copy_(out[r0:r1], non_blocking=True)
+        B["inputs_free"] = torch.cuda.Event()
+        B["inputs_free"].record(s_run)
+        B["out_free"] = torch.cuda.Event()
+        B["out_free"].record(s_out)
+
+    def drain():
         for s in (s_in, s_run, s_out):
             main.wait_stream(s)
 
-    step()
+    step(0)
+    drain()
     torch.cuda.synchronize()
     # the pipelined result equals the device-resident path's on sampled rows
-    check = torch.empty((8, H, 512), dtype=torch.bfloat16, device="cuda")
     rows = torch.linspace(0, T - 1, 8).long().tolist()
-    for i, r in enumerate(rows):
-        check[i] = out_h[r].to("cuda")
-    n = max(1, min(args.steps, args.e2e_steps))
+    check = torch.stack([out_h[r] for r in rows]).to("cuda")
+    n = max(2, min(max(args.steps, 4), args.e2e_steps))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(n):
-        step()
+    for s in (s_in, s_run, s_out):
+        s.wait_stream(main)
+    for i in range(1, n + 1):
+        step(i)
+    drain()
     e1.record()
     torch.cuda.synchronize()
     assert dsa.dsa_device_error() == 0
     ms = e0.elapsed_time(e1) / n
     return {"value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": n,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "pinned": bool(host["q"].is_pinned()), "pipeline": f"{n_blocks} query-row blocks, 3 streams",
+            "pinned": bool(host["q"].is_pinned()),
+            "pipeline": f"{n_blocks} query-row blocks, 3 streams, double-buffered across steps",
             "_check_rows": rows, "_check": check}
 
 
@@ -671,7 +691,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-rows", type=int, default=256)
     ap.add_argument("--ref-rows", type=int, default=2)
     ap.add_argument("--workload", default=PREFILL, choices=[w for w, c in synth.WORKLOADS.items() if c["kind"] == "prefill"],
