@@ -83,16 +83,25 @@ typedef struct {
 } dsa_kv_desc;
 
 /*
+ * Query scale granularity (q_scale_heads), shared by every call that runs the indexer (the
+ * indexer runs in FP8: "DeepSeek-V3.2 论文解读", section 二, subsection "工作原理"):
+ *   1    q_scale holds one fp32 scale per query row, shared by its H_I heads ([rows]);
+ *   H_I  q_scale holds one scale per (query row, indexer head) ([rows, H_I], row-major),
+ *        as a per-(token, head) FP8 quantisation of q_I produces (dsa_quantize_fp8 over
+ *        rows * H_I rows of d_I columns).
+ * The dequantised query of head j is e4m3(q_fp8[r, j, :]) * q_scale[r] (resp. q_scale[r, j]).
+ * Scales must be finite and positive; any other q_scale_heads -> DSA_ERR_INVALID_ARGUMENT.
+ *
  * Lightning indexer scores (method step 1), written to HBM for a range of query rows.
  *   prefill (keys contiguous): rows are packed query tokens [row_begin, row_end) of
- *     q_fp8 [T, H_I, d_I], q_scale [T], w [T, H_I]; row r (local position t in a sequence
+ *     q_fp8 [T, H_I, d_I], q_scale [T] or [T, H_I], w [T, H_I]; row r (local position t in a sequence
  *     of length n) gets scores[(r-row_begin)*ld_scores + s] = I[t,s] for s <= t and -INFINITY
  *     for t < s < n.  ld_scores >= keys->max_seqlen and a multiple of 4.
  *   decode (keys paged): rows are sequences b in [row_begin, row_end) with q_fp8 [B, H_I, d_I],
- *     q_scale [B], w [B, H_I]; scores[(b-row_begin)*ld_scores + s] = I for s < ctx[b].
+ *     q_scale [B] or [B, H_I], w [B, H_I]; scores[(b-row_begin)*ld_scores + s] = I for s < ctx[b].
  * Scores are fp32, accumulated in fp32 on the tensor cores (e4m3 x e4m3).
  */
-dsa_status dsa_indexer_scores(const uint8_t* q_fp8, const float* q_scale, const float* w,
+dsa_status dsa_indexer_scores(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
                               const dsa_kv_desc* keys, int32_t B, int32_t H_I, int32_t d_I,
                               int64_t row_begin, int64_t row_end, float* scores, int64_t ld_scores,
                               void* stream);
@@ -105,8 +114,9 @@ dsa_status dsa_indexer_scores(const uint8_t* q_fp8, const float* q_scale, const 
  * shared memory with a rising threshold.  The selection equals dsa_topk applied to the
  * scores dsa_indexer_scores writes (same fp32 arithmetic).  keys->max_seqlen <= 196608 (d_I = 128) or 98304 (d_I = 64).
  */
-dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, const float* w, const dsa_kv_desc* keys,
-                            int32_t B, int32_t H_I, int32_t d_I, int32_t k, int32_t* idx_out, void* stream);
+dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
+                            const dsa_kv_desc* keys, int32_t B, int32_t H_I, int32_t d_I, int32_t k, int32_t* idx_out,
+                            void* stream);
 
 /*
  * Top-k selection (method step 2) over score rows: for row r the first row_len[r] entries
@@ -130,14 +140,14 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, int64_t rows, const 
  * holds every key and latent row -- gathered from the others -- and its own block of query
  * rows).  keys / latent describe ONE contiguous sequence (cu_seqlens = {0, L}).
  *   dsa_indexer_topk_rows: like dsa_indexer_topk for query rows [row_begin, row_end) only;
- *     q_fp8 [R, H_I, d_I], q_scale [R], w [R, H_I] and idx_out [R, k] hold just those
+ *     q_fp8 [R, H_I, d_I], q_scale [R] or [R, H_I], w [R, H_I] and idx_out [R, k] hold just those
  *     R = row_end - row_begin rows (row 0 = query row_begin).
  *   dsa_sparse_mla_prefill_rows: like dsa_sparse_mla_prefill for rows [row_begin, row_end);
  *     q [R, H, 576], idx [R, k], out [R, H, 512], lse [R, H] hold just those rows.
  * Each block's results equal the corresponding rows of the whole-sequence call.  row_begin ==
  * row_end is a no-op; 0 <= row_begin <= row_end <= L, else DSA_ERR_INVALID_ARGUMENT.
  */
-dsa_status dsa_indexer_topk_rows(const uint8_t* q_fp8, const float* q_scale, const float* w,
+dsa_status dsa_indexer_topk_rows(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
                                  const dsa_kv_desc* keys, int32_t H_I, int32_t d_I, int32_t k,
                                  int64_t row_begin, int64_t row_end, int32_t* idx_out, void* stream);
 dsa_status dsa_sparse_mla_prefill_rows(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t H,
@@ -200,8 +210,8 @@ dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const dsa_kv_desc* laten
  *     sparse MLA with a log-sum-exp merge.
  * idx_out [rows, k] receives the selection when not NULL (otherwise it lives in workspace).
  */
-dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale, const float* w,
-                       const dsa_kv_desc* keys, const void* q, const dsa_kv_desc* latent, int32_t B,
+dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads,
+                       const float* w, const dsa_kv_desc* keys, const void* q, const dsa_kv_desc* latent, int32_t B,
                        int32_t H_I, int32_t d_I, int32_t H, int32_t k, float sm_scale, void* out,
                        float* lse, int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream);
 

@@ -8,7 +8,8 @@ is the only library primitive used as a step.  Readings taken where the pages ar
 
 * FP8 means OCP E4M3FN (bias 7, subnormals, max 448, S.1111.111 = NaN, no infinities).
 * Dequantisation is per token: q_I[t,j,:] = e4m3(q8[t,j,:]) * q_scale[t],
-  k_I[s,:] = e4m3(k8[s,:]) * k_scale[s].
+  k_I[s,:] = e4m3(k8[s,:]) * k_scale[s]; or, for queries quantised per (token, head),
+  q_I[t,j,:] = e4m3(q8[t,j,:]) * q_scale[t,j].
 * "All preceding tokens" is the causal prefix s <= t (the query's own key included), so a
   prefill row keeps min(k, t+1) entries; a decode query sits at position ctx-1 and sees all
   ctx cached keys.
@@ -105,11 +106,13 @@ def indexer_scores_query(q8: np.ndarray, q_scale: float, w: np.ndarray, k8: np.n
                          k_scale: np.ndarray) -> np.ndarray:
     """Index scores of one query token against a set of keys.
 
-    I[s] = sum_j w[j] * ReLU(q_I[j] . k_I[s]) with q_I = e4m3(q8) * q_scale and
-    k_I = e4m3(k8) * k_scale (per-token scales).  q8: [H_I, d_I] bytes, w: [H_I],
-    k8: [n, d_I] bytes, k_scale: [n].  Returns float64 [n].
+    I[s] = sum_j w[j] * ReLU(q_I[j] . k_I[s]) with q_I[j] = e4m3(q8[j]) * q_scale (one scale
+    for the token, or q_scale[j] when given one per head) and k_I = e4m3(k8) * k_scale.
+    q8: [H_I, d_I] bytes, q_scale: scalar or [H_I], w: [H_I], k8: [n, d_I] bytes,
+    k_scale: [n].  Returns float64 [n].
     """
-    q = decode_e4m3(q8) * float(q_scale)                       # [H_I, d_I]
+    qs = np.asarray(q_scale, np.float64)
+    q = decode_e4m3(q8) * (qs[:, None] if qs.ndim == 1 else qs)   # [H_I, d_I], dequantised
     k = decode_e4m3(k8) * np.asarray(k_scale, np.float64)[:, None]  # [n, d_I]
     dots = q @ k.T                                              # [H_I, n]
     return np.asarray(w, np.float64) @ np.maximum(dots, 0.0)    # sum over indexer heads j
@@ -128,7 +131,7 @@ def indexer_scores(q8: np.ndarray, q_scale: np.ndarray, w: np.ndarray, k8: np.nd
                    k_scale: np.ndarray, rows=None) -> np.ndarray:
     """Prefill index scores of one sequence, for the causal prefix of each query row.
 
-    q8: [L, H_I, d_I], q_scale: [L], w: [L, H_I], k8: [L, d_I], k_scale: [L].
+    q8: [L, H_I, d_I], q_scale: [L] or [L, H_I], w: [L, H_I], k8: [L, d_I], k_scale: [L].
     Returns float64 [len(rows), L]: I[t, s] for s <= t and -inf for s > t.
     """
     L = k8.shape[0]
@@ -271,7 +274,7 @@ def decode_indexer_scores(q8, q_scale, w, kcache8, kscale_cache, block_table_row
 def dsa_prefill_rows(seq: dict, k: int, sm_scale: float, rows, dv: int = 512):
     """DSA prefill of one sequence for the given query rows.
 
-    seq holds numpy arrays: q8 [L,H_I,d_I], q_scale [L], w [L,H_I], k8 [L,d_I], k_scale [L],
+    seq holds numpy arrays: q8 [L,H_I,d_I], q_scale [L] or [L,H_I], w [L,H_I], k8 [L,d_I], k_scale [L],
     q [L,H,D], latent [L,D].  Returns dict(scores32 per row, idx [rows,k], out, lse).
     """
     rows = list(rows)
@@ -291,7 +294,7 @@ def dsa_decode(seq: dict, k: int, sm_scale: float, dv: int = 512):
     """DSA decode step of one sequence: indexer over the paged FP8 keys, top-k, sparse MLA over
     the paged latent cache.
 
-    seq holds numpy arrays: q8 [H_I,d_I], q_scale (scalar), w [H_I], kcache8 [nb,bs,d_I],
+    seq holds numpy arrays: q8 [H_I,d_I], q_scale (scalar, or [H_I] per head), w [H_I], kcache8 [nb,bs,d_I],
     kscale_cache [nb,bs], latent_cache [nb,bs,D], block_table [max_blocks], ctx, q [H,D].
     """
     ctx = int(seq["ctx"])

@@ -67,16 +67,16 @@ _lib.dsa_device_error.argtypes = [ctypes.POINTER(_I32), _P]
 _lib.dsa_device_error.restype = _I32
 _lib.dsa_topk.argtypes = [_P, _I64, _I64, _P, _I32, _P, _P]
 _lib.dsa_topk.restype = _I32
-_lib.dsa_indexer_scores.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I64, _I64, _P, _I64, _P]
+_lib.dsa_indexer_scores.argtypes = [_P, _P, _I32, _P, _DESC, _I32, _I32, _I32, _I64, _I64, _P, _I64, _P]
 _lib.dsa_indexer_scores.restype = _I32
 _lib.dsa_sparse_mla_prefill.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P]
 _lib.dsa_sparse_mla_prefill.restype = _I32
 _lib.dsa_sparse_mla_decode.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P, _SZ, _P]
 _lib.dsa_sparse_mla_decode.restype = _I32
-_lib.dsa_forward.argtypes = [_I32, _P, _P, _P, _DESC, _P, _DESC, _I32, _I32, _I32, _I32, _I32, _F32, _P, _P, _P,
+_lib.dsa_forward.argtypes = [_I32, _P, _P, _I32, _P, _DESC, _P, _DESC, _I32, _I32, _I32, _I32, _I32, _F32, _P, _P, _P,
                              _P, _SZ, _P]
 _lib.dsa_forward.restype = _I32
-_lib.dsa_indexer_topk.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I32, _P, _P]
+_lib.dsa_indexer_topk.argtypes = [_P, _P, _I32, _P, _DESC, _I32, _I32, _I32, _I32, _P, _P]
 _lib.dsa_indexer_topk.restype = _I32
 _lib.dsa_sparse_mla_decode_noalloc.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P]
 _lib.dsa_sparse_mla_decode_noalloc.restype = _I32
@@ -86,7 +86,7 @@ _lib.dsa_indexer_kl.argtypes = [_P, _P, _P, _I64, _I32, _P, _P, _P]
 _lib.dsa_indexer_kl.restype = _I32
 _lib.dsa_selftest_wait_timeout.argtypes = [_I32, _P]
 _lib.dsa_selftest_wait_timeout.restype = _I32
-_lib.dsa_indexer_topk_rows.argtypes = [_P, _P, _P, _DESC, _I32, _I32, _I32, _I64, _I64, _P, _P]
+_lib.dsa_indexer_topk_rows.argtypes = [_P, _P, _I32, _P, _DESC, _I32, _I32, _I32, _I64, _I64, _P, _P]
 _lib.dsa_indexer_topk_rows.restype = _I32
 _lib.dsa_sparse_mla_prefill_rows.argtypes = [_P, _DESC, _P, _I32, _I32, _F32, _I64, _I64, _P, _P, _P]
 _lib.dsa_sparse_mla_prefill_rows.restype = _I32
@@ -171,9 +171,20 @@ def dsa_topk(scores, row_len, k, idx, stream=None):
     return idx
 
 
+def _q_scale_heads(q_scale, H_I) -> int:
+    """The C ABI's q_scale_heads from the scale tensor's shape: [rows] -> 1 (one scale per
+    token), [rows, H_I] -> H_I (one per token and indexer head)."""
+    if q_scale is not None and q_scale.dim() == 2:
+        if q_scale.shape[1] != int(H_I):
+            raise ValueError(f"q_scale has {q_scale.shape[1]} columns, expected H_I = {H_I}")
+        return int(H_I)
+    return 1
+
+
 def dsa_indexer_scores(q_fp8, q_scale, w, keys: Desc, B, H_I, d_I, row_begin, row_end, scores, stream=None):
-    _check(_lib.dsa_indexer_scores(_ptr(q_fp8), _ptr(q_scale), _ptr(w), keys.ref(), int(B), int(H_I), int(d_I),
-                                   int(row_begin), int(row_end), _ptr(scores), scores.stride(0), _stream(stream)),
+    _check(_lib.dsa_indexer_scores(_ptr(q_fp8), _ptr(q_scale), _q_scale_heads(q_scale, H_I), _ptr(w), keys.ref(),
+                                   int(B), int(H_I), int(d_I), int(row_begin), int(row_end), _ptr(scores),
+                                   scores.stride(0), _stream(stream)),
            "dsa_indexer_scores")
     return scores
 
@@ -201,8 +212,9 @@ def dsa_selftest_wait_timeout(limit_us, stream=None):
 def dsa_indexer_topk_rows(q_fp8, q_scale, w, keys: Desc, H_I, d_I, k, row_begin, row_end, idx, stream=None):
     """Fused indexer + top-k for query rows [row_begin, row_end) of one sequence; the query
     arrays and idx hold just those rows."""
-    _check(_lib.dsa_indexer_topk_rows(_ptr(q_fp8), _ptr(q_scale), _ptr(w), keys.ref(), int(H_I), int(d_I), int(k),
-                                      int(row_begin), int(row_end), _ptr(idx), _stream(stream)), "dsa_indexer_topk_rows")
+    _check(_lib.dsa_indexer_topk_rows(_ptr(q_fp8), _ptr(q_scale), _q_scale_heads(q_scale, H_I), _ptr(w),
+                                      keys.ref(), int(H_I), int(d_I), int(k), int(row_begin), int(row_end),
+                                      _ptr(idx), _stream(stream)), "dsa_indexer_topk_rows")
     return idx
 
 
@@ -238,7 +250,8 @@ def dsa_sparse_mla_decode(q, latent: Desc, idx, B, H, k, sm_scale, out, lse=None
 def dsa_forward(mode, q_fp8, q_scale, w, keys: Desc, q, latent: Desc, B, H_I, d_I, H, k, sm_scale, out, lse=None,
                 idx_out=None, workspace=None, stream=None):
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(_lib.dsa_forward(int(mode), _ptr(q_fp8), _ptr(q_scale), _ptr(w), keys.ref(), _ptr(q), latent.ref(),
+    _check(_lib.dsa_forward(int(mode), _ptr(q_fp8), _ptr(q_scale), _q_scale_heads(q_scale, H_I), _ptr(w), keys.ref(),
+                            _ptr(q), latent.ref(),
                             int(B), int(H_I), int(d_I), int(H), int(k), float(sm_scale), _ptr(out), _ptr(lse),
                             _ptr(idx_out), _ptr(workspace), ws_bytes, _stream(stream)), "dsa_forward")
     return out
@@ -256,7 +269,8 @@ def dsa_device_error(stream=None) -> int:
 
 def dsa_indexer_topk(q_fp8, q_scale, w, keys: Desc, B, H_I, d_I, k, idx_out, stream=None):
     """Fused indexer + top-k for prefill: idx_out [T, k] (ascending, -1 padded)."""
-    _check(_lib.dsa_indexer_topk(_ptr(q_fp8), _ptr(q_scale), _ptr(w), keys.ref(), int(B), int(H_I), int(d_I), int(k),
+    _check(_lib.dsa_indexer_topk(_ptr(q_fp8), _ptr(q_scale), _q_scale_heads(q_scale, H_I), _ptr(w), keys.ref(),
+                                 int(B), int(H_I), int(d_I), int(k),
                                  _ptr(idx_out), _stream(stream)), "dsa_indexer_topk")
     return idx_out
 

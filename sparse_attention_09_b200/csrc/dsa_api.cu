@@ -98,12 +98,13 @@ bool indexer_shape_ok(int H_I, int d_I) { return (H_I == 4 || H_I == 64) && (d_I
 
 // Validates the common indexer arguments and builds the Q / K tensor maps.
 // q_rows: rows held by the query arrays (prefill: the packed tokens they cover; 0 = all of them)
-dsa_status indexer_common(const uint8_t* q_fp8, const float* q_scale, const float* w, const dsa_kv_desc* keys,
-                          int32_t B, int32_t H_I, int32_t d_I, CUtensorMap* qm, CUtensorMap* km,
-                          IndexerParams* p, int64_t q_rows = 0) {
+dsa_status indexer_common(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
+                          const dsa_kv_desc* keys, int32_t B, int32_t H_I, int32_t d_I, CUtensorMap* qm,
+                          CUtensorMap* km, IndexerParams* p, int64_t q_rows = 0) {
   if (q_fp8 == nullptr || q_scale == nullptr || w == nullptr || keys == nullptr || keys->data == nullptr ||
       keys->scale == nullptr || B <= 0)
     return DSA_ERR_INVALID_ARGUMENT;
+  if (q_scale_heads != 1 && q_scale_heads != H_I) return DSA_ERR_INVALID_ARGUMENT;
   if (!aligned(q_fp8, 16) || !aligned(keys->data, 16)) return DSA_ERR_INVALID_ARGUMENT;
   if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED;
   const CUtensorMapSwizzle sw = d_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -112,6 +113,7 @@ dsa_status indexer_common(const uint8_t* q_fp8, const float* q_scale, const floa
   p->tok_end = 0x7FFFFFFF;
   p->q_row0 = 0;
   p->q_scale = q_scale;
+  p->q_scale_heads = q_scale_heads;
   p->w = w;
   p->k_scale = keys->scale;
   if (keys->kind == DSA_KV_CONTIGUOUS) {
@@ -314,15 +316,15 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, int64_t rows, const 
   return launch_status();
 }
 
-dsa_status dsa_indexer_scores(const uint8_t* q_fp8, const float* q_scale, const float* w, const dsa_kv_desc* keys,
-                              int32_t B, int32_t H_I, int32_t d_I, int64_t row_begin, int64_t row_end,
-                              float* scores, int64_t ld_scores, void* stream) {
+dsa_status dsa_indexer_scores(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
+                              const dsa_kv_desc* keys, int32_t B, int32_t H_I, int32_t d_I, int64_t row_begin,
+                              int64_t row_end, float* scores, int64_t ld_scores, void* stream) {
   if (scores == nullptr || row_begin < 0 || row_end < row_begin) return DSA_ERR_INVALID_ARGUMENT;
   if (keys == nullptr) return DSA_ERR_INVALID_ARGUMENT;
   if (row_end == row_begin) return DSA_OK;
   CUtensorMap qm, km;
   IndexerParams p;
-  dsa_status st = indexer_common(q_fp8, q_scale, w, keys, B, H_I, d_I, &qm, &km, &p);
+  dsa_status st = indexer_common(q_fp8, q_scale, q_scale_heads, w, keys, B, H_I, d_I, &qm, &km, &p);
   if (st != DSA_OK) return st;
   if (ld_scores < keys->max_seqlen) return DSA_ERR_INVALID_ARGUMENT;
   p.scores = scores;
@@ -339,14 +341,15 @@ dsa_status dsa_indexer_scores(const uint8_t* q_fp8, const float* q_scale, const 
   return launch_indexer<kIdxScores, true>(d_I, H_I, qm, km, p, grid, as_stream(stream));
 }
 
-dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, const float* w, const dsa_kv_desc* keys,
-                            int32_t B, int32_t H_I, int32_t d_I, int32_t k, int32_t* idx_out, void* stream) {
+dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
+                            const dsa_kv_desc* keys, int32_t B, int32_t H_I, int32_t d_I, int32_t k, int32_t* idx_out,
+                            void* stream) {
   if (idx_out == nullptr || keys == nullptr || k <= 0) return DSA_ERR_INVALID_ARGUMENT;
   if (keys->kind != DSA_KV_CONTIGUOUS) return DSA_ERR_UNSUPPORTED;
   if (k > 2048) return DSA_ERR_UNSUPPORTED;
   CUtensorMap qm, km;
   IndexerParams p;
-  dsa_status st = indexer_common(q_fp8, q_scale, w, keys, B, H_I, d_I, &qm, &km, &p);
+  dsa_status st = indexer_common(q_fp8, q_scale, q_scale_heads, w, keys, B, H_I, d_I, &qm, &km, &p);
   if (st != DSA_OK) return st;
   // the final ascending emission uses a bitmap of the causal prefix inside the key ring
   const int64_t bitmap_bytes = (static_cast<int64_t>(keys->max_seqlen) + 31) / 32 * 4;
@@ -361,9 +364,9 @@ dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, const fl
   return launch_indexer<kIdxTopk, false>(d_I, H_I, qm, km, p, grid, as_stream(stream));
 }
 
-dsa_status dsa_indexer_topk_rows(const uint8_t* q_fp8, const float* q_scale, const float* w, const dsa_kv_desc* keys,
-                                 int32_t H_I, int32_t d_I, int32_t k, int64_t row_begin, int64_t row_end,
-                                 int32_t* idx_out, void* stream) {
+dsa_status dsa_indexer_topk_rows(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
+                                 const dsa_kv_desc* keys, int32_t H_I, int32_t d_I, int32_t k, int64_t row_begin,
+                                 int64_t row_end, int32_t* idx_out, void* stream) {
   if (keys == nullptr || k <= 0 || row_begin < 0 || row_end < row_begin) return DSA_ERR_INVALID_ARGUMENT;
   if (keys->kind != DSA_KV_CONTIGUOUS) return DSA_ERR_UNSUPPORTED;
   if (k > 2048) return DSA_ERR_UNSUPPORTED;
@@ -372,7 +375,8 @@ dsa_status dsa_indexer_topk_rows(const uint8_t* q_fp8, const float* q_scale, con
   if (idx_out == nullptr) return DSA_ERR_INVALID_ARGUMENT;
   CUtensorMap qm, km;
   IndexerParams p;
-  dsa_status st = indexer_common(q_fp8, q_scale, w, keys, 1, H_I, d_I, &qm, &km, &p, row_end - row_begin);
+  dsa_status st = indexer_common(q_fp8, q_scale, q_scale_heads, w, keys, 1, H_I, d_I, &qm, &km, &p,
+                                 row_end - row_begin);
   if (st != DSA_OK) return st;
   const int64_t bitmap_bytes = (static_cast<int64_t>(keys->max_seqlen) + 31) / 32 * 4;
   if (bitmap_bytes > static_cast<int64_t>(kIdxStagesTopk) * 128 * d_I / 2 || keys->max_seqlen > (1 << 24))
@@ -530,10 +534,10 @@ dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const dsa_kv_desc* laten
                                stream);
 }
 
-dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale, const float* w,
-                       const dsa_kv_desc* keys, const void* q, const dsa_kv_desc* latent, int32_t B, int32_t H_I,
-                       int32_t d_I, int32_t H, int32_t k, float sm_scale, void* out, float* lse, int32_t* idx_out,
-                       void* workspace, size_t ws_bytes, void* stream) {
+dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads,
+                       const float* w, const dsa_kv_desc* keys, const void* q, const dsa_kv_desc* latent, int32_t B,
+                       int32_t H_I, int32_t d_I, int32_t H, int32_t k, float sm_scale, void* out, float* lse,
+                       int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream) {
   if (keys == nullptr || latent == nullptr || B <= 0) return DSA_ERR_INVALID_ARGUMENT;
   if (!mla_shape_ok(H, k)) return DSA_ERR_UNSUPPORTED;
   const size_t need = dsa_workspace_size(mode, B, keys->total_tokens, keys->max_seqlen, H, H_I, k);
@@ -545,7 +549,7 @@ dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale,
       if (ws_bytes < need) return DSA_ERR_WORKSPACE_TOO_SMALL;
       idx = static_cast<int32_t*>(workspace);
     }
-    dsa_status st = dsa_indexer_topk(q_fp8, q_scale, w, keys, B, H_I, d_I, k, idx, stream);
+    dsa_status st = dsa_indexer_topk(q_fp8, q_scale, q_scale_heads, w, keys, B, H_I, d_I, k, idx, stream);
     if (st != DSA_OK) return st;
     return dsa_sparse_mla_prefill(q, latent, idx, B, H, k, sm_scale, out, lse, stream);
   }
@@ -562,7 +566,7 @@ dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale,
                      ? idx_out
                      : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + part +
                                                   align256(static_cast<size_t>(B) * ld * 4));
-  dsa_status st = dsa_indexer_scores(q_fp8, q_scale, w, keys, B, H_I, d_I, 0, B, scores, ld, stream);
+  dsa_status st = dsa_indexer_scores(q_fp8, q_scale, q_scale_heads, w, keys, B, H_I, d_I, 0, B, scores, ld, stream);
   if (st != DSA_OK) return st;
   st = dsa_topk(scores, ld, B, keys->context_lens, k, idx, stream);
   if (st != DSA_OK) return st;

@@ -1,6 +1,10 @@
 // Lightning indexer on the 5th-generation tensor cores, with the selection fused in.
 //
-// I[t,s] = k_scale[s] * sum_j (w[t,j] * q_scale[t]) * ReLU(sum_d q8[t,j,d] * k8[s,d])
+// I[t,s] = k_scale[s] * sum_j (w[t,j] * q_scale[t,j]) * ReLU(sum_d q8[t,j,d] * k8[s,d])
+//
+// with one query scale per token shared by its heads (q_scale[t,j] = q_scale[t]) or one per
+// (token, head).  Every scale is positive, so it commutes with the ReLU and folds into the
+// head weight once per CTA.
 //
 // The e4m3 x e4m3 products run as one tcgen05.mma (kind::f8f6f4, fp32 accumulate in TMEM)
 // per 32-deep K slice with
@@ -36,7 +40,7 @@ namespace dsa {
 enum { kIdxScores = 0, kIdxTopk = 1 };
 
 struct IndexerParams {
-  const float* q_scale;       // [rows]
+  const float* q_scale;       // [rows] (q_scale_heads == 1) or [rows, H_I] (q_scale_heads == H_I)
   const float* w;             // [rows, H_I]
   const float* k_scale;       // contiguous [T] | paged [num_blocks * 64]
   const int32_t* cu_seqlens;  // prefill [B+1]
@@ -52,6 +56,7 @@ struct IndexerParams {
   int64_t q_row0;             // prefill: packed row held by row 0 of q / q_scale / w / idx_out
   int32_t k;
   int32_t cap;                // candidate capacity per token (kIdxTopk)
+  int32_t q_scale_heads;      // 1: one query scale per token; H_I: one per (token, head)
 };
 
 namespace idx_detail {
@@ -179,7 +184,7 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
     float v = 0.f;
     if (tt < ntok) {
       const int64_t row = PAGED ? b : (p.cu_seqlens[b] + t0 + tt - p.q_row0);
-      v = p.w[row * H_I + j] * p.q_scale[row];
+      v = p.w[row * H_I + j] * p.q_scale[p.q_scale_heads == 1 ? row : row * H_I + j];
     }
     sWq[i] = v;
   }

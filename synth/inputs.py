@@ -74,19 +74,28 @@ def _normal_bf16(shape, std, g, device):
     return out
 
 
-def _indexer_operand(shape, std, as_bf16, g, device, planted=0.0, g_plant=None):
+def _indexer_operand(shape, std, as_bf16, g, device, planted=0.0, g_plant=None, per_head=False):
+    """e4m3 codes and fp32 scales of a seeded normal operand [T, ...]: one scale per token, or
+    with per_head (shape [T, H_I, d_I]) one per (token, head), head j drawn 2^-(j mod 8) times
+    smaller so that the heads' scales differ."""
     T = shape[0]
     codes = torch.empty(shape, dtype=torch.uint8, device=device)
-    scales = torch.empty((T,), dtype=torch.float32, device=device)
+    scales = torch.empty((T, shape[1]) if per_head else (T,), dtype=torch.float32, device=device)
     for t0 in range(0, T, _CHUNK):
         t1 = min(T, t0 + _CHUNK)
         x = torch.randn((t1 - t0,) + tuple(shape[1:]), generator=g, device=device) * std
+        if per_head:
+            x *= (2.0 ** -(torch.arange(shape[1], device=device) % 8)).reshape(1, -1, 1)
         if as_bf16:
             x = x.to(torch.bfloat16).float()
         if planted > 0:
             hot = torch.rand((t1 - t0,), generator=g_plant, device=device) < planted
             x[hot] *= 4.0
-        c, s = quantize_e4m3_per_token(x)
+        if per_head:
+            c, s = quantize_e4m3_per_token(x.reshape(-1, shape[2]))
+            c, s = c.reshape(x.shape), s.reshape(t1 - t0, shape[1])
+        else:
+            c, s = quantize_e4m3_per_token(x)
         codes[t0:t1] = c
         scales[t0:t1] = s
     return codes, scales
@@ -101,17 +110,18 @@ def _weights(shape, dist, g, device):
 
 
 def prefill_inputs(seqlens, H_I, d_I, H, *, seed, device, w_dist="normal8", idx_std=1.0,
-                   idx_bf16=False, planted=0.0, **_):
+                   idx_bf16=False, planted=0.0, q_scale_per_head=False, **_):
     """Packed prefill inputs for sequences of the given lengths (queries == keys per sequence).
 
-    Returns a dict of device tensors: cu_seqlens [B+1] i32, q8 [T,H_I,d_I] u8, q_scale [T],
-    w [T,H_I], k8 [T,d_I] u8, k_scale [T], q [T,H,576] bf16, latent [T,576] bf16, plus the
-    host-side ``seqlens`` list.
+    Returns a dict of device tensors: cu_seqlens [B+1] i32, q8 [T,H_I,d_I] u8, q_scale [T]
+    (or [T,H_I] with q_scale_per_head), w [T,H_I], k8 [T,d_I] u8, k_scale [T], q [T,H,576]
+    bf16, latent [T,576] bf16, plus the host-side ``seqlens`` list.
     """
     seqlens = [int(x) for x in seqlens]
     T = sum(seqlens)
     cu = torch.tensor(np.concatenate([[0], np.cumsum(seqlens)]), dtype=torch.int32, device=device)
-    q8, q_scale = _indexer_operand((T, H_I, d_I), idx_std, idx_bf16, _gen(device, seed, 1), device)
+    q8, q_scale = _indexer_operand((T, H_I, d_I), idx_std, idx_bf16, _gen(device, seed, 1), device,
+                                   per_head=q_scale_per_head)
     k8, k_scale = _indexer_operand((T, d_I), idx_std, idx_bf16, _gen(device, seed, 2), device,
                                    planted=planted, g_plant=_gen(device, seed, 7))
     w = _weights((T, H_I), w_dist, _gen(device, seed, 3), device)
@@ -122,14 +132,15 @@ def prefill_inputs(seqlens, H_I, d_I, H, *, seed, device, w_dist="normal8", idx_
 
 
 def decode_inputs(B, ctx_lo, ctx_hi, H_I, d_I, H, *, seed, device, block_size=64, w_dist="normal8",
-                  idx_std=1.0, ctx=None, spare_blocks=3, **_):
+                  idx_std=1.0, ctx=None, spare_blocks=3, q_scale_per_head=False, **_):
     """Paged decode inputs: one query per sequence over a cache of ctx[b] tokens.
 
     Blocks of ``block_size`` tokens are taken from a pool in the order of a seeded
     permutation, so a sequence's blocks are scattered.  Returns device tensors ctx [B] i32,
     block_table [B,max_blocks] i32 (unused entries -1), kcache8 [nb,bs,d_I] u8,
-    kscale_cache [nb,bs] f32, latent_cache [nb,bs,576] bf16, q8 [B,H_I,d_I], q_scale [B],
-    w [B,H_I], q [B,H,576], plus host copies ``ctx_host`` and ``max_ctx``.
+    kscale_cache [nb,bs] f32, latent_cache [nb,bs,576] bf16, q8 [B,H_I,d_I], q_scale [B]
+    (or [B,H_I] with q_scale_per_head), w [B,H_I], q [B,H,576], plus host copies ``ctx_host``
+    and ``max_ctx``.
     """
     rs = np.random.default_rng(int(seed))
     if ctx is None:
@@ -150,7 +161,8 @@ def decode_inputs(B, ctx_lo, ctx_hi, H_I, d_I, H, *, seed, device, block_size=64
     kscale = kscale.reshape(num_blocks, block_size)
     latent = _normal_bf16((num_blocks * block_size, D_QK), 1.0 / math.sqrt(D_QK), _gen(device, seed, 5), device)
     latent = latent.reshape(num_blocks, block_size, D_QK)
-    q8, q_scale = _indexer_operand((int(B), H_I, d_I), idx_std, False, _gen(device, seed, 1), device)
+    q8, q_scale = _indexer_operand((int(B), H_I, d_I), idx_std, False, _gen(device, seed, 1), device,
+                                   per_head=q_scale_per_head)
     w = _weights((int(B), H_I), w_dist, _gen(device, seed, 3), device)
     q = _normal_bf16((int(B), H, D_QK), 1.0 / math.sqrt(D_QK), _gen(device, seed, 4), device)
     return dict(ctx=torch.tensor(ctx, dtype=torch.int32, device=device), ctx_host=ctx.tolist(),
@@ -159,14 +171,15 @@ def decode_inputs(B, ctx_lo, ctx_hi, H_I, d_I, H, *, seed, device, block_size=64
                 w=w, q=q, block_size=block_size, num_blocks=num_blocks, H_I=H_I, d_I=d_I, H=H, B=int(B))
 
 
-def exact_prefill_inputs(seqlens, H_I, d_I, H, *, seed, device, small_scores=False):
+def exact_prefill_inputs(seqlens, H_I, d_I, H, *, seed, device, small_scores=False, q_scale_per_head=False):
     """Inputs on which every float32 partial sum of the indexer is exact.
 
     e4m3 codes of small integers |x| <= 4 (dots of 128 terms stay below 2^11), head weights
     multiples of 1/16 in [-1, 1], per-token scales powers of two.  Every partial sum of
     w * ReLU(dot) then needs at most 21 significant bits, so float32 accumulation in any
     order is exact and GPU and CPU scores agree bit for bit.
-    With small_scores the integers are in [-1, 1] (few distinct scores, many ties).
+    With small_scores the integers are in [-1, 1] (few distinct scores, many ties).  With
+    q_scale_per_head the query scales are drawn per (token, head), [T, H_I].
     """
     seqlens = [int(x) for x in seqlens]
     T = sum(seqlens)
@@ -178,6 +191,8 @@ def exact_prefill_inputs(seqlens, H_I, d_I, H, *, seed, device, small_scores=Fal
     k8 = torch.from_numpy(ints_k).to(torch.float8_e4m3fn).view(torch.uint8)
     q_scale = torch.from_numpy(2.0 ** rs.integers(-3, 2, size=T)).float()
     k_scale = torch.from_numpy(2.0 ** rs.integers(-3, 2, size=T)).float()
+    if q_scale_per_head:
+        q_scale = torch.from_numpy(2.0 ** rs.integers(-3, 2, size=(T, H_I))).float()
     w = torch.from_numpy(rs.integers(-16, 17, size=(T, H_I)) / 16.0).float()
     base = prefill_inputs(seqlens, H_I, d_I, H, seed=seed, device=device)
     base.update(q8=q8.to(device), k8=k8.to(device), q_scale=q_scale.to(device),
@@ -220,7 +235,7 @@ def seq_slice_numpy(inp: dict, b: int, rows=None):
         H_I, d_I = inp["q8"].shape[1], inp["q8"].shape[2]
         H = inp["q"].shape[1]
         q8 = np.zeros((L, H_I, d_I), np.uint8)
-        qs = np.ones(L)
+        qs = np.ones((L,) + tuple(inp["q_scale"].shape[1:]))
         w = np.zeros((L, H_I))
         q = np.zeros((L, H, D_QK))
         rl = list(rows)
@@ -248,7 +263,9 @@ def decode_seq_numpy(inp: dict, b: int, keep_paging: bool = True):
     else:
         pool = bt
         local = torch.arange(nb_used, device=bt.device)
-    return dict(q8=inp["q8"][b].cpu().numpy(), q_scale=float(inp["q_scale"][b].item()),
+    qs = inp["q_scale"][b]
+    return dict(q8=inp["q8"][b].cpu().numpy(),
+                q_scale=float(qs.item()) if qs.dim() == 0 else qs.double().cpu().numpy(),
                 w=inp["w"][b].double().cpu().numpy(), kcache8=inp["kcache8"][pool].cpu().numpy(),
                 kscale_cache=inp["kscale_cache"][pool].double().cpu().numpy(),
                 latent_cache=inp["latent_cache"][pool].float().cpu().numpy().astype(np.float64),

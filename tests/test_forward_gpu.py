@@ -68,6 +68,15 @@ def test_prefill_forward(name, seqlens, k, rows):
     _check_prefill(inp, k, rows_per_seq, out, idx)
 
 
+def test_prefill_forward_per_head_scales():
+    # one query scale per (token, head); heads drawn up to 128x apart in size
+    cfg = dict(synth.WORKLOADS["prefill_8k"])
+    cfg["seqlens"] = [1500, 700]
+    inp = synth.prefill_inputs(device="cuda", q_scale_per_head=True, **cfg)
+    out, lse, idx = _forward_prefill(inp, 1024)
+    _check_prefill(inp, 1024, [[0, 1023, 1024, 1499], [0, 350, 699]], out, idx)
+
+
 @pytest.mark.parametrize("name", ["prefill_8k", "prefill_2x32k", "prefill_128k"])
 def test_prefill_forward_full_size_sampled(name):
     cfg = dict(synth.WORKLOADS[name])
@@ -93,8 +102,8 @@ def _decode(d, k):
     return out, idx, keys
 
 
-@pytest.mark.parametrize("full", [False, True])
-def test_decode_forward(full):
+@pytest.mark.parametrize("full,per_head", [(False, False), (True, False), (False, True)])
+def test_decode_forward(full, per_head):
     import sparse_attention_09_b200 as dsa
     k = 2048
     if full:
@@ -103,7 +112,7 @@ def test_decode_forward(full):
         check = [0, 17, 63]
     else:
         d = synth.decode_inputs(B=6, ctx_lo=1, ctx_hi=9000, H_I=64, d_I=128, H=128, seed=8, device="cuda",
-                                ctx=[1, 64, 2047, 2048, 2049, 8999])
+                                ctx=[1, 64, 2047, 2048, 2049, 8999], q_scale_per_head=per_head)
         check = range(6)
     out, idx, keys = _decode(d, k)
     ld = ((d["max_ctx"] + 3) // 4) * 4

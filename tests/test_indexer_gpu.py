@@ -118,3 +118,78 @@ def test_decode_paged_scores_match_oracle():
         err = np.abs(S[b, :ctx] - ref)
         assert np.all(err <= 1e-3 * mag + 1e-30), f"seq {b}"
         assert np.all(np.isnan(S[b, ctx:])), "wrote past ctx"
+
+
+# ---- one query scale per (token, head) ------------------------------------------------------
+@pytest.mark.parametrize("H_I,d_I", [(64, 128), (4, 64)])
+def test_per_head_scales_exact_inputs_bit_identical(H_I, d_I):
+    seqlens = [333, 600]
+    inp = synth.exact_prefill_inputs(seqlens, H_I, d_I, 16, seed=17 + H_I, device="cuda", q_scale_per_head=True)
+    assert inp["q_scale"].shape == (sum(seqlens), H_I)
+    S = indexer_scores(inp).cpu().numpy()
+    k = 64
+    idx = indexer_topk(inp, k).cpu().numpy()
+    cu = inp["cu_seqlens"].cpu().numpy()
+    for b, L in enumerate(seqlens):
+        seq = synth.seq_slice_numpy(inp, b)
+        ref = oracle.indexer_scores(seq["q8"], seq["q_scale"], seq["w"], seq["k8"], seq["k_scale"]).astype(np.float32)
+        assert np.array_equal(S[cu[b]:cu[b + 1], :L], ref), "exact-arithmetic per-head scores differ"
+        assert np.array_equal(idx[cu[b]:cu[b + 1]], oracle.topk_rows(ref, np.arange(1, L + 1), k))
+
+
+def test_per_head_scales_match_oracle_and_fused_topk():
+    # heads drawn 2^-(j mod 8) apart, so their scales differ by up to 128x
+    inp, _ = _inputs("prefill_8k", seqlens=[900, 300], q_scale_per_head=True)
+    S = indexer_scores(inp)
+    Sn = S.cpu().numpy()
+    cu = inp["cu_seqlens"].cpu().numpy()
+    for b, L in enumerate(inp["seqlens"]):
+        seq = synth.seq_slice_numpy(inp, b)
+        rr = [0, 1, 127, 128, L // 2, L - 1]
+        I, A = oracle_scores(seq, rr)
+        for t, ref, mag in zip(rr, I, A):
+            assert_scores_close(Sn[cu[b] + t], ref, mag, t, L)
+    k = 256
+    idx = indexer_topk(inp, k).cpu().numpy()
+    for b, L in enumerate(inp["seqlens"]):
+        rows = np.arange(cu[b], cu[b + 1])
+        ref = oracle.topk_rows(Sn[rows], np.arange(1, L + 1), k)
+        assert np.array_equal(idx[rows], ref)
+
+
+def test_per_head_scales_row_blocks_equal_whole_sequence():
+    import sparse_attention_09_b200 as dsa
+    inp, _ = _inputs("prefill_8k", seqlens=[2000], q_scale_per_head=True)
+    k, H_I, d_I = 512, 64, 128
+    keys = dsa.contiguous_desc(inp["k8"], inp["cu_seqlens"], 2000, scale=inp["k_scale"])
+    whole = indexer_topk(inp, k)
+    for rb, re in [(0, 700), (700, 1333), (1333, 2000)]:
+        ib = torch.full((re - rb, k), -7, dtype=torch.int32, device="cuda")
+        dsa.dsa_indexer_topk_rows(inp["q8"][rb:re].contiguous(), inp["q_scale"][rb:re].contiguous(),
+                                  inp["w"][rb:re].contiguous(), keys, H_I, d_I, k, rb, re, ib)
+        torch.cuda.synchronize()
+        assert torch.equal(ib, whole[rb:re]), f"rows [{rb}, {re})"
+    assert dsa.dsa_device_error() == 0
+
+
+def test_decode_per_head_scales_match_oracle():
+    import sparse_attention_09_b200 as dsa
+    d = synth.decode_inputs(B=4, ctx_lo=1, ctx_hi=5000, H_I=64, d_I=128, H=16, seed=13, device="cuda",
+                            ctx=[1, 130, 2048 + 5, 4321], q_scale_per_head=True)
+    assert d["q_scale"].shape == (4, 64)
+    keys = dsa.paged_desc(d["kcache8"], d["block_table"], d["ctx"], d["max_ctx"], scale=d["kscale_cache"])
+    ld = ((d["max_ctx"] + 3) // 4) * 4
+    S = torch.full((4, ld), float("nan"), device="cuda")
+    dsa.dsa_indexer_scores(d["q8"], d["q_scale"], d["w"], keys, 4, 64, 128, 0, 4, S)
+    assert dsa.dsa_device_error() == 0
+    S = S.cpu().numpy()
+    for b in range(4):
+        seq = synth.decode_seq_numpy(d, b)
+        ref = oracle.decode_indexer_scores(seq["q8"], seq["q_scale"], seq["w"], seq["kcache8"],
+                                           seq["kscale_cache"], seq["block_table"], seq["ctx"])
+        k8 = oracle.paged_gather(seq["kcache8"], seq["block_table"], seq["ctx"])
+        ks = oracle.paged_gather(seq["kscale_cache"], seq["block_table"], seq["ctx"])
+        mag = oracle.indexer_magnitude_query(seq["q8"], seq["q_scale"], seq["w"], k8, ks)
+        ctx = seq["ctx"]
+        assert np.all(np.abs(S[b, :ctx] - ref) <= 1e-3 * mag + 1e-30), f"seq {b}"
+        assert np.all(np.isnan(S[b, ctx:])), "wrote past ctx"

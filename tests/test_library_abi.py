@@ -70,11 +70,25 @@ def test_row_block_entries_host_validation():
     d = dsa.KVDesc(dsa.DSA_KV_CONTIGUOUS, 4096, 4096, 4096, 0, 0, 100, 100, 0, 0, 0)
     ref = ctypes.byref(d)
     # empty blocks are no-ops even with NULL row arrays
-    assert lib.dsa_indexer_topk_rows(null, null, null, ref, 64, 128, 2048, 40, 40, null, null) == dsa.DSA_OK
+    assert lib.dsa_indexer_topk_rows(null, null, 1, null, ref, 64, 128, 2048, 40, 40, null, null) == dsa.DSA_OK
     assert lib.dsa_sparse_mla_prefill_rows(null, ref, null, 128, 2048, ctypes.c_float(0.04), 40, 40, null, null,
                                            null) == dsa.DSA_OK
     # bad ranges
-    assert lib.dsa_indexer_topk_rows(cu, cu, cu, ref, 64, 128, 2048, 50, 40, cu, null) == dsa.DSA_ERR_INVALID_ARGUMENT
-    assert lib.dsa_indexer_topk_rows(cu, cu, cu, ref, 64, 128, 2048, 0, 101, cu, null) == dsa.DSA_ERR_INVALID_ARGUMENT
+    assert lib.dsa_indexer_topk_rows(cu, cu, 1, cu, ref, 64, 128, 2048, 50, 40, cu, null) == dsa.DSA_ERR_INVALID_ARGUMENT
+    assert lib.dsa_indexer_topk_rows(cu, cu, 1, cu, ref, 64, 128, 2048, 0, 101, cu, null) == dsa.DSA_ERR_INVALID_ARGUMENT
+    # the query-scale granularity is 1 (per token) or H_I (per token and head), nothing else
+    for heads in (0, 2, 63, 65, -1):
+        assert lib.dsa_indexer_topk_rows(cu, cu, heads, cu, ref, 64, 128, 2048, 0, 40, cu, null) == \
+            dsa.DSA_ERR_INVALID_ARGUMENT
     assert lib.dsa_sparse_mla_prefill_rows(cu, ref, cu, 128, 2048, ctypes.c_float(0.04), -1, 4, cu, null,
                                            null) == dsa.DSA_ERR_INVALID_ARGUMENT
+
+
+def test_q_scale_heads_from_shape():
+    import torch
+
+    import sparse_attention_09_b200 as dsa
+    assert dsa._q_scale_heads(torch.ones(10), 64) == 1
+    assert dsa._q_scale_heads(torch.ones(10, 64), 64) == 64
+    with pytest.raises(ValueError):
+        dsa._q_scale_heads(torch.ones(10, 4), 64)
