@@ -19,8 +19,8 @@
  *     frees or synchronises (dsa_device_error is the one call that synchronises).  All work
  *     is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream).
  *   - Layouts are row-major and dense unless a leading dimension is given.  bf16 tensors are
- *     passed as `const void*`.  FP8 operands are OCP e4m3 bytes with one fp32 scale per token
- *     (dequantised value = e4m3(byte) * scale).
+ *     passed as `const void*`.  FP8 operands are OCP e4m3 bytes with fp32 scales: one per token,
+ *     or for indexer queries optionally one per (token, head) (dequantised value = e4m3(byte) * scale).
  *   - Indices are sequence-local token positions.  A prefill query at local position t has
  *     the causal prefix 0..t (min(k, t+1) entries are selected); a decode query sits at
  *     position ctx-1 and sees all ctx cached tokens.
