@@ -175,7 +175,8 @@ dsa_status dsa_sparse_mla_prefill(const void* q, const dsa_kv_desc* latent, cons
 /*
  * Sparse MLA decode: one query per sequence, q [B, H, 576]; idx [B, k] holds logical positions
  * (< ctx[b]) resolved through the paged latent cache (latent->kind == DSA_KV_PAGED).  The work
- * is split over the k selected rows; partial results go to `workspace`
+ * is split over the k selected rows (into more parts for fewer sequences, so that all the
+ * parts run in one round on the GPU); partial results go to `workspace`
  * (dsa_workspace_size(DSA_MODE_DECODE, ...) bytes) and are merged by log-sum-exp.
  */
 dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const int32_t* idx,
@@ -194,7 +195,8 @@ dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const
  *     current); make that first call before any stream capture.
  *   - Every call on a device shares the one array, which keeps the last call's contents: calls
  *     whose kernels overlap on the GPU (different streams, no ordering) race with each other.
- *   - Sizes whose partial results do not fit (B * H * splits * 2056 bytes, splits = min(4, k/64))
+ *   - Sizes whose partial results do not fit (B * H * splits * 2056 bytes; splits is the largest
+ *     power of two s with B * s <= 74 and s <= k/64, at least 1, so B * splits <= 74 for B <= 74)
  *     return DSA_ERR_UNSUPPORTED before any launch.
  */
 #define DSA_NOALLOC_SCRATCH_BYTES (32u << 20)

@@ -150,7 +150,6 @@ dsa_status indexer_common(const uint8_t* q_fp8, const float* q_scale, int32_t q_
 
 // ---- sparse MLA ------------------------------------------------------------------------------
 constexpr int kMlaClusters = 74;   // one CTA pair per two SMs of a 148-SM B200
-constexpr int kDecodeSplits = 4;   // decode: splits of each sequence's selection
 constexpr int kLatentDim = 576, kValueDim = 512;
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -159,7 +158,18 @@ size_t decode_partials_bytes(int B, int H, int splits) {
   return align256(static_cast<size_t>(B) * splits * H * kValueDim * 4) + align256(static_cast<size_t>(B) * splits * H * 2 * 4);
 }
 
-int decode_splits(int k) { return k / 64 < kDecodeSplits ? k / 64 : kDecodeSplits; }
+// Decode divides each sequence's selection into `splits` work units of whole 64-row chunks,
+// merged afterwards by a log-sum-exp combine.  Splitting pays only while the units still fit
+// one round on the CTA pairs: each unit costs a Q load, an O readout and fp32 partials, and
+// every chunk of a unit is one step of the same latency chain.  So splits is the largest power
+// of two s with B * s <= the number of CTA pairs (one round) and s <= k / 64 (a chunk per
+// unit), at least 1.  Measured on a B200 for 64 sequences, k = 2048 (MLA + combine): 1 split
+// 100 us, 2 splits 117 us, 4 splits 151 us, 8 splits 221 us.
+int decode_splits(int B, int k) {
+  int s = 1;
+  while (2 * s <= k / 64 && static_cast<int64_t>(B) * 2 * s <= kMlaClusters) s *= 2;
+  return s;
+}
 
 template <bool DECODE, bool DENSE = false>
 dsa_status launch_mla(const void* latent, const MlaParams& p, int64_t units, cudaStream_t s,
@@ -496,7 +506,7 @@ dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const
     return DSA_ERR_INVALID_ARGUMENT;
   if (!mla_shape_ok(H, k)) return DSA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(latent->num_blocks) * 64 > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
-  const int splits = decode_splits(k);
+  const int splits = decode_splits(B, k);
   if (workspace == nullptr || ws_bytes < decode_partials_bytes(B, H, splits) || !aligned(workspace, 256))
     return workspace == nullptr ? DSA_ERR_INVALID_ARGUMENT : DSA_ERR_WORKSPACE_TOO_SMALL;
   MlaParams p;
@@ -526,7 +536,7 @@ dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const dsa_kv_desc* laten
                                          int32_t H, int32_t k, float sm_scale, void* out, float* lse, void* stream) {
   if (B <= 0) return DSA_ERR_INVALID_ARGUMENT;
   if (!mla_shape_ok(H, k)) return DSA_ERR_UNSUPPORTED;
-  if (decode_partials_bytes(B, H, decode_splits(k)) > DSA_NOALLOC_SCRATCH_BYTES) return DSA_ERR_UNSUPPORTED;
+  if (decode_partials_bytes(B, H, decode_splits(B, k)) > DSA_NOALLOC_SCRATCH_BYTES) return DSA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   const dsa_status st = noalloc_scratch(&scratch);
   if (st != DSA_OK) return st;
@@ -558,7 +568,7 @@ dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale,
   if (workspace == nullptr) return DSA_ERR_INVALID_ARGUMENT;
   if (ws_bytes < need || !aligned(workspace, 256)) return DSA_ERR_WORKSPACE_TOO_SMALL;
   // workspace: [decode partials][scores B x ld][selection B x k]
-  const int splits = decode_splits(k);
+  const int splits = decode_splits(B, k);
   const size_t part = decode_partials_bytes(B, H, splits);
   const int64_t ld = (static_cast<int64_t>(keys->max_seqlen) + 3) / 4 * 4;
   float* scores = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + part);
@@ -579,7 +589,7 @@ size_t dsa_workspace_size(int32_t mode, int32_t B, int64_t total_tokens, int32_t
   if (B <= 0 || k <= 0 || H <= 0) return 0;
   if (mode == DSA_MODE_PREFILL) return align256(static_cast<size_t>(total_tokens > 0 ? total_tokens : 0) * k * 4);
   const int64_t ld = (static_cast<int64_t>(max_ctx > 0 ? max_ctx : 0) + 3) / 4 * 4;
-  return decode_partials_bytes(B, H, decode_splits(k)) + align256(static_cast<size_t>(B) * ld * 4) +
+  return decode_partials_bytes(B, H, decode_splits(B, k)) + align256(static_cast<size_t>(B) * ld * 4) +
          align256(static_cast<size_t>(B) * k * 4);
 }
 

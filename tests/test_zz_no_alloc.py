@@ -54,7 +54,7 @@ def test_noalloc_decode_rejects_sizes_beyond_its_scratch():
     import sparse_attention_09_b200 as dsa
     d, idx, B, k = _inputs()
     latent = dsa.paged_desc(d["latent_cache"], d["block_table"], d["ctx"], d["max_ctx"])
-    big_B = 4096  # partials of 4096 x 128 heads x 4 splits do not fit the fixed scratch
+    big_B = 4096  # partials of 4096 x 128 heads (1 split) need 1.08 GB: more than the fixed scratch
     st = dsa._lib.dsa_sparse_mla_decode_noalloc(
         ctypes.c_void_p(d["q"].data_ptr()), latent.ref(), ctypes.c_void_p(idx.data_ptr()), big_B, 128, k,
         ctypes.c_float(0.04), ctypes.c_void_p(d["q"].data_ptr()), None,
