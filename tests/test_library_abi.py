@@ -92,3 +92,23 @@ def test_q_scale_heads_from_shape():
     assert dsa._q_scale_heads(torch.ones(10, 64), 64) == 64
     with pytest.raises(ValueError):
         dsa._q_scale_heads(torch.ones(10, 4), 64)
+
+
+def test_decode_split_rule_through_workspace_size():
+    # Decode splits each selection into the largest power of two s of parts with B * s <= 74
+    # (CTA pairs: one round) and s <= k / 64, at least 1.  The workspace holds, per (sequence,
+    # split, head), 512 fp32 partial outputs and 2 fp32 (max, sum), then the scores
+    # (max_ctx = 0 here: none) and the selection.
+    import sparse_attention_09_b200 as dsa
+
+    def a256(x):
+        return (x + 255) // 256 * 256
+
+    def expected(B, H, k, s):
+        return a256(B * s * H * 512 * 4) + a256(B * s * H * 2 * 4) + a256(B * k * 4)
+
+    table = {1: 32, 2: 32, 3: 16, 5: 8, 9: 8, 10: 4, 18: 4, 19: 2, 37: 2, 38: 1, 64: 1, 200: 1}
+    for B, s in table.items():
+        assert dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, 0, 128, 64, 2048) == expected(B, 128, 2048, s), B
+    # k / 64 caps the count: two 64-row chunks allow two splits
+    assert dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, 1, 0, 0, 128, 64, 128) == expected(1, 128, 128, 2)
