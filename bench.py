@@ -368,7 +368,7 @@ def run_ours(args, world, rank, local):
                 "peak_source": f"{peak_src} (bf16 sustained x{'2 for e4m3' if dom == 'indexer_topk' else '1'})"}
 
     # ---- decode chain, same process ----
-    decode = run_decode(args, dsa, sm) if (rank == 0 and not args.no_decode) else None
+    decode = run_decode(args, dsa, sm, peaks) if (rank == 0 and not args.no_decode) else None
     next_rows = ({"f1_quantize_fp8": run_quantizer(dsa, peaks), "f2_masked_mla": run_masked(dsa, sm),
                   "f3_indexer_kl": run_kl(dsa, inp, idx, cfg, sm)}
                  if (rank == 0 and not args.no_decode) else None)
@@ -510,7 +510,7 @@ def run_kl(dsa, inp, idx, cfg, sm):
     return res
 
 
-def run_decode(args, dsa, sm):
+def run_decode(args, dsa, sm, peaks):
     cfg = dict(synth.WORKLOADS[DECODE])
     d = synth.decode_inputs(device="cuda", **cfg)
     B, k = d["B"], cfg["k"]
@@ -537,9 +537,49 @@ def run_decode(args, dsa, sm):
     assert dsa.dsa_device_error() == 0
     ms = e0.elapsed_time(e1) / n
     keys_scanned = int(sum(d["ctx_host"]))
+
+    # the same chain call by call, each kernel bracketed by events on the launching stream
+    ld = (d["max_ctx"] + 3) // 4 * 4
+    S = torch.empty((B, ld), device="cuda")
+    idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+    for i in range(-3, n):
+        e = ev[i] if i >= 0 else None
+        if e:
+            e[0].record()
+        dsa.dsa_indexer_scores(d["q8"], d["q_scale"], d["w"], keys, B, 64, 128, 0, B, S)
+        if e:
+            e[1].record()
+        dsa.dsa_topk(S, d["ctx"], k, idx)
+        if e:
+            e[2].record()
+        dsa.dsa_sparse_mla_decode(d["q"], lat, idx, B, 128, k, sm, out, None, ws)
+        if e:
+            e[3].record()
+    torch.cuda.synchronize()
+    assert dsa.dsa_device_error() == 0
+    t = [float(np.mean([e[j].elapsed_time(e[j + 1]) for e in ev])) for j in range(3)]
+    hbm = peaks["hbm_gbs"]
+    # algorithmic bytes: the indexer reads 132 B per cached key (e4m3 key + fp32 scale) and each
+    # query's q_I, w and scale, and writes a 4-byte score per key; top-k reads the scores and
+    # writes the selection; sparse MLA gathers 1152 B per selected row and reads q, writes out
+    idx_bytes = keys_scanned * (132 + 4) + B * (64 * 128 + 64 * 4 + 4)
+    topk_bytes = keys_scanned * 4 + B * k * 4
+    mla_bytes = B * k * 1152 + B * 128 * 576 * 2 + B * 128 * 512 * 2 + B * k * 4
+    mla_flops = B * k * 278528
+    kernels = {
+        "indexer_scores": {"ms": t[0], "bytes": idx_bytes, "gbs": idx_bytes / (t[0] * 1e-3) / 1e9},
+        "topk": {"ms": t[1], "bytes": topk_bytes, "gbs": topk_bytes / (t[1] * 1e-3) / 1e9},
+        "sparse_mla_decode": {"ms": t[2], "bytes": mla_bytes, "gbs": mla_bytes / (t[2] * 1e-3) / 1e9,
+                              "tflops": mla_flops / (t[2] * 1e-3) / 1e12,
+                              "frac_of_bf16": mla_flops / (t[2] * 1e-3) / 1e12 / peaks["bf16_tflops"]},
+    }
+    for kk in kernels.values():
+        kk["frac_of_hbm"] = kk["gbs"] / hbm
     return {"workload": f"{DECODE}: 64 sequences, ctx ~ U[8192,131072] (sum {keys_scanned}), paged 64-token blocks",
             "value": B / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": n,
-            "indexer_key_bytes": keys_scanned * 132, "indexer_gbs_equiv": keys_scanned * 132 / (ms * 1e-3) / 1e9,
+            "kernels": kernels, "peaks": {"hbm_gbs": hbm, "bf16_tflops": peaks["bf16_tflops"],
+                                          "note": "measured; burst bf16 (kernels timed alone)"},
             "gpu_launches_per_step": 4}
 
 
