@@ -29,8 +29,14 @@
  *   - Host-side validation runs before any launch: NULL or misaligned pointers and
  *     inconsistent sizes return DSA_ERR_INVALID_ARGUMENT, shapes outside the supported set
  *     return DSA_ERR_UNSUPPORTED, a launch failure returns DSA_ERR_CUDA.  Errors found on the
- *     device (a bounded wait that expired, NaN scores) are recorded in a per-process device
- *     error word and reported by dsa_device_error().
+ *     device are recorded in a per-process device error word and reported by
+ *     dsa_device_error(): a bounded wait that expired (DSA_ERR_TIMEOUT), or an input only the
+ *     GPU reads that contradicts the host arguments (DSA_ERR_DEVICE_CHECK): a NaN index score;
+ *     a selection entry that is neither -1 nor a position of its sequence (the entry is
+ *     masked); a block-table entry of a position inside the context that is not a block of the
+ *     pool (that position is masked: no load is made through it); a context length above the
+ *     descriptor's max_seqlen, or a top-k row length outside [0, ld_scores] (clamped).  Results
+ *     that do not depend on the offending input are those of a clean call.
  *   - Supported shapes: indexer heads H_I in {4, 64} with d_I in {64, 128}; query heads
  *     H = 128 (prefill and decode) or 16 (prefill only); latent dim 576 with value dim 512;
  *     1 <= k <= 2048 with k a multiple of 64 for attention; paged block size 64.
@@ -52,7 +58,7 @@ typedef enum {
   DSA_ERR_WORKSPACE_TOO_SMALL = 3,
   DSA_ERR_CUDA = 4,
   DSA_ERR_TIMEOUT = 5,      /* a device-side bounded wait expired */
-  DSA_ERR_DEVICE_CHECK = 6  /* a device-side input check failed (e.g. NaN index score) */
+  DSA_ERR_DEVICE_CHECK = 6  /* a device-side input check failed (NaN score, index or length out of range) */
 } dsa_status;
 
 typedef enum { DSA_KV_CONTIGUOUS = 0, DSA_KV_PAGED = 1 } dsa_kv_kind;

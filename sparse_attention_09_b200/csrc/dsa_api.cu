@@ -141,6 +141,8 @@ dsa_status indexer_common(const uint8_t* q_fp8, const float* q_scale, int32_t q_
     p->block_table = keys->block_table;
     p->context_lens = keys->context_lens;
     p->max_blocks_per_seq = keys->max_blocks_per_seq;
+    p->num_blocks = keys->num_blocks;
+    p->max_len = keys->max_seqlen;  // validated above: 0 < max_seqlen <= 64 * max_blocks_per_seq
     p->tiles_per_cta = kDecodeTilesPerCta;
   } else {
     return DSA_ERR_INVALID_ARGUMENT;
@@ -516,6 +518,7 @@ dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const
   p.block_table = latent->block_table;
   p.context_lens = latent->context_lens;
   p.max_blocks_per_seq = latent->max_blocks_per_seq;
+  p.num_blocks = latent->num_blocks;
   p.B = B;
   p.H = H;
   p.k = k;

@@ -47,6 +47,8 @@ struct IndexerParams {
   const int32_t* block_table; // decode [B, max_blocks_per_seq]
   const int32_t* context_lens;// decode [B]
   int32_t max_blocks_per_seq;
+  int32_t num_blocks;         // decode: blocks in the paged key pool
+  int32_t max_len;            // decode: the declared longest context (<= 64 * max_blocks_per_seq)
   int32_t tiles_per_cta;      // decode: key tiles per CTA
   float* scores;              // kIdxScores output
   int64_t ld;
@@ -150,7 +152,11 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
     q_row = (static_cast<int64_t>(seq_start + t0) - p.q_row0) * H_I;
   } else {
     if (b < p.row_begin || b >= p.row_end) return;
-    len = min(p.context_lens[b], p.max_blocks_per_seq * 64);  // never read past the block table row
+    // never read past the block table row nor write past the declared longest context (the
+    // width of the caller's score rows): a longer context is an input error
+    const int ctx = p.context_lens[b];
+    if (ctx > p.max_len && blockIdx.x == 0 && threadIdx.x == 0) record_device_error(DSA_ERR_DEVICE_CHECK);
+    len = min(ctx, p.max_len);
     tile0 = static_cast<int>(blockIdx.x) * p.tiles_per_cta;
     const int total_tiles = (len + 127) / 128;
     if (tile0 >= total_tiles) return;
@@ -291,7 +297,11 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
       float ksc = 0.f;                       // k_scale of this lane's key (0 beyond the sequence)
       if (s < len) {
         if constexpr (!PAGED) ksc = p.k_scale[seq_start + s];
-        else ksc = p.k_scale[static_cast<int64_t>(bt[s >> 6]) * 64 + (s & 63)];
+        else {
+          const int blk = bt[s >> 6];
+          if (blk >= 0 && blk < p.num_blocks) ksc = p.k_scale[static_cast<int64_t>(blk) * 64 + (s & 63)];
+          else record_device_error(DSA_ERR_DEVICE_CHECK);  // a block id outside the key pool
+        }
       }
       const bool ok = mbar_wait(&bar_accfull[acc], aph);
       if (!ok) record_device_error(DSA_ERR_TIMEOUT);

@@ -58,6 +58,7 @@ struct MlaParams {
   const int32_t* block_table; // decode [B, max_blocks_per_seq]
   const int32_t* context_lens;// decode [B]
   int32_t max_blocks_per_seq;
+  int32_t num_blocks;         // decode: blocks in the paged latent pool
   int32_t B;
   int32_t H;                  // query heads (<= 128; rows >= H are padding)
   int32_t k;                  // selected entries per row (multiple of 64)
@@ -331,6 +332,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
       unit_chunks(qrow, kbeg, kend, seq_start, c0, c1);
       const int32_t* row = p.idx + qrow * p.k;
       const int32_t* bt = DECODE ? p.block_table + static_cast<int64_t>(seq) * p.max_blocks_per_seq : nullptr;
+      // masked rows still copy a real row (never NaN bits): the sequence's first key; in decode
+      // the first row of its first block when that block id lies in the pool, else pool row 0
+      int pad_row = seq_start;
+      if constexpr (DECODE) {
+        const int b0 = bt[0];
+        pad_row = (b0 >= 0 && b0 < p.num_blocks) ? b0 * 64 : 0;
+      }
       for (int c = c0; c < c1; ++c, ++g) {
         const int stage = static_cast<int>(g % kStages);
         if (!mbar_wait(&bar_kvempty[stage], ((g / kStages) & 1u) ^ 1u)) {
@@ -339,11 +347,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::kThreads, 1)
           break;
         }
         const int v = row[c * kChunk + 32 * pw + lane];
-        const bool valid = v >= 0 && v < seq_len;
-        const int pos = valid ? v : 0;  // masked rows still copy a real row (never NaN bits)
-        int prow;
-        if constexpr (DECODE) prow = bt[pos >> 6] * 64 + (pos & 63);
-        else prow = seq_start + pos;
+        bool valid = v >= 0 && v < seq_len;
+        bool bad = !valid && v != -1;  // neither padding nor a position of the sequence
+        int prow = pad_row;
+        if constexpr (DECODE) {
+          const int blk = valid ? bt[v >> 6] : 0;
+          const bool blk_ok = blk >= 0 && blk < p.num_blocks;  // a block id outside the pool
+          bad = bad || (valid && !blk_ok);
+          valid = valid && blk_ok;
+          if (valid) prow = blk * 64 + (v & 63);
+        } else {
+          if (valid) prow = seq_start + v;
+        }
+        if (bad) record_device_error(DSA_ERR_DEVICE_CHECK);  // the entry is masked
         const uint32_t vbits = __ballot_sync(0xffffffffu, valid);
         if (lane == 0) reinterpret_cast<uint32_t*>(&s_vmask[stage])[pw] = vbits;
         const uint32_t st = smem_addr(sKV + stage * kStageBytes);

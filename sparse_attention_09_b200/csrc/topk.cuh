@@ -65,7 +65,11 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
   const int64_t r = blockIdx.x / C;
   const float* row = scores + r * ld;
   int32_t* out = idx + r * static_cast<int64_t>(k);
-  const int n = row_len[r];
+  int n = row_len[r];
+  if (n < 0 || n > ld) {  // a row length outside [0, ld] is an input error; the row is clamped
+    if (threadIdx.x == 0 && rank == 0) record_device_error(DSA_ERR_DEVICE_CHECK);
+    n = n < 0 ? 0 : static_cast<int>(ld);
+  }
 
   if (n <= k) {  // every candidate is selected (the same decision in every CTA of the row)
     if (rank == 0)
