@@ -119,6 +119,57 @@ def test_per_head_quantisation_tracks_heads_of_different_magnitude():
     assert err_t.mean() > 10 * err_h.mean()
 
 
+def test_single_head_unit_weight_is_scaled_relu_matmul():
+    # H_I = 1, w = 1: I = ReLU(Q K^T) on the dequantised operands, causal-masked.
+    rs = np.random.default_rng(5)
+    L, d_I = 40, 16
+    q8, q_scale, w, k8, k_scale = _random_case(rs, L=L, H_I=1, d_I=d_I)
+    w[:] = 1.0
+    tab = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64)
+    Q = tab[torch.from_numpy(q8[:, 0, :]).long()] * torch.from_numpy(q_scale)[:, None]
+    K = tab[torch.from_numpy(k8).long()] * torch.from_numpy(k_scale)[:, None]
+    ref = torch.relu(Q @ K.T)
+    ref = ref.masked_fill(torch.triu(torch.ones(L, L, dtype=torch.bool), 1), float("-inf")).numpy()
+    assert _close(oracle.indexer_scores(q8, q_scale, w, k8, k_scale), ref, rtol=1e-13)
+
+
+def test_hand_worked_example():
+    g = json.load(open(GOLDEN))["indexer"]
+    got = oracle.indexer_scores(np.array(g["q8"], np.uint8), np.array(g["q_scale"]), np.array(g["w"]),
+                                np.array(g["k8"], np.uint8), np.array(g["k_scale"]))
+    exp = np.array([[float(x) for x in row] for row in g["expected_scores"]])
+    assert np.array_equal(got, exp)
+
+
+def test_causal_prefix_and_linearity_in_w():
+    rs = np.random.default_rng(9)
+    q8, q_scale, w, k8, k_scale = _random_case(rs, L=12, H_I=4, d_I=8)
+    I = oracle.indexer_scores(q8, q_scale, w, k8, k_scale)
+    assert all(np.isfinite(I[t, : t + 1]).all() and np.isneginf(I[t, t + 1:]).all() for t in range(12))
+    w2 = rs.normal(size=w.shape)
+    I2 = oracle.indexer_scores(q8, q_scale, w2, k8, k_scale)
+    I12 = oracle.indexer_scores(q8, q_scale, w + w2, k8, k_scale)
+    fin = np.isfinite(I)
+    assert np.allclose(I12[fin], I[fin] + I2[fin], rtol=1e-12, atol=1e-12)
+
+
+def test_relu_zeroes_negative_dot_products():
+    # keys pointing against every head's query contribute nothing, whatever the weights
+    q8 = np.full((2, 3, 4), 0x38, np.uint8)                      # every q entry = 1
+    k8 = np.array([[0x38] * 4, [0xB8] * 4], np.uint8)            # key0 = +1s, key1 = -1s
+    I = oracle.indexer_scores(q8, np.ones(2), np.array([[1.0, -2.0, 3.0]] * 2), k8, np.ones(2))
+    assert I[1, 1] == 0.0 and I[1, 0] == 4.0 * (1 - 2 + 3)
+
+
+def test_magnitude_bounds_score():
+    rs = np.random.default_rng(3)
+    q8, q_scale, w, k8, k_scale = _random_case(rs, L=8, H_I=4, d_I=8)
+    for t in range(8):
+        I = oracle.indexer_scores_query(q8[t], q_scale[t], w[t], k8[: t + 1], k_scale[: t + 1])
+        A = oracle.indexer_magnitude_query(q8[t], q_scale[t], w[t], k8[: t + 1], k_scale[: t + 1])
+        assert np.all(np.abs(I) <= A * (1 + 1e-12))
+
+
 # ---- planted mistakes: each must be caught by a pin above -----------------------------------
 def _mutant(kind):
     def f(q8, q_scale, w, k8, k_scale):
