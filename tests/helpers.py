@@ -1,12 +1,10 @@
 """Shared helpers for the GPU parity tests: run the library on synth inputs, run the oracle on
 host copies of the same inputs, and compare under the tolerances the method states."""
-import math
 
 import numpy as np
 import torch
 
 import oracle
-import synth
 
 
 def lib():
