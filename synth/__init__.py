@@ -15,4 +15,5 @@ from .inputs import (  # noqa: F401
     sample_rows,
     seq_slice_numpy,
     decode_seq_numpy,
+    SampledRows,
 )

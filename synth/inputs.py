@@ -218,10 +218,24 @@ def sample_rows(L: int, k: int, count: int, seed: int):
     return sorted(set(fixed + rest))
 
 
+class SampledRows:
+    """The rows of a per-token array for a sample of tokens only: ``x[t]`` is token t's row
+    (a KeyError for a token outside the sample) and ``shape`` is the whole array's, so code
+    written against the whole array reads the sample without it being allocated."""
+
+    def __init__(self, rows: dict, shape):
+        self._rows = {int(t): v for t, v in rows.items()}
+        self.shape = tuple(shape)
+
+    def __getitem__(self, t):
+        return self._rows[int(t)]
+
+
 def seq_slice_numpy(inp: dict, b: int, rows=None):
     """Host copies (numpy) of sequence b of prefill inputs, for the oracle.
 
-    rows restricts q and the indexer queries to those local rows (keys stay whole)."""
+    rows restricts q and the indexer queries to those local rows (keys stay whole); q is then
+    a SampledRows (a whole [L, H, 576] float64 q of a long sequence would take tens of GB)."""
     s0 = int(inp["cu_seqlens"][b].item())
     s1 = int(inp["cu_seqlens"][b + 1].item())
     out = dict(k8=inp["k8"][s0:s1].cpu().numpy(), k_scale=inp["k_scale"][s0:s1].double().cpu().numpy(),
@@ -237,12 +251,12 @@ def seq_slice_numpy(inp: dict, b: int, rows=None):
         q8 = np.zeros((L, H_I, d_I), np.uint8)
         qs = np.ones((L,) + tuple(inp["q_scale"].shape[1:]))
         w = np.zeros((L, H_I))
-        q = np.zeros((L, H, D_QK))
         rl = list(rows)
         q8[rl] = inp["q8"][r].cpu().numpy()
         qs[rl] = inp["q_scale"][r].double().cpu().numpy()
         w[rl] = inp["w"][r].double().cpu().numpy()
-        q[rl] = inp["q"][r].float().cpu().numpy().astype(np.float64)
+        qr = inp["q"][r].float().cpu().numpy().astype(np.float64)
+        q = SampledRows({t: qr[i] for i, t in enumerate(rl)}, (L, H, D_QK))
         out.update(q8=q8, q_scale=qs, w=w, q=q)
     return out
 
