@@ -267,10 +267,12 @@ dsa_status dsa_indexer_kl(const float* p, const float* scores, const int32_t* id
 dsa_status dsa_selftest_wait_timeout(int32_t limit_us, void* stream);
 
 /*
- * Per-token FP8 quantiser for the indexer operands (the step that produces a2's input
- * contract; "DeepSeek-V3.2 论文解读", section 二, subsection "工作原理": the indexer runs in FP8).  For each row r
- * of x [rows, cols] bf16 (row-major, contiguous; one token: all of its indexer heads for
- * q_I, its key for k_I):
+ * Per-row FP8 quantiser for the indexer operands (the step that produces the indexer's input
+ * contract; "DeepSeek-V3.2 论文解读", section 二, subsection "工作原理": the indexer runs in
+ * FP8).  For each row r of x [rows, cols] bf16 (row-major, contiguous), where a row is a key of
+ * k_I, or the queries of one token (all H_I heads: one q scale per token, q_scale_heads = 1),
+ * or one (token, head) query of q_I passed as [T * H_I, d_I] (one q scale per head,
+ * q_scale_heads = H_I):
  *   scale[r] = amax_c |x[r,c]| / 448 in IEEE fp32 (1 for an all-zero row),
  *   codes[r*cols + c] = e4m3(x[r,c] / scale[r]), the quotient in IEEE fp32 rounded to the
  *   nearest e4m3 value (ties to even), saturating at +-448.  NaN elements take no part in
