@@ -112,3 +112,27 @@ def test_decode_split_rule_through_workspace_size():
         assert dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, 0, 128, 64, 2048) == expected(B, 128, 2048, s), B
     # k / 64 caps the count: two 64-row chunks allow two splits
     assert dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, 1, 0, 0, 128, 64, 128) == expected(1, 128, 128, 2)
+
+
+def test_decode_split_count_partitions_every_selection():
+    # Decode split sp of a sequence takes the 64-row chunks [floor(sp * per / 64),
+    # floor((sp + 1) * per / 64)) with per = k / splits.  For every batch size and every
+    # supported k, the split count the library picks (read back through the workspace size)
+    # must divide k and leave no split empty, so the splits partition the selection's chunks
+    # exactly: an empty split would be made to repeat a chunk.
+    import sparse_attention_09_b200 as dsa
+
+    def a256(x):
+        return (x + 255) // 256 * 256
+
+    for k in range(64, 2049, 64):
+        for B in range(1, 257):
+            ws = dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, 0, 128, 64, k)
+            base = a256(B * k * 4)
+            s = next(s for s in (1, 2, 4, 8, 16, 32)
+                     if a256(B * s * 128 * 512 * 4) + a256(B * s * 128 * 2 * 4) + base == ws)
+            assert k % s == 0 and s <= k // 64, (B, k, s)
+            per = k // s
+            bounds = [sp * per // 64 for sp in range(s)] + [k // 64]
+            assert all(bounds[i] < bounds[i + 1] for i in range(s)), (B, k, s)
+            assert B * s <= 74 or s == 1, (B, k, s)   # one round on the CTA pairs
