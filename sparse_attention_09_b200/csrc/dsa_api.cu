@@ -17,6 +17,7 @@
 #include "indexer_kl.cuh"
 #include "selftest.cuh"
 #include "sparse_mla.cuh"
+#include "sparse_mla_pair.cuh"
 #include "topk.cuh"
 
 namespace dsa {
@@ -185,6 +186,24 @@ dsa_status launch_mla(const void* latent, const MlaParams& p, int64_t units, cud
   const int clusters = static_cast<int>(units < kMlaClusters ? units : kMlaClusters);
   kern<<<2 * clusters, mla::kThreads, smem, s>>>(static_cast<const __nv_bfloat16*>(latent), p,
                                                   nope_map ? *nope_map : unused, rope_map ? *rope_map : unused);
+  return launch_status();
+}
+
+// Sparse prefill and decode: the head-split pair kernel.  Q is read by TMA as a [q_rows * H, 576]
+// bf16 matrix in 64 x 64 tiles (128-byte swizzle).
+template <bool DECODE>
+dsa_status launch_mla_pair(const void* latent, const void* q, int64_t q_rows, const MlaParams& p, int64_t units,
+                           cudaStream_t s) {
+  CUtensorMap qm;
+  if (!make_map_2d(&qm, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kLatentDim, static_cast<uint64_t>(q_rows) * p.H,
+                   kLatentDim * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_INVALID_ARGUMENT;
+  auto kern = sparse_mla_pair_kernel<DECODE>;
+  const int smem = mlap::kSmemBytes + 1024;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  const int clusters = static_cast<int>(units < kMlaClusters ? units : kMlaClusters);
+  kern<<<2 * clusters, mlap::kThreads, smem, s>>>(static_cast<const __nv_bfloat16*>(latent), p, qm);
   return launch_status();
 }
 
@@ -431,7 +450,7 @@ dsa_status dsa_sparse_mla_prefill_rows(const void* q, const dsa_kv_desc* latent,
   p.scale_log2 = sm_scale * 1.4426950408889634f;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  return launch_mla<false>(latent->data, p, p.rows, as_stream(stream));
+  return launch_mla_pair<false>(latent->data, q, p.rows, p, p.rows, as_stream(stream));
 }
 
 dsa_status dsa_sparse_mla_prefill(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B, int32_t H,
@@ -457,7 +476,7 @@ dsa_status dsa_sparse_mla_prefill(const void* q, const dsa_kv_desc* latent, cons
   p.scale_log2 = sm_scale * 1.4426950408889634f;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  return launch_mla<false>(latent->data, p, p.rows, as_stream(stream));
+  return launch_mla_pair<false>(latent->data, q, p.rows, p, p.rows, as_stream(stream));
 }
 
 dsa_status dsa_masked_mla_prefill(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B, int32_t H,
@@ -529,7 +548,7 @@ dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const
   p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                        align256(static_cast<size_t>(B) * splits * H * kValueDim * 4));
   cudaStream_t s = as_stream(stream);
-  dsa_status st = launch_mla<true>(latent->data, p, static_cast<int64_t>(B) * splits, s);
+  dsa_status st = launch_mla_pair<true>(latent->data, q, B, p, static_cast<int64_t>(B) * splits, s);
   if (st != DSA_OK) return st;
   mla_combine_kernel<<<dim3(H, B), 128, 0, s>>>(p.part_o, p.part_ml, splits, H, static_cast<__nv_bfloat16*>(out), lse);
   return launch_status();

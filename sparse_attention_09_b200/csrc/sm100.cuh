@@ -113,6 +113,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Same, spinning on the non-blocking probe: for waits on the critical path, where a thread that
+// try_wait suspended can resume well after the phase completes.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_addr(bar);
+  if (mbar_poll(a, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_poll(a, parity)) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
 // Same, with cluster-scope acquire: used where the arrivals come from the peer CTA.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_addr(bar);
@@ -407,6 +421,102 @@ __device__ __forceinline__ void umma_e4m3_ss(uint32_t d_tmem, uint64_t a_desc, u
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
                : "memory");
+}
+
+// ---------------------------------------------------------------------------------------
+// tcgen05 on a CTA pair (cta_group::2).  A kernel that uses these uses no cta_group::1
+// tcgen05 instruction: allocation, MMA and commit all name the pair.
+// ---------------------------------------------------------------------------------------
+// Warp-collective, run by the same warp index in both CTAs of the pair; each CTA's copy of
+// *dst receives the (common) TMEM base address.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Issued by one thread of the even CTA of the pair.  A (M/2 rows per CTA) and B (N/2 rows per
+// CTA) are read from the same shared-memory offsets in both CTAs; each CTA's TMEM receives its
+// M/2 rows x N columns of D (for M = 128: columns [0, N/2) on lanes 0-63, [N/2, N) on lanes 64-127).
+__device__ __forceinline__ void umma_bf16_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                  uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Warp-collective form of the above: every lane passes the same (warp-uniform) operands and one
+// elected lane issues.  Measured on B200 for M = 128, N = 64: 25 cycles per MMA (the shared-memory
+// operand rate) against 45 when one lane builds the descriptors and issues inside a lane branch.
+__device__ __forceinline__ void umma_bf16_ss_pair_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Same, A from tensor memory (each CTA's 64 rows of A held twice: rows 0-31 on lanes 0-31 and
+// 64-95, rows 32-63 on lanes 32-63 and 96-127; K = 16 bf16 = 8 columns per instruction).
+__device__ __forceinline__ void umma_bf16_ts_pair_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Copies a 64-row x 16-byte slice of a shared-memory matrix (described like an MMA operand) into
+// tensor memory of both CTAs of the pair, rows 0-31 to lanes 0-31 and 64-95, rows 32-63 to lanes
+// 32-63 and 96-127 (the layout of a pair MMA's A operand in tensor memory), 4 columns.  Issued by
+// one elected lane; ordered with the same thread's later tcgen05.mma.
+__device__ __forceinline__ void tmem_cp_pair_64x128b_warp(uint32_t taddr, uint64_t s_desc) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.cp.cta_group::2.64x128b.warpx2::02_13 [%0], %1;\n\t}\n" ::"r"(taddr),
+      "l"(s_desc)
+      : "memory");
+}
+
+// Arrive (once) on the barrier at the same shared-memory offset in every CTA of `cta_mask`
+// when all previously issued pair MMAs of this thread complete.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_addr(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
+// Arrive on a barrier of any CTA of the cluster (default semantics: release at CTA scope).  The
+// arrivals that use it order no generic-memory data for the waiter: tensor-memory reads are
+// ordered by tcgen05 fences and shared-memory operands by the writer's async-proxy fence, so the
+// costlier cluster-scope release (a cluster-wide memory fence per arrival) is not needed.
+__device__ __forceinline__ void mbar_arrive_peer(uint32_t cluster_bar_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar_addr) : "memory");
+}
+
+// Non-blocking probe with cluster-scope acquire (the barrier receives arrivals from the peer).
+__device__ __forceinline__ bool mbar_poll_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 
 // ---------------------------------------------------------------------------------------
