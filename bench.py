@@ -516,7 +516,7 @@ def run_decode(args, dsa, sm, peaks):
     B, k = d["B"], cfg["k"]
     keys = dsa.paged_desc(d["kcache8"], d["block_table"], d["ctx"], d["max_ctx"], scale=d["kscale_cache"])
     lat = dsa.paged_desc(d["latent_cache"], d["block_table"], d["ctx"], d["max_ctx"])
-    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, 64, k), dtype=torch.uint8,
+    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, k), dtype=torch.uint8,
                      device="cuda")
     out = torch.empty((B, 128, 512), dtype=torch.bfloat16, device="cuda")
 

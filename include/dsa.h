@@ -125,7 +125,10 @@ dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, int32_t 
                             void* stream);
 
 /*
- * Top-k selection (method step 2) over score rows: for row r the first row_len[r] entries
+ * Top-k selection (method step 2: the index scores pick the k = 2048 highest-scoring tokens
+ * of each query -- "DeepSeek-V3.2 论文解读", section 二, subsection "工作原理" and table
+ * "附：DSA 关键参数"; 36881.com.cn digest, "第二步：Fine-grained Token Selection") over score
+ * rows: for row r the first row_len[r] entries
  * of scores[r*ld_scores ...] are candidates; idx[r*k ...] receives the indices of the
  * min(k, row_len[r]) largest (ties -> lower index), ascending, -1 padded.  row_len is a device
  * array.  scores must be 16-byte aligned and ld_scores a multiple of 4.  NaN scores set
@@ -134,13 +137,6 @@ dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, int32_t 
 dsa_status dsa_topk(const float* scores, int64_t ld_scores, int64_t rows, const int32_t* row_len,
                     int32_t k, int32_t* idx, void* stream);
 
-/*
- * Sparse MLA prefill (method step 3): for every packed query token t and head h,
- *   out[t,h,:] = sum_i softmax_i(sm_scale * q[t,h,:] . c[idx[t,i],:]) * c[idx[t,i], 0:512]
- * over the valid (>= 0) entries of idx [T, k]; c is the contiguous latent of t's sequence.
- * q [T, H, 576] bf16, out [T, H, 512] bf16, lse [T, H] fp32 natural log (may be NULL).
- * Every row must hold at least one valid index.
- */
 /*
  * Row blocks of one sequence, for sharding a long prefill over GPUs by query rows (each GPU
  * holds every key and latent row -- gathered from the others -- and its own block of query
@@ -174,12 +170,24 @@ dsa_status dsa_sparse_mla_prefill_rows(const void* q, const dsa_kv_desc* latent,
 dsa_status dsa_masked_mla_prefill(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B,
                                   int32_t H, int32_t k, float sm_scale, void* out, float* lse, void* stream);
 
+/*
+ * Sparse MLA prefill (method step 3: attention runs only over the selected entries, on MLA in
+ * MQA mode, where one latent row per token is the key of every query head and its first 512
+ * dims are the value -- "DeepSeek-V3.2 论文解读", section 二, subsection "挂在 MLA 上"; jienda.com
+ * section 2.1 on MLA's latent K/V): for every packed query token t and head h,
+ *   out[t,h,:] = sum_i softmax_i(sm_scale * q[t,h,:] . c[idx[t,i],:]) * c[idx[t,i], 0:512]
+ * over the valid (>= 0) entries of idx [T, k]; c is the contiguous latent of t's sequence.
+ * q [T, H, 576] bf16, out [T, H, 512] bf16, lse [T, H] fp32 natural log (may be NULL).
+ * A row without a valid index gets out = 0 and lse = -INFINITY.
+ */
 dsa_status dsa_sparse_mla_prefill(const void* q, const dsa_kv_desc* latent, const int32_t* idx,
                                   int32_t B, int32_t H, int32_t k, float sm_scale, void* out,
                                   float* lse, void* stream);
 
 /*
- * Sparse MLA decode: one query per sequence, q [B, H, 576]; idx [B, k] holds logical positions
+ * Sparse MLA decode (method step 3 for the decode step the pages' long-context cost curves
+ * measure -- "DeepSeek-V3.2 论文解读", section 二, subsection "等性能验证"; techwalker.com,
+ * section 五 "成本效益与部署优势"): one query per sequence, q [B, H, 576]; idx [B, k] holds logical positions
  * (< ctx[b]) resolved through the paged latent cache (latent->kind == DSA_KV_PAGED).  The work
  * is split over the k selected rows (into more parts for fewer sequences, so that all the
  * parts run in one round on the GPU); partial results go to `workspace`
@@ -198,12 +206,15 @@ dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const
  * all device memory to its own pool at start-up, or a latency-critical loop that cannot
  * afford cudaMalloc's implicit device-wide synchronisation.
  *   - The first call on a device looks up the array's device address (with that device
- *     current); make that first call before any stream capture.
+ *     current); make that first call before any stream capture.  The address is cached for the
+ *     life of the device's primary context: after cudaDeviceReset (or anything else that tears
+ *     that context down) this entry point must not be called again in the process.
  *   - Every call on a device shares the one array, which keeps the last call's contents: calls
  *     whose kernels overlap on the GPU (different streams, no ordering) race with each other.
  *   - Sizes whose partial results do not fit (B * H * splits * 2056 bytes; splits is the largest
  *     power of two s with B * s <= 74 and s <= k/64, at least 1, so B * splits <= 74 for B <= 74)
- *     return DSA_ERR_UNSUPPORTED before any launch.
+ *     return DSA_ERR_UNSUPPORTED before any launch: at H = 128 every B <= 127 fits and B = 128
+ *     does not.
  */
 #define DSA_NOALLOC_SCRATCH_BYTES (32u << 20)
 dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B,
@@ -211,7 +222,9 @@ dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const dsa_kv_desc* laten
                                          void* stream);
 
 /*
- * Whole DSA forward.
+ * Whole DSA forward (method steps 1-3: lightning indexer, fine-grained top-k selection, sparse
+ * MLA in MQA mode -- "DeepSeek-V3.2 论文解读", section 二, subsections "工作原理" and "挂在 MLA
+ * 上"; prefill and decode as in its subsection "等性能验证").
  *   DSA_MODE_PREFILL: indexer and top-k run fused (no score matrix is written to HBM), then
  *     sparse MLA.  keys/latent contiguous with the same cu_seqlens; q_fp8 [T, H_I, d_I], etc.
  *   DSA_MODE_DECODE: paged indexer scores for each sequence's context, top-k, then split
@@ -223,9 +236,10 @@ dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale,
                        int32_t H_I, int32_t d_I, int32_t H, int32_t k, float sm_scale, void* out,
                        float* lse, int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream);
 
-/* Bytes of workspace dsa_forward / dsa_sparse_mla_decode need (0 when none). */
-size_t dsa_workspace_size(int32_t mode, int32_t B, int64_t total_tokens, int32_t max_ctx, int32_t H,
-                          int32_t H_I, int32_t k);
+/* Bytes of workspace dsa_forward / dsa_sparse_mla_decode need (0 when none): prefill, the
+ * selection [total_tokens, k] int32; decode, the split partials of B sequences with H heads,
+ * one score row of max_ctx entries per sequence and the selection [B, k]. */
+size_t dsa_workspace_size(int32_t mode, int32_t B, int64_t total_tokens, int32_t max_ctx, int32_t H, int32_t k);
 
 /* Static description of a status code. */
 const char* dsa_status_string(int32_t status);

@@ -94,7 +94,7 @@ _lib.dsa_masked_mla_prefill.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _
 _lib.dsa_masked_mla_prefill.restype = _I32
 _lib.dsa_quantize_fp8.argtypes = [_P, _I64, _I32, _P, _P, _P]
 _lib.dsa_quantize_fp8.restype = _I32
-_lib.dsa_workspace_size.argtypes = [_I32, _I32, _I64, _I32, _I32, _I32, _I32]
+_lib.dsa_workspace_size.argtypes = [_I32, _I32, _I64, _I32, _I32, _I32]
 _lib.dsa_workspace_size.restype = _SZ
 
 
@@ -257,8 +257,8 @@ def dsa_forward(mode, q_fp8, q_scale, w, keys: Desc, q, latent: Desc, B, H_I, d_
     return out
 
 
-def dsa_workspace_size(mode, B, total_tokens, max_ctx, H, H_I, k) -> int:
-    return int(_lib.dsa_workspace_size(int(mode), int(B), int(total_tokens), int(max_ctx), int(H), int(H_I), int(k)))
+def dsa_workspace_size(mode, B, total_tokens, max_ctx, H, k) -> int:
+    return int(_lib.dsa_workspace_size(int(mode), int(B), int(total_tokens), int(max_ctx), int(H), int(k)))
 
 
 def dsa_device_error(stream=None) -> int:

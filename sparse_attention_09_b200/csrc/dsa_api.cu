@@ -572,7 +572,7 @@ dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale,
                        int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream) {
   if (keys == nullptr || latent == nullptr || B <= 0) return DSA_ERR_INVALID_ARGUMENT;
   if (!mla_shape_ok(H, k)) return DSA_ERR_UNSUPPORTED;
-  const size_t need = dsa_workspace_size(mode, B, keys->total_tokens, keys->max_seqlen, H, H_I, k);
+  const size_t need = dsa_workspace_size(mode, B, keys->total_tokens, keys->max_seqlen, H, k);
   if (mode == DSA_MODE_PREFILL) {
     if (keys->kind != DSA_KV_CONTIGUOUS || latent->kind != DSA_KV_CONTIGUOUS) return DSA_ERR_INVALID_ARGUMENT;
     int32_t* idx = idx_out;
@@ -605,9 +605,7 @@ dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale,
   return dsa_sparse_mla_decode(q, latent, idx, B, H, k, sm_scale, out, lse, workspace, part, stream);
 }
 
-size_t dsa_workspace_size(int32_t mode, int32_t B, int64_t total_tokens, int32_t max_ctx, int32_t H, int32_t H_I,
-                          int32_t k) {
-  (void)H_I;
+size_t dsa_workspace_size(int32_t mode, int32_t B, int64_t total_tokens, int32_t max_ctx, int32_t H, int32_t k) {
   if (B <= 0 || k <= 0 || H <= 0) return 0;
   if (mode == DSA_MODE_PREFILL) return align256(static_cast<size_t>(total_tokens > 0 ? total_tokens : 0) * k * 4);
   const int64_t ld = (static_cast<int64_t>(max_ctx > 0 ? max_ctx : 0) + 3) / 4 * 4;

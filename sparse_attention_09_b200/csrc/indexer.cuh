@@ -226,7 +226,10 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int lb = (tile0 + it) * 2 + h;
-            const int phys = bt[lb < nblocks_seq ? lb : 0];
+            int phys = bt[lb < nblocks_seq ? lb : 0];
+            // a block id outside the key pool never reaches the TMA unit: block 0 is loaded in
+            // its place and the epilogue scores the block's keys -inf (and reports them)
+            if (phys < 0 || phys >= p.num_blocks) phys = 0;
             tma_load_2d(dst + h * 64 * D_I, &k_map, &bar_kfull[stage], 0, phys * 64);
           }
         }
@@ -295,12 +298,17 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
       const uint32_t aph = (it >> 1) & 1;
       const int s = (tile0 + it) * 128 + e;  // local key position
       float ksc = 0.f;                       // k_scale of this lane's key (0 beyond the sequence)
+      bool bad_blk = false;                  // paged: the key's block id lies outside the pool
       if (s < len) {
         if constexpr (!PAGED) ksc = p.k_scale[seq_start + s];
         else {
           const int blk = bt[s >> 6];
-          if (blk >= 0 && blk < p.num_blocks) ksc = p.k_scale[static_cast<int64_t>(blk) * 64 + (s & 63)];
-          else record_device_error(DSA_ERR_DEVICE_CHECK);  // a block id outside the key pool
+          if (blk >= 0 && blk < p.num_blocks) {
+            ksc = p.k_scale[static_cast<int64_t>(blk) * 64 + (s & 63)];
+          } else {
+            bad_blk = true;
+            record_device_error(DSA_ERR_DEVICE_CHECK);
+          }
         }
       }
       const bool ok = mbar_wait(&bar_accfull[acc], aph);
@@ -398,7 +406,7 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
             if (gr >= p.row_begin && gr < p.row_end && s < len)
               p.scores[(gr - p.row_begin) * p.ld + s] = s <= t ? score : -INFINITY;
           } else {
-            if (s < len) p.scores[(b - p.row_begin) * p.ld + s] = score;
+            if (s < len) p.scores[(b - p.row_begin) * p.ld + s] = bad_blk ? -INFINITY : score;
           }
         }
       } else {

@@ -44,8 +44,8 @@ static int host_checks(void) {
   CHECK(dsa_topk(NULL, 8, 0, NULL, 4, NULL, NULL) == DSA_OK, "zero rows is not a no-op");
   CHECK(dsa_quantize_fp8(fake, 4, 12, (uint8_t*)fake, (float*)fake, NULL) == DSA_ERR_INVALID_ARGUMENT,
         "dsa_quantize_fp8 accepted cols not a multiple of 8");
-  CHECK(dsa_workspace_size(DSA_MODE_PREFILL, 0, 10, 10, 128, 64, 2048) == 0, "workspace for B = 0");
-  CHECK(dsa_workspace_size(DSA_MODE_PREFILL, 1, 1000, 1000, 128, 64, 2048) >= (size_t)1000 * 2048 * 4,
+  CHECK(dsa_workspace_size(DSA_MODE_PREFILL, 0, 10, 10, 128, 2048) == 0, "workspace for B = 0");
+  CHECK(dsa_workspace_size(DSA_MODE_PREFILL, 1, 1000, 1000, 128, 2048) >= (size_t)1000 * 2048 * 4,
         "prefill workspace smaller than the selection");
   return 0;
 }

@@ -27,7 +27,7 @@ def _decode(d, block_table, max_ctx):
     B = d["B"]
     keys = dsa.paged_desc(d["kcache8"], block_table, d["ctx"], max_ctx, scale=d["kscale_cache"])
     lat = dsa.paged_desc(d["latent_cache"], block_table, d["ctx"], max_ctx)
-    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, max_ctx, 128, 64, K), dtype=torch.uint8,
+    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, max_ctx, 128, K), dtype=torch.uint8,
                      device="cuda")
     out = torch.full((B, 128, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
     idx = torch.full((B, K), -7, dtype=torch.int32, device="cuda")
@@ -50,6 +50,12 @@ def test_block_ids_outside_the_pool_are_reported_and_masked():
     for b in (0, 3):                  # sequences with valid tables: exactly the clean results
         assert torch.equal(idx[b], clean_idx[b]) and torch.equal(out[b], clean_out[b]), f"seq {b}"
     assert torch.isfinite(out[1].float()).all() and torch.isfinite(out[2].float()).all()
+    # keys of a block outside the pool score -inf, so with more than K valid keys left in the
+    # context none of them is selected
+    sel1, sel2 = idx[1].cpu().numpy(), idx[2].cpu().numpy()
+    assert not ((sel1 >= 5 * 64) & (sel1 < 6 * 64)).any(), "a key of the bad block of sequence 1 was selected"
+    assert not ((sel2 >= 0) & (sel2 < 64)).any(), "a key of the bad block of sequence 2 was selected"
+    assert (sel1 >= 0).sum() == min(K, 3000) and (sel2 >= 0).sum() == min(K, 2500)
     assert dsa.dsa_device_error() == dsa.DSA_OK  # the read cleared the word
 
 

@@ -13,7 +13,7 @@ import torch
 
 import oracle
 import synth
-from helpers import assert_attention_close, indexer_scores, keys_desc, latent_desc, oracle_scores
+from helpers import assert_attention_close, assert_scores_close, indexer_scores, keys_desc, latent_desc, oracle_scores
 
 pytestmark = pytest.mark.gpu
 SM = 1.0 / math.sqrt(576)
@@ -39,7 +39,9 @@ def _check_prefill(inp, k, rows_per_seq, out, idx):
         # GPU scores of exactly these rows, then the oracle's selection of them
         I_gpu = [indexer_scores(inp, row_begin=g0 + t, row_end=g0 + t + 1)[0].cpu().numpy() for t in rows]
         I_ref, A_ref = oracle_scores(seq, rows)
+        L = int(cu[b + 1] - cu[b])
         for t, sg, ir, ar in zip(rows, I_gpu, I_ref, A_ref):
+            assert_scores_close(sg, ir, ar, t, L)   # the indexer's scores of this row, element by element
             got = idx[g0 + t].cpu().numpy()
             exp = oracle.topk_rows(sg[None, : t + 1], np.array([t + 1]), k)[0]
             assert np.array_equal(got, exp), f"seq {b} row {t}: selection != top-k of GPU scores"
@@ -92,7 +94,7 @@ def _decode(d, k):
     B = d["B"]
     keys = dsa.paged_desc(d["kcache8"], d["block_table"], d["ctx"], d["max_ctx"], scale=d["kscale_cache"])
     latent = dsa.paged_desc(d["latent_cache"], d["block_table"], d["ctx"], d["max_ctx"])
-    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, 64, k), dtype=torch.uint8,
+    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, k), dtype=torch.uint8,
                      device="cuda")
     out = torch.full((B, 128, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
     idx = torch.full((B, k), -7, dtype=torch.int32, device="cuda")

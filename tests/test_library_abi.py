@@ -109,9 +109,9 @@ def test_decode_split_rule_through_workspace_size():
 
     table = {1: 32, 2: 32, 3: 16, 5: 8, 9: 8, 10: 4, 18: 4, 19: 2, 37: 2, 38: 1, 64: 1, 200: 1}
     for B, s in table.items():
-        assert dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, 0, 128, 64, 2048) == expected(B, 128, 2048, s), B
+        assert dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, 0, 128, 2048) == expected(B, 128, 2048, s), B
     # k / 64 caps the count: two 64-row chunks allow two splits
-    assert dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, 1, 0, 0, 128, 64, 128) == expected(1, 128, 128, 2)
+    assert dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, 1, 0, 0, 128, 128) == expected(1, 128, 128, 2)
 
 
 def test_decode_split_count_partitions_every_selection():
@@ -127,7 +127,7 @@ def test_decode_split_count_partitions_every_selection():
 
     for k in range(64, 2049, 64):
         for B in range(1, 257):
-            ws = dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, 0, 128, 64, k)
+            ws = dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, 0, 128, k)
             base = a256(B * k * 4)
             s = next(s for s in (1, 2, 4, 8, 16, 32)
                      if a256(B * s * 128 * 512 * 4) + a256(B * s * 128 * 2 * 4) + base == ws)

@@ -101,7 +101,7 @@ def test_decode_paged_matches_oracle(B):
         sel = torch.sort(torch.randperm(c, generator=g, device="cuda")[:m]).values
         idx[b, :m] = sel.to(torch.int32)
     latent = dsa.paged_desc(d["latent_cache"], d["block_table"], d["ctx"], d["max_ctx"])
-    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, 64, k), dtype=torch.uint8,
+    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, k), dtype=torch.uint8,
                      device="cuda")
     out = torch.full((B, 128, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
     lse = torch.full((B, 128), float("nan"), device="cuda")

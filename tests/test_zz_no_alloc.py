@@ -31,7 +31,7 @@ def test_noalloc_decode_matches_workspace_decode_twice():
     d, idx, B, k = _inputs()
     sm = 1.0 / math.sqrt(576)
     latent = dsa.paged_desc(d["latent_cache"], d["block_table"], d["ctx"], d["max_ctx"])
-    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, 64, k), dtype=torch.uint8,
+    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, k), dtype=torch.uint8,
                      device="cuda")
     ref = torch.empty((B, 128, 512), dtype=torch.bfloat16, device="cuda")
     ref_lse = torch.empty((B, 128), device="cuda")
@@ -60,3 +60,38 @@ def test_noalloc_decode_rejects_sizes_beyond_its_scratch():
         ctypes.c_float(0.04), ctypes.c_void_p(d["q"].data_ptr()), None,
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == dsa.DSA_ERR_UNSUPPORTED
+
+
+def test_noalloc_decode_size_edge_at_128_heads():
+    """At H = 128 the partials of B = 127 sequences (one split each) fit the scratch array and
+    B = 128 do not: the last size that fits runs and equals the workspace call, the first that
+    does not is refused before any launch."""
+    import sparse_attention_09_b200 as dsa
+    B, k = 127, 2048
+    d = synth.decode_inputs(B=B, ctx_lo=1, ctx_hi=2500, H_I=64, d_I=128, H=128, seed=31, device="cuda")
+    idx = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(8)
+    for b, c in enumerate(d["ctx_host"]):
+        m = min(k, c)
+        idx[b, :m] = torch.sort(torch.randperm(c, generator=g, device="cuda")[:m]).values.to(torch.int32)
+    sm = 1.0 / math.sqrt(576)
+    latent = dsa.paged_desc(d["latent_cache"], d["block_table"], d["ctx"], d["max_ctx"])
+    ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, k), dtype=torch.uint8,
+                     device="cuda")
+    ref = torch.empty((B, 128, 512), dtype=torch.bfloat16, device="cuda")
+    dsa.dsa_sparse_mla_decode(d["q"], latent, idx, B, 128, k, sm, ref, None, ws)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    out = torch.full((B, 128, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
+    st = dsa._lib.dsa_sparse_mla_decode_noalloc(ctypes.c_void_p(d["q"].data_ptr()), latent.ref(),
+                                                ctypes.c_void_p(idx.data_ptr()), B, 128, k, ctypes.c_float(sm),
+                                                ctypes.c_void_p(out.data_ptr()), None, stream)
+    assert st == dsa.DSA_OK, dsa.dsa_status_string(st)
+    assert dsa.dsa_device_error() == 0
+    assert torch.equal(out, ref)  # the same kernels on the same inputs
+    poison = out.clone()
+    st = dsa._lib.dsa_sparse_mla_decode_noalloc(ctypes.c_void_p(d["q"].data_ptr()), latent.ref(),
+                                                ctypes.c_void_p(idx.data_ptr()), B + 1, 128, k, ctypes.c_float(sm),
+                                                ctypes.c_void_p(out.data_ptr()), None, stream)
+    assert st == dsa.DSA_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert torch.equal(out, poison)  # nothing was launched
