@@ -39,7 +39,7 @@ DECODE = "decode_64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {
     "indexer_topk": ["indexer.cuh", "select.cuh", "sm100.cuh", "common.cuh"],
-    "sparse_mla": ["sparse_mla.cuh", "sm100.cuh", "common.cuh"],
+    "sparse_mla": ["sparse_mla_pair.cuh", "sparse_mla.cuh", "sm100.cuh", "common.cuh"],
 }
 
 
@@ -200,58 +200,28 @@ def prefill_work(cfg):
 # ------------------------------------------------------------------------------------------
 # strong scaling: one sequence sharded by query rows (NEXT row f4)
 # ------------------------------------------------------------------------------------------
-def balanced_row_blocks(L, k, world, w_index=137.0, w_mla=145.0):
-    """Boundaries b[0] = 0 < ... < b[world] = L of query-row blocks of equal estimated cost.
-    A row t costs w_index * (t + 1) / sum(t + 1) (the indexer scans its causal prefix) plus
-    w_mla * min(t + 1, k) / sum(min(t + 1, k)) (sparse MLA over its selection); the weights
-    are the two kernels' measured shares of one step."""
-    t = np.arange(L, dtype=np.float64) + 1.0
-    ci = t / t.sum()
-    cm = np.minimum(t, k)
-    cm /= cm.sum()
-    cum = np.cumsum(w_index * ci + w_mla * cm)
-    targets = cum[-1] * np.arange(1, world) / world
-    inner = np.searchsorted(cum, targets, side="left") + 1
-    b = [0] + [int(x) for x in inner] + [L]
-    for i in range(1, len(b)):  # keep the blocks non-empty and ordered
-        b[i] = max(b[i], min(L, b[i - 1] + 1)) if i < len(b) - 1 else L
-    return b
-
-
-def even_row_blocks(L, world):
-    """Equal row blocks (how the key / latent rows are spread before the all-gather)."""
-    return [L * r // world for r in range(world + 1)]
-
-
-def gather_rows(local, full, world):
-    """All-gather of equal row blocks of `full` (block r comes from rank r) into `full`."""
-    if world == 1:
-        full.copy_(local)
-        return full
-    import torch.distributed as dist
-    if dist.get_backend() == "nccl":
-        dist.all_gather_into_tensor(full, local.contiguous())
-    else:
-        parts = list(full.chunk(world, 0))
-        dist.all_gather(parts, local.contiguous())
-        full.copy_(torch.cat(parts, 0))
-    return full
-
-
 def run_strong(args, world, rank, local):
-    """One L=131072 prefill sharded over the ranks by query-row blocks: every step all-gathers
-    the key (k_I, k_scale) and latent rows each rank holds, then runs the fused indexer top-k
-    and sparse MLA on the rank's own rows.  value = L tokens per (slowest rank's) step."""
+    """One L=131072 prefill sharded over the ranks by query-row blocks (the library's sharding
+    helpers): the key (k_I, k_scale) and latent rows each rank holds are all-gathered once for
+    the sequence, then every step runs the fused indexer top-k and sparse MLA on the rank's own
+    rows.  The blocks are balanced with the two kernels' measured whole-sequence times
+    (--idx-ms, --mla-ms).  value = L tokens per (slowest rank's) step."""
     import sparse_attention_09_b200 as dsa
+    from sparse_attention_09_b200 import sharding
     cfg = dict(synth.WORKLOADS[args.workload])
     k, sm, H, H_I, d_I = cfg["k"], 1.0 / math.sqrt(576), cfg["H"], cfg["H_I"], cfg["d_I"]
     inp = synth.prefill_inputs(device="cuda", **cfg)  # same seed on every rank: rank r keeps its blocks
     L = inp["q"].shape[0]
-    rb = balanced_row_blocks(L, k, world)
+    rb = sharding.row_blocks(L, k, world, args.idx_ms, args.mla_ms)
     q0, q1 = rb[rank], rb[rank + 1]
-    kb = even_row_blocks(L, world)
+    kb = sharding.even_blocks(L, world)
     k0, k1 = kb[rank], kb[rank + 1]
     my_k8, my_ks, my_lat = inp["k8"][k0:k1].clone(), inp["k_scale"][k0:k1].clone(), inp["latent"][k0:k1].clone()
+    for t in (inp["k8"], inp["k_scale"], inp["latent"]):  # only the gathered rows may reach the kernels
+        t.zero_()
+    sharding.gather_sequence(my_k8, inp["k8"], world, rank)
+    sharding.gather_sequence(my_ks, inp["k_scale"], world, rank)
+    sharding.gather_sequence(my_lat, inp["latent"], world, rank)
     keys = dsa.contiguous_desc(inp["k8"], inp["cu_seqlens"], L, scale=inp["k_scale"])
     lat = dsa.contiguous_desc(inp["latent"], inp["cu_seqlens"], L)
     R = q1 - q0
@@ -260,9 +230,6 @@ def run_strong(args, world, rank, local):
     qb = (inp["q8"][q0:q1], inp["q_scale"][q0:q1], inp["w"][q0:q1], inp["q"][q0:q1])
 
     def step():
-        gather_rows(my_k8, inp["k8"], world)
-        gather_rows(my_ks, inp["k_scale"], world)
-        gather_rows(my_lat, inp["latent"], world)
         dsa.dsa_indexer_topk_rows(qb[0], qb[1], qb[2], keys, H_I, d_I, k, q0, q1, idx)
         dsa.dsa_sparse_mla_prefill_rows(qb[3], lat, idx, H, k, sm, q0, q1, out)
 
@@ -288,7 +255,7 @@ def run_strong(args, world, rank, local):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
                 "scaling": "strong", "vs_baseline": None, "dtype": "e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
                 "config": {"workload": f"{args.workload}: one sequence sharded by query-row blocks {rb}, "
-                                       "keys and latent all-gathered every step",
+                                       "keys and latent all-gathered once per sequence",
                            "global_batch": 1, "seq_len": L, "k": k, "parallelism": f"row-sharded x{world}",
                            "l2": "inputs larger than L2; no flush"},
                 "clocks": clk, "gpu_launches": 2 * args.steps}
@@ -385,7 +352,8 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = synth.sample_rows(L, k, args.cpu_rows, seed=3)
         secs = oracle_prefill_sample(inp, k, rows, sm)
-        cpu = {"value": len(rows) / secs, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+        cpu = {"value": len(rows) / secs, "unit": "tokens/s", "cores": blas_threads(), "host_cores": os.cpu_count(),
+               "kind": "oracle",
                "sample": f"{len(rows)} query rows of the L=131072 prefill (full causal prefix each: indexer, "
                          f"top-k, attention), {secs:.1f} s"}
 
@@ -405,6 +373,67 @@ def run_ours(args, world, rank, local):
             "clocks": clk, "gpu_launches": 2 * args.steps,
         }
         print(json.dumps(line), flush=True)
+
+
+def run_profile_case(args, dsa, sm):
+    """Small cases of the bench's kernels for counter captures (the full-size step holds ~40 GB on
+    the device and runs 0.1-s kernels, too much for a capture).  Every kernel is launched twice,
+    a warm-up and the launch to capture (ncu -s 1 -c 1 with -k naming the kernel).
+      rows_128k      the last 2048 query rows of the L=131072 prefill (keys, k_scale and latent of
+                     the whole sequence, queries of the block only): dsa_indexer_topk_rows, then
+                     dsa_sparse_mla_prefill_rows.  Both kernels' DRAM bytes per query row scale to
+                     the full launch (per row: its queries, selection and output, and the latent
+                     rows gathered for its 2048 selected entries, as for every row of the run).
+      decode_8x128k  8 sequences at contexts drawn from [122880, 131072]: paged indexer scores,
+                     top-k, sparse MLA decode and the combine."""
+    cfg = dict(synth.WORKLOADS[PREFILL])
+    k = cfg["k"]
+    out = {"profile_case": args.profile_case}
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    if args.profile_case == "rows_128k":
+        L, R = cfg["seqlens"][0], 2048
+        blk = synth.prefill_block_inputs(L, L - R, L, cfg["H_I"], cfg["d_I"], cfg["H"], seed=cfg["seed"],
+                                         device="cuda", w_dist=cfg.get("w_dist", "normal8"),
+                                         planted=cfg.get("planted", 0.0))
+        keys = dsa.contiguous_desc(blk["k8"], blk["cu_seqlens"], L, scale=blk["k_scale"])
+        lat = dsa.contiguous_desc(blk["latent"], blk["cu_seqlens"], L)
+        idx = torch.empty((R, k), dtype=torch.int32, device="cuda")
+        o = torch.empty((R, cfg["H"], 512), dtype=torch.bfloat16, device="cuda")
+        for i in range(2):
+            evs[0].record()
+            dsa.dsa_indexer_topk_rows(blk["q8"], blk["q_scale"], blk["w"], keys, cfg["H_I"], cfg["d_I"], k, L - R, L, idx)
+            evs[1].record()
+            dsa.dsa_sparse_mla_prefill_rows(blk["q"], lat, idx, cfg["H"], k, sm, L - R, L, o, None)
+            evs[2].record()
+        torch.cuda.synchronize()
+        out.update(rows=R, L=L, indexer_topk_ms=evs[0].elapsed_time(evs[1]),
+                   sparse_mla_ms=evs[1].elapsed_time(evs[2]))
+    elif args.profile_case == "decode_8x128k":
+        B = 8
+        d = synth.decode_inputs(B=B, ctx_lo=122880, ctx_hi=131072, H_I=64, d_I=128, H=128, seed=31, device="cuda")
+        keys = dsa.paged_desc(d["kcache8"], d["block_table"], d["ctx"], d["max_ctx"], scale=d["kscale_cache"])
+        lat = dsa.paged_desc(d["latent_cache"], d["block_table"], d["ctx"], d["max_ctx"])
+        ld = (d["max_ctx"] + 3) // 4 * 4
+        scores = torch.empty((B, ld), device="cuda")
+        idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+        o = torch.empty((B, 128, 512), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, k), dtype=torch.uint8,
+                         device="cuda")
+        for i in range(2):
+            evs[0].record()
+            dsa.dsa_indexer_scores(d["q8"], d["q_scale"], d["w"], keys, B, 64, 128, 0, B, scores)
+            evs[1].record()
+            dsa.dsa_topk(scores, d["ctx"], k, idx)
+            evs[2].record()
+            dsa.dsa_sparse_mla_decode(d["q"], lat, idx, B, 128, k, sm, o, None, ws)
+            evs[3].record()
+        torch.cuda.synchronize()
+        out.update(B=B, ctx=[int(c) for c in d["ctx_host"]], indexer_ms=evs[0].elapsed_time(evs[1]),
+                   topk_ms=evs[1].elapsed_time(evs[2]), sparse_mla_decode_ms=evs[2].elapsed_time(evs[3]))
+    else:
+        raise SystemExit(f"unknown profile case {args.profile_case}")
+    assert dsa.dsa_device_error() == 0
+    print(json.dumps(out), flush=True)
 
 
 def run_quantizer(dsa, peaks):
@@ -576,11 +605,29 @@ def run_decode(args, dsa, sm, peaks):
     }
     for kk in kernels.values():
         kk["frac_of_hbm"] = kk["gbs"] / hbm
-    return {"workload": f"{DECODE}: 64 sequences, ctx ~ U[8192,131072] (sum {keys_scanned}), paged 64-token blocks",
-            "value": B / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": n,
-            "kernels": kernels, "peaks": {"hbm_gbs": hbm, "bf16_tflops": peaks["bf16_tflops"],
-                                          "note": "measured; burst bf16 (kernels timed alone)"},
-            "gpu_launches_per_step": 4}
+    res = {"workload": f"{DECODE}: 64 sequences, ctx ~ U[8192,131072] (sum {keys_scanned}), paged 64-token blocks",
+           "value": B / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": n,
+           "kernels": kernels, "peaks": {"hbm_gbs": hbm, "bf16_tflops": peaks["bf16_tflops"],
+                                         "note": "measured; burst bf16 (kernels timed alone)"},
+           "gpu_launches_per_step": 4}
+    if not args.no_cpu_baseline:
+        res["cpu_baseline"] = oracle_decode_sample(d, k, sm, args.cpu_decode_seqs)
+    return res
+
+
+def oracle_decode_sample(d, k, sm, nseq):
+    """The oracle's decode step (paged indexer over the whole context, top-k, sparse MLA) on the
+    first nseq sequences of the decode workload, timed on the host; tokens/s = nseq / time."""
+    import oracle
+    seqs = [synth.decode_seq_numpy(d, b) for b in range(nseq)]
+    t0 = time.perf_counter()
+    for s in seqs:
+        oracle.dsa_decode(s, k, sm)
+    secs = time.perf_counter() - t0
+    ctx = [int(d["ctx_host"][b]) for b in range(nseq)]
+    return {"value": nseq / secs, "unit": "tokens/s", "cores": blas_threads(), "host_cores": os.cpu_count(),
+            "kind": "oracle",
+            "sample": f"{nseq} of the 64 decode sequences (contexts {ctx}), one decode token each, {secs:.1f} s"}
 
 
 def run_e2e(args, dsa, inp, cfg, sm, n_blocks=32):
@@ -717,7 +764,7 @@ def run_reference(args, world, rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{PREFILL}: DSA prefill, L=131072, top-k 2048 (oracle on {per_step} sampled "
                                    "query rows per step)", "seq_len": L, "k": k},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "host_cores": os.cpu_count(), "kind": "oracle",
                              "sample": f"{per_step} random query rows per step of the L=131072 prefill"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -733,10 +780,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--cpu-decode-seqs", type=int, default=4)
     ap.add_argument("--ref-rows", type=int, default=2)
     ap.add_argument("--workload", default=PREFILL, choices=[w for w, c in synth.WORKLOADS.items() if c["kind"] == "prefill"],
                     help="prefill workload of the timed step (the headline is prefill_128k; smaller ones are for profiling)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--profile-case", choices=["rows_128k", "decode_8x128k"], default=None,
+                    help="run one small case of the kernels for a counter capture and exit")
+    ap.add_argument("--idx-ms", type=float, default=142.0,
+                    help="--strong: measured time of the fused indexer top-k over the whole sequence")
+    ap.add_argument("--mla-ms", type=float, default=93.0,
+                    help="--strong: measured time of sparse MLA over the whole sequence")
     ap.add_argument("--strong", action="store_true",
                     help="shard ONE sequence over the ranks by query rows (strong scaling) instead of one problem per rank")
     args = ap.parse_args()
@@ -747,6 +801,10 @@ def main():
         run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
         return
     world, rank, local = dist_setup(args)
+    if args.profile_case is not None:
+        import sparse_attention_09_b200 as dsa
+        run_profile_case(args, dsa, 1.0 / math.sqrt(576))
+        return
     if args.strong:
         run_strong(args, world, rank, local)
     else:

@@ -149,6 +149,20 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, int64_t rows, const 
  * Each block's results equal the corresponding rows of the whole-sequence call.  row_begin ==
  * row_end is a no-op; 0 <= row_begin <= row_end <= L, else DSA_ERR_INVALID_ARGUMENT.
  */
+/*
+ * Row blocks of balanced cost for sharding one prefill of length L over `parts` GPUs (host
+ * only, no device work): bounds[0] = 0 < bounds[1] < ... < bounds[parts] = L, every block
+ * non-empty.  Query row t costs indexer_cost * (t+1) / sum_t (t+1) -- the indexer scans its
+ * causal prefix -- plus mla_cost * min(t+1, k) / sum_t min(t+1, k) -- sparse MLA over its
+ * selection; pass the two kernels' measured times of one whole-sequence step (any unit, both
+ * >= 0, not both 0).  Block r ends at the first row where the cumulative cost reaches r/parts
+ * of the total.  The pages describe no parallelism; this is a scale-out helper for the row-block
+ * entry points below.  DSA_ERR_INVALID_ARGUMENT for bounds == NULL, L < 1, k < 1,
+ * parts outside [1, L] or costs as above.
+ */
+dsa_status dsa_row_partition(int64_t L, int32_t k, int32_t parts, double indexer_cost, double mla_cost,
+                             int64_t* bounds);
+
 dsa_status dsa_indexer_topk_rows(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
                                  const dsa_kv_desc* keys, int32_t H_I, int32_t d_I, int32_t k,
                                  int64_t row_begin, int64_t row_end, int32_t* idx_out, void* stream);

@@ -35,7 +35,7 @@ EXPORTED = ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_ml
             "dsa_forward", "dsa_workspace_size", "dsa_status_string", "dsa_device_error",
             "dsa_sparse_mla_decode_noalloc", "dsa_quantize_fp8", "dsa_masked_mla_prefill",
             "dsa_indexer_topk_rows", "dsa_sparse_mla_prefill_rows", "dsa_attn_distribution", "dsa_indexer_kl",
-            "dsa_selftest_wait_timeout")
+            "dsa_selftest_wait_timeout", "dsa_row_partition")
 
 
 class KVDesc(ctypes.Structure):
@@ -89,6 +89,8 @@ _lib.dsa_selftest_wait_timeout.restype = _I32
 _lib.dsa_indexer_topk_rows.argtypes = [_P, _P, _I32, _P, _DESC, _I32, _I32, _I32, _I64, _I64, _P, _P]
 _lib.dsa_indexer_topk_rows.restype = _I32
 _lib.dsa_sparse_mla_prefill_rows.argtypes = [_P, _DESC, _P, _I32, _I32, _F32, _I64, _I64, _P, _P, _P]
+_lib.dsa_row_partition.argtypes = [_I64, _I32, _I32, ctypes.c_double, ctypes.c_double, ctypes.POINTER(_I64)]
+_lib.dsa_row_partition.restype = _I32
 _lib.dsa_sparse_mla_prefill_rows.restype = _I32
 _lib.dsa_masked_mla_prefill.argtypes = [_P, _DESC, _P, _I32, _I32, _I32, _F32, _P, _P, _P]
 _lib.dsa_masked_mla_prefill.restype = _I32
@@ -282,3 +284,12 @@ def dsa_sparse_mla_decode_noalloc(q, latent: Desc, idx, B, H, k, sm_scale, out, 
                                               float(sm_scale), _ptr(out), _ptr(lse), _stream(stream)),
            "dsa_sparse_mla_decode_noalloc")
     return out
+
+
+def dsa_row_partition(L, k, parts, indexer_cost, mla_cost):
+    """Row-block boundaries [0, ..., L] of balanced estimated cost for sharding one prefill of
+    length L over `parts` GPUs (host only; see dsa_row_partition in include/dsa.h)."""
+    out = (_I64 * (int(parts) + 1))()
+    _check(_lib.dsa_row_partition(int(L), int(k), int(parts), float(indexer_cost), float(mla_cost), out),
+           "dsa_row_partition")
+    return [int(x) for x in out]

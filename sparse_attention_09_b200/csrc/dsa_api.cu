@@ -605,6 +605,38 @@ dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale,
   return dsa_sparse_mla_decode(q, latent, idx, B, H, k, sm_scale, out, lse, workspace, part, stream);
 }
 
+dsa_status dsa_row_partition(int64_t L, int32_t k, int32_t parts, double indexer_cost, double mla_cost,
+                             int64_t* bounds) {
+  if (bounds == nullptr || L < 1 || k < 1 || parts < 1 || parts > L) return DSA_ERR_INVALID_ARGUMENT;
+  if (!(indexer_cost >= 0.0) || !(mla_cost >= 0.0) || !(indexer_cost + mla_cost > 0.0)) return DSA_ERR_INVALID_ARGUMENT;
+  // cost of rows [0, n): indexer_cost * C(n) / C(L) + mla_cost * M(n) / M(L), with
+  // C(n) = sum_{t<n} (t+1) (the causal prefixes the indexer scans) and
+  // M(n) = sum_{t<n} min(t+1, k) (the rows sparse MLA attends to)
+  const double kk = static_cast<double>(k);
+  auto C = [](double n) { return n * (n + 1.0) / 2.0; };
+  auto M = [&](double n) { return n <= kk ? n * (n + 1.0) / 2.0 : kk * (kk + 1.0) / 2.0 + (n - kk) * kk; };
+  const double Lf = static_cast<double>(L), CL = C(Lf), ML = M(Lf);
+  auto cost = [&](int64_t n) {
+    const double x = static_cast<double>(n);
+    return indexer_cost * C(x) / CL + mla_cost * M(x) / ML;
+  };
+  const double total = cost(L);
+  bounds[0] = 0;
+  for (int32_t r = 1; r < parts; ++r) {
+    const double target = total * static_cast<double>(r) / static_cast<double>(parts);
+    int64_t lo = bounds[r - 1] + 1, hi = L - (parts - r);  // every block keeps at least one row
+    if (lo > hi) return DSA_ERR_INVALID_ARGUMENT;
+    while (lo < hi) {  // the first boundary whose cost reaches the target
+      const int64_t mid = lo + (hi - lo) / 2;
+      if (cost(mid) >= target) hi = mid;
+      else lo = mid + 1;
+    }
+    bounds[r] = lo;
+  }
+  bounds[parts] = L;
+  return DSA_OK;
+}
+
 size_t dsa_workspace_size(int32_t mode, int32_t B, int64_t total_tokens, int32_t max_ctx, int32_t H, int32_t k) {
   if (B <= 0 || k <= 0 || H <= 0) return 0;
   if (mode == DSA_MODE_PREFILL) return align256(static_cast<size_t>(total_tokens > 0 ? total_tokens : 0) * k * 4);

@@ -9,6 +9,7 @@ from .inputs import (  # noqa: F401
     WORKLOADS,
     quantize_e4m3_per_token,
     prefill_inputs,
+    prefill_block_inputs,
     decode_inputs,
     exact_prefill_inputs,
     tie_heavy_scores,

@@ -81,24 +81,42 @@ def test_job_value_single_rank():
     json.dumps({"v": bench.job_value(1, 1, 1.0)})
 
 
-def test_balanced_row_blocks_cover_and_balance():
+def test_row_partition_covers_and_balances():
+    """The library's row partition (dsa_row_partition through the binding, host only): blocks
+    cover [0, L), are non-empty and carry equal estimated cost to within one row's cost; the
+    cost model is the two kernels' measured times spread over the rows."""
     sys.path.insert(0, ROOT)
     import numpy as np
 
-    import bench
+    from sparse_attention_09_b200 import sharding
 
     L, k = 131072, 2048
     t = np.arange(L, dtype=np.float64) + 1
-    cost = 137.0 * t / t.sum() + 145.0 * np.minimum(t, k) / np.minimum(t, k).sum()
-    for world in (1, 2, 3, 4, 8):
-        b = bench.balanced_row_blocks(L, k, world)
-        assert b[0] == 0 and b[-1] == L and len(b) == world + 1
-        assert all(b[i] < b[i + 1] for i in range(world))
-        per = [cost[b[i]:b[i + 1]].sum() for i in range(world)]
-        assert max(per) - min(per) <= 1e-3 * sum(per)   # balanced to a row
-    tiny = bench.balanced_row_blocks(5, 2048, 8)   # more ranks than rows: some blocks empty
-    assert tiny[0] == 0 and tiny[-1] == 5 and all(tiny[i] <= tiny[i + 1] for i in range(8))
-    assert bench.even_row_blocks(10, 3) == [0, 3, 6, 10]
+    for idx_ms, mla_ms in ((142.0, 93.0), (137.0, 145.0), (1.0, 0.0), (0.0, 1.0)):
+        cost = idx_ms * t / t.sum() + mla_ms * np.minimum(t, k) / np.minimum(t, k).sum()
+        for world in (1, 2, 3, 4, 8):
+            b = sharding.row_blocks(L, k, world, idx_ms, mla_ms)
+            assert b[0] == 0 and b[-1] == L and len(b) == world + 1
+            assert all(b[i] < b[i + 1] for i in range(world))
+            per = [cost[b[i]:b[i + 1]].sum() for i in range(world)]
+            assert max(per) - min(per) <= 2 * cost.max() + 1e-9 * sum(per), (idx_ms, mla_ms, world, per)
+    # the indexer alone: the 2-way split sits at L / sqrt(2) (half of the causal pairs)
+    b = sharding.row_blocks(L, k, 2, 1.0, 0.0)
+    assert abs(b[1] - L / np.sqrt(2)) < 2
+    assert sharding.row_blocks(8, 2048, 8, 1.0, 1.0) == list(range(9))   # as many ranks as rows
+    assert sharding.even_blocks(10, 3) == [0, 3, 6, 10]
+
+
+def test_row_partition_rejects_bad_arguments():
+    sys.path.insert(0, ROOT)
+    import pytest
+
+    import sparse_attention_09_b200 as dsa
+
+    for args in ((0, 2048, 1, 1.0, 1.0), (5, 2048, 6, 1.0, 1.0), (10, 0, 2, 1.0, 1.0), (10, 64, 2, 0.0, 0.0),
+                 (10, 64, 2, -1.0, 2.0), (10, 64, 0, 1.0, 1.0)):
+        with pytest.raises(RuntimeError):
+            dsa.dsa_row_partition(*args)
 
 
 def _gather_main(rank, world, port, q):
@@ -106,24 +124,26 @@ def _gather_main(rank, world, port, q):
     import torch
     import torch.distributed as dist
 
-    import bench
+    from sparse_attention_09_b200 import sharding
 
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        L = 12
-        full_ref = torch.arange(L * 3, dtype=torch.float32).reshape(L, 3)
-        kb = bench.even_row_blocks(L, world)
-        local = full_ref[kb[rank]:kb[rank + 1]].clone()
-        full = torch.zeros_like(full_ref)
-        bench.gather_rows(local, full, world)
-        q.put((rank, bool(torch.equal(full, full_ref))))
+        ok = True
+        for L in (12, 13):   # even and uneven row blocks
+            full_ref = torch.arange(L * 3, dtype=torch.float32).reshape(L, 3)
+            kb = sharding.even_blocks(L, world)
+            local = full_ref[kb[rank]:kb[rank + 1]].clone()
+            full = torch.zeros_like(full_ref)
+            sharding.gather_sequence(local, full, world, rank)
+            ok = ok and bool(torch.equal(full, full_ref))
+        q.put((rank, ok))
     finally:
         dist.barrier()
         dist.destroy_process_group()
 
 
-def test_gather_rows_two_gloo_ranks():
+def test_gather_sequence_two_gloo_ranks():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
