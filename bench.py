@@ -385,7 +385,14 @@ def run_profile_case(args, dsa, sm):
                      the full launch (per row: its queries, selection and output, and the latent
                      rows gathered for its 2048 selected entries, as for every row of the run).
       decode_8x128k  8 sequences at contexts drawn from [122880, 131072]: paged indexer scores,
-                     top-k, sparse MLA decode and the combine."""
+                     top-k, sparse MLA decode and the combine.
+      indexer_128k   the whole fused indexer + top-k launch of the L=131072 prefill (the bench's
+                     own call and launch shape) with only the indexer's operands on the device
+                     (~2.3 GB): its per-launch DRAM bytes need no scaling.
+      mla_quarters_128k  dsa_sparse_mla_prefill_rows on four blocks of 2048 query rows of the
+                     L=131072 sequence, centred on the midpoints of its quarters (the whole latent
+                     on the device): midpoint-rule samples of the per-row DRAM bytes, whose
+                     sum x 16 estimates the full launch.  Each block is launched twice in turn."""
     cfg = dict(synth.WORKLOADS[PREFILL])
     k = cfg["k"]
     out = {"profile_case": args.profile_case}
@@ -430,6 +437,42 @@ def run_profile_case(args, dsa, sm):
         torch.cuda.synchronize()
         out.update(B=B, ctx=[int(c) for c in d["ctx_host"]], indexer_ms=evs[0].elapsed_time(evs[1]),
                    topk_ms=evs[1].elapsed_time(evs[2]), sparse_mla_decode_ms=evs[2].elapsed_time(evs[3]))
+    elif args.profile_case == "indexer_128k":
+        L = cfg["seqlens"][0]
+        blk = synth.prefill_block_inputs(L, 0, L, cfg["H_I"], cfg["d_I"], cfg["H"], seed=cfg["seed"], device="cuda",
+                                         w_dist=cfg.get("w_dist", "normal8"), planted=cfg.get("planted", 0.0),
+                                         mla=False)
+        keys = dsa.contiguous_desc(blk["k8"], blk["cu_seqlens"], L, scale=blk["k_scale"])
+        idx = torch.empty((L, k), dtype=torch.int32, device="cuda")
+        for i in range(2):
+            evs[0].record()
+            dsa.dsa_indexer_topk(blk["q8"], blk["q_scale"], blk["w"], keys, 1, cfg["H_I"], cfg["d_I"], k, idx)
+            evs[1].record()
+        torch.cuda.synchronize()
+        out.update(L=L, indexer_topk_ms=evs[0].elapsed_time(evs[1]))
+    elif args.profile_case == "mla_quarters_128k":
+        L, R = cfg["seqlens"][0], 2048
+        ms = []
+        for j in range(4):
+            mid = L // 8 + j * (L // 4)
+            r0, r1 = mid - R // 2, mid + R // 2
+            blk = synth.prefill_block_inputs(L, r0, r1, cfg["H_I"], cfg["d_I"], cfg["H"], seed=cfg["seed"] + j,
+                                             device="cuda", w_dist=cfg.get("w_dist", "normal8"),
+                                             planted=cfg.get("planted", 0.0))
+            keys = dsa.contiguous_desc(blk["k8"], blk["cu_seqlens"], L, scale=blk["k_scale"])
+            lat = dsa.contiguous_desc(blk["latent"], blk["cu_seqlens"], L)
+            idx = torch.empty((R, k), dtype=torch.int32, device="cuda")
+            o = torch.empty((R, cfg["H"], 512), dtype=torch.bfloat16, device="cuda")
+            dsa.dsa_indexer_topk_rows(blk["q8"], blk["q_scale"], blk["w"], keys, cfg["H_I"], cfg["d_I"], k, r0, r1, idx)
+            for i in range(2):
+                evs[1].record()
+                dsa.dsa_sparse_mla_prefill_rows(blk["q"], lat, idx, cfg["H"], k, sm, r0, r1, o, None)
+                evs[2].record()
+            torch.cuda.synchronize()
+            ms.append(evs[1].elapsed_time(evs[2]))
+            del blk, keys, lat, idx, o
+        out.update(rows=R, L=L, blocks=[[L // 8 + j * (L // 4) - R // 2, L // 8 + j * (L // 4) + R // 2]
+                                        for j in range(4)], sparse_mla_ms=ms)
     else:
         raise SystemExit(f"unknown profile case {args.profile_case}")
     assert dsa.dsa_device_error() == 0
@@ -785,7 +828,7 @@ def main():
     ap.add_argument("--workload", default=PREFILL, choices=[w for w, c in synth.WORKLOADS.items() if c["kind"] == "prefill"],
                     help="prefill workload of the timed step (the headline is prefill_128k; smaller ones are for profiling)")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--profile-case", choices=["rows_128k", "decode_8x128k"], default=None,
+    ap.add_argument("--profile-case", choices=["rows_128k", "decode_8x128k", "indexer_128k", "mla_quarters_128k"], default=None,
                     help="run one small case of the kernels for a counter capture and exit")
     ap.add_argument("--idx-ms", type=float, default=142.0,
                     help="--strong: measured time of the fused indexer top-k over the whole sequence")

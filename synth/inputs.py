@@ -132,19 +132,20 @@ def prefill_inputs(seqlens, H_I, d_I, H, *, seed, device, w_dist="normal8", idx_
 
 
 def prefill_block_inputs(L, row_begin, row_end, H_I, d_I, H, *, seed, device, w_dist="normal8", idx_std=1.0,
-                         planted=0.0, **_):
+                         planted=0.0, mla=True, **_):
     """Inputs for a block of query rows [row_begin, row_end) of ONE sequence of length L: the keys
     (k8, k_scale) and latent of the whole sequence, the query-side tensors (q8, q_scale, w, q) of
     the block only, with the distributions prefill_inputs draws (a small-footprint case of the
-    same workload for counter captures; the values are not those rows of prefill_inputs)."""
+    same workload for counter captures; the values are not those rows of prefill_inputs).
+    With mla=False the attention operands (q, latent) are left out (None): indexer-only cases."""
     R = int(row_end) - int(row_begin)
     cu = torch.tensor([0, int(L)], dtype=torch.int32, device=device)
     q8, q_scale = _indexer_operand((R, H_I, d_I), idx_std, False, _gen(device, seed, 11), device)
     k8, k_scale = _indexer_operand((int(L), d_I), idx_std, False, _gen(device, seed, 12), device,
                                    planted=planted, g_plant=_gen(device, seed, 17))
     w = _weights((R, H_I), w_dist, _gen(device, seed, 13), device)
-    q = _normal_bf16((R, H, D_QK), 1.0 / math.sqrt(D_QK), _gen(device, seed, 14), device)
-    latent = _normal_bf16((int(L), D_QK), 1.0 / math.sqrt(D_QK), _gen(device, seed, 15), device)
+    q = _normal_bf16((R, H, D_QK), 1.0 / math.sqrt(D_QK), _gen(device, seed, 14), device) if mla else None
+    latent = _normal_bf16((int(L), D_QK), 1.0 / math.sqrt(D_QK), _gen(device, seed, 15), device) if mla else None
     return dict(cu_seqlens=cu, seqlens=[int(L)], q8=q8, q_scale=q_scale, w=w, k8=k8, k_scale=k_scale, q=q,
                 latent=latent, H_I=H_I, d_I=d_I, H=H, row_begin=int(row_begin), row_end=int(row_end))
 
