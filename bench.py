@@ -384,8 +384,9 @@ def run_profile_case(args, dsa, sm):
                      dsa_sparse_mla_prefill_rows.  Both kernels' DRAM bytes per query row scale to
                      the full launch (per row: its queries, selection and output, and the latent
                      rows gathered for its 2048 selected entries, as for every row of the run).
-      decode_8x128k  8 sequences at contexts drawn from [122880, 131072]: paged indexer scores,
-                     top-k, sparse MLA decode and the combine.
+      decode_8x128k  8 sequences at contexts drawn from [122880, 131072]: the fused decode
+                     selection (paged indexer scan + selection kernel), sparse MLA decode and
+                     the combine.
       indexer_128k   the whole fused indexer + top-k launch of the L=131072 prefill (the bench's
                      own call and launch shape) with only the indexer's operands on the device
                      (~2.3 GB): its per-launch DRAM bytes need no scaling.
@@ -420,23 +421,20 @@ def run_profile_case(args, dsa, sm):
         d = synth.decode_inputs(B=B, ctx_lo=122880, ctx_hi=131072, H_I=64, d_I=128, H=128, seed=31, device="cuda")
         keys = dsa.paged_desc(d["kcache8"], d["block_table"], d["ctx"], d["max_ctx"], scale=d["kscale_cache"])
         lat = dsa.paged_desc(d["latent_cache"], d["block_table"], d["ctx"], d["max_ctx"])
-        ld = (d["max_ctx"] + 3) // 4 * 4
-        scores = torch.empty((B, ld), device="cuda")
         idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
         o = torch.empty((B, 128, 512), dtype=torch.bfloat16, device="cuda")
         ws = torch.empty(dsa.dsa_workspace_size(dsa.DSA_MODE_DECODE, B, 0, d["max_ctx"], 128, k), dtype=torch.uint8,
                          device="cuda")
+        ws_sel = torch.empty(dsa.dsa_decode_select_workspace_size(B, d["max_ctx"]), dtype=torch.uint8, device="cuda")
         for i in range(2):
             evs[0].record()
-            dsa.dsa_indexer_scores(d["q8"], d["q_scale"], d["w"], keys, B, 64, 128, 0, B, scores)
+            dsa.dsa_indexer_topk_decode(d["q8"], d["q_scale"], d["w"], keys, B, 64, 128, k, idx, ws_sel)
             evs[1].record()
-            dsa.dsa_topk(scores, d["ctx"], k, idx)
-            evs[2].record()
             dsa.dsa_sparse_mla_decode(d["q"], lat, idx, B, 128, k, sm, o, None, ws)
-            evs[3].record()
+            evs[2].record()
         torch.cuda.synchronize()
-        out.update(B=B, ctx=[int(c) for c in d["ctx_host"]], indexer_ms=evs[0].elapsed_time(evs[1]),
-                   topk_ms=evs[1].elapsed_time(evs[2]), sparse_mla_decode_ms=evs[2].elapsed_time(evs[3]))
+        out.update(B=B, ctx=[int(c) for c in d["ctx_host"]], indexer_topk_ms=evs[0].elapsed_time(evs[1]),
+                   sparse_mla_decode_ms=evs[1].elapsed_time(evs[2]))
     elif args.profile_case == "indexer_128k":
         L = cfg["seqlens"][0]
         blk = synth.prefill_block_inputs(L, 0, L, cfg["H_I"], cfg["d_I"], cfg["H"], seed=cfg["seed"], device="cuda",
@@ -610,10 +608,13 @@ def run_decode(args, dsa, sm, peaks):
     ms = e0.elapsed_time(e1) / n
     keys_scanned = int(sum(d["ctx_host"]))
 
-    # the same chain call by call, each kernel bracketed by events on the launching stream
+    # the same chain call by call, each call bracketed by events on the launching stream; the
+    # paged scan alone (dsa_indexer_scores) is timed beside the fused selection call, whose
+    # selection kernel takes the difference
     ld = (d["max_ctx"] + 3) // 4 * 4
     S = torch.empty((B, ld), device="cuda")
     idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    ws_sel = torch.empty(dsa.dsa_decode_select_workspace_size(B, d["max_ctx"]), dtype=torch.uint8, device="cuda")
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
     for i in range(-3, n):
         e = ev[i] if i >= 0 else None
@@ -622,7 +623,7 @@ def run_decode(args, dsa, sm, peaks):
         dsa.dsa_indexer_scores(d["q8"], d["q_scale"], d["w"], keys, B, 64, 128, 0, B, S)
         if e:
             e[1].record()
-        dsa.dsa_topk(S, d["ctx"], k, idx)
+        dsa.dsa_indexer_topk_decode(d["q8"], d["q_scale"], d["w"], keys, B, 64, 128, k, idx, ws_sel)
         if e:
             e[2].record()
         dsa.dsa_sparse_mla_decode(d["q"], lat, idx, B, 128, k, sm, out, None, ws)
@@ -632,16 +633,19 @@ def run_decode(args, dsa, sm, peaks):
     assert dsa.dsa_device_error() == 0
     t = [float(np.mean([e[j].elapsed_time(e[j + 1]) for e in ev])) for j in range(3)]
     hbm = peaks["hbm_gbs"]
-    # algorithmic bytes: the indexer reads 132 B per cached key (e4m3 key + fp32 scale) and each
-    # query's q_I, w and scale, and writes a 4-byte score per key; top-k reads the scores and
-    # writes the selection; sparse MLA gathers 1152 B per selected row and reads q, writes out
-    idx_bytes = keys_scanned * (132 + 4) + B * (64 * 128 + 64 * 4 + 4)
-    topk_bytes = keys_scanned * 4 + B * k * 4
+    # algorithmic bytes: the paged scan reads 132 B per cached key (e4m3 key + fp32 scale) and
+    # each query's q_I, w and scale, and writes a 4-byte score per key (and, in the fused call, a
+    # 4-byte maximum per 16 keys); the selection reads the scores and maxima once and writes the
+    # selection; sparse MLA gathers 1152 B per selected row and reads q, writes out
+    q_bytes = B * (64 * 128 + 64 * 4 + 4)
+    idx_bytes = keys_scanned * (132 + 4) + q_bytes
+    sel_bytes = keys_scanned * (132 + 4 + 0.25 + 4 + 0.25) + q_bytes + B * k * 4
     mla_bytes = B * k * 1152 + B * 128 * 576 * 2 + B * 128 * 512 * 2 + B * k * 4
     mla_flops = B * k * 278528
     kernels = {
         "indexer_scores": {"ms": t[0], "bytes": idx_bytes, "gbs": idx_bytes / (t[0] * 1e-3) / 1e9},
-        "topk": {"ms": t[1], "bytes": topk_bytes, "gbs": topk_bytes / (t[1] * 1e-3) / 1e9},
+        "indexer_topk_decode": {"ms": t[1], "bytes": sel_bytes, "gbs": sel_bytes / (t[1] * 1e-3) / 1e9,
+                                "selection_ms": t[1] - t[0]},
         "sparse_mla_decode": {"ms": t[2], "bytes": mla_bytes, "gbs": mla_bytes / (t[2] * 1e-3) / 1e9,
                               "tflops": mla_flops / (t[2] * 1e-3) / 1e12,
                               "frac_of_bf16": mla_flops / (t[2] * 1e-3) / 1e12 / peaks["bf16_tflops"]},
@@ -652,7 +656,7 @@ def run_decode(args, dsa, sm, peaks):
            "value": B / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": n,
            "kernels": kernels, "peaks": {"hbm_gbs": hbm, "bf16_tflops": peaks["bf16_tflops"],
                                          "note": "measured; burst bf16 (kernels timed alone)"},
-           "gpu_launches_per_step": 4}
+           "gpu_launches_per_step": 3 if B * 2 > 74 else 4}
     if not args.no_cpu_baseline:
         res["cpu_baseline"] = oracle_decode_sample(d, k, sm, args.cpu_decode_seqs)
     return res

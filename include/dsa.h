@@ -125,6 +125,30 @@ dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, int32_t 
                             void* stream);
 
 /*
+ * Fused decode selection (method steps 1 and 2 for one decode query per sequence): the paged
+ * lightning indexer over each sequence's context (as dsa_indexer_scores, decode form, rows
+ * 0..B-1), then the per-sequence top-k.  idx_out [B, k] receives, for sequence b, the indices
+ * of the min(k, ctx_b) highest-scoring context positions, ties to the lower position,
+ * ascending, -1 padded, with ctx_b = min(context_lens[b], keys->max_seqlen) -- the result
+ * dsa_topk gives on the scores dsa_indexer_scores writes.  While it scans, the indexer
+ * records the largest score of every 16 consecutive keys; the k-th largest of those maxima
+ * bounds the k-th largest score from below, so the selection reads each score row once and
+ * keeps only the scores at or above that bound (falling back to a full radix select of the
+ * row when they do not fit on chip).  keys must be paged (else DSA_ERR_UNSUPPORTED).
+ * workspace (device, 256-byte aligned, caller-owned, contents unspecified on return) holds
+ * the score rows and group maxima: ws_bytes >= dsa_decode_select_workspace_size(B,
+ * keys->max_seqlen), else DSA_ERR_WORKSPACE_TOO_SMALL.  A context longer than
+ * keys->max_seqlen and NaN scores set DSA_ERR_DEVICE_CHECK in the device error word.
+ */
+dsa_status dsa_indexer_topk_decode(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
+                                   const dsa_kv_desc* keys, int32_t B, int32_t H_I, int32_t d_I, int32_t k,
+                                   int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of dsa_indexer_topk_decode for B sequences of at most max_ctx keys (0 when
+ * B or max_ctx is not positive). */
+size_t dsa_decode_select_workspace_size(int32_t B, int32_t max_ctx);
+
+/*
  * Top-k selection (method step 2: the index scores pick the k = 2048 highest-scoring tokens
  * of each query -- "DeepSeek-V3.2 论文解读", section 二, subsection "工作原理" and table
  * "附：DSA 关键参数"; 36881.com.cn digest, "第二步：Fine-grained Token Selection") over score
@@ -205,7 +229,8 @@ dsa_status dsa_sparse_mla_prefill(const void* q, const dsa_kv_desc* latent, cons
  * (< ctx[b]) resolved through the paged latent cache (latent->kind == DSA_KV_PAGED).  The work
  * is split over the k selected rows (into more parts for fewer sequences, so that all the
  * parts run in one round on the GPU); partial results go to `workspace`
- * (dsa_workspace_size(DSA_MODE_DECODE, ...) bytes) and are merged by log-sum-exp.
+ * (dsa_workspace_size(DSA_MODE_DECODE, ...) bytes) and are merged by log-sum-exp.  When the
+ * sequences alone fill the GPU (one part each) the kernel writes out and lse directly.
  */
 dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const int32_t* idx,
                                  int32_t B, int32_t H, int32_t k, float sm_scale, void* out,
@@ -241,7 +266,7 @@ dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const dsa_kv_desc* laten
  * 上"; prefill and decode as in its subsection "等性能验证").
  *   DSA_MODE_PREFILL: indexer and top-k run fused (no score matrix is written to HBM), then
  *     sparse MLA.  keys/latent contiguous with the same cu_seqlens; q_fp8 [T, H_I, d_I], etc.
- *   DSA_MODE_DECODE: paged indexer scores for each sequence's context, top-k, then split
+ *   DSA_MODE_DECODE: the fused decode selection (dsa_indexer_topk_decode), then split
  *     sparse MLA with a log-sum-exp merge.
  * idx_out [rows, k] receives the selection when not NULL (otherwise it lives in workspace).
  */
@@ -252,7 +277,7 @@ dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale,
 
 /* Bytes of workspace dsa_forward / dsa_sparse_mla_decode need (0 when none): prefill, the
  * selection [total_tokens, k] int32; decode, the split partials of B sequences with H heads,
- * one score row of max_ctx entries per sequence and the selection [B, k]. */
+ * the decode selection's workspace (dsa_decode_select_workspace_size) and the selection [B, k]. */
 size_t dsa_workspace_size(int32_t mode, int32_t B, int64_t total_tokens, int32_t max_ctx, int32_t H, int32_t k);
 
 /* Static description of a status code. */

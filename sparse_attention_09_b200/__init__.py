@@ -35,7 +35,8 @@ EXPORTED = ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_ml
             "dsa_forward", "dsa_workspace_size", "dsa_status_string", "dsa_device_error",
             "dsa_sparse_mla_decode_noalloc", "dsa_quantize_fp8", "dsa_masked_mla_prefill",
             "dsa_indexer_topk_rows", "dsa_sparse_mla_prefill_rows", "dsa_attn_distribution", "dsa_indexer_kl",
-            "dsa_selftest_wait_timeout", "dsa_row_partition")
+            "dsa_selftest_wait_timeout", "dsa_row_partition", "dsa_indexer_topk_decode",
+            "dsa_decode_select_workspace_size")
 
 
 class KVDesc(ctypes.Structure):
@@ -98,6 +99,10 @@ _lib.dsa_quantize_fp8.argtypes = [_P, _I64, _I32, _P, _P, _P]
 _lib.dsa_quantize_fp8.restype = _I32
 _lib.dsa_workspace_size.argtypes = [_I32, _I32, _I64, _I32, _I32, _I32]
 _lib.dsa_workspace_size.restype = _SZ
+_lib.dsa_indexer_topk_decode.argtypes = [_P, _P, _I32, _P, _DESC, _I32, _I32, _I32, _I32, _P, _P, _SZ, _P]
+_lib.dsa_indexer_topk_decode.restype = _I32
+_lib.dsa_decode_select_workspace_size.argtypes = [_I32, _I32]
+_lib.dsa_decode_select_workspace_size.restype = _SZ
 
 
 class DSAError(RuntimeError):
@@ -261,6 +266,20 @@ def dsa_forward(mode, q_fp8, q_scale, w, keys: Desc, q, latent: Desc, B, H_I, d_
 
 def dsa_workspace_size(mode, B, total_tokens, max_ctx, H, k) -> int:
     return int(_lib.dsa_workspace_size(int(mode), int(B), int(total_tokens), int(max_ctx), int(H), int(k)))
+
+
+def dsa_decode_select_workspace_size(B, max_ctx) -> int:
+    return int(_lib.dsa_decode_select_workspace_size(int(B), int(max_ctx)))
+
+
+def dsa_indexer_topk_decode(q_fp8, q_scale, w, keys: Desc, B, H_I, d_I, k, idx_out, workspace, stream=None):
+    """Fused decode selection: paged indexer + per-sequence top-k; idx_out [B, k] (ascending,
+    -1 padded); workspace is a uint8 device tensor of dsa_decode_select_workspace_size bytes."""
+    _check(_lib.dsa_indexer_topk_decode(_ptr(q_fp8), _ptr(q_scale), _q_scale_heads(q_scale, H_I), _ptr(w),
+                                        keys.ref(), int(B), int(H_I), int(d_I), int(k), _ptr(idx_out),
+                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                        _stream(stream)), "dsa_indexer_topk_decode")
+    return idx_out
 
 
 def dsa_device_error(stream=None) -> int:

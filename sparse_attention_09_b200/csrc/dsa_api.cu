@@ -166,8 +166,10 @@ size_t decode_partials_bytes(int B, int H, int splits) {
 // one round on the CTA pairs: each unit costs a Q load, an O readout and fp32 partials, and
 // every chunk of a unit is one step of the same latency chain.  So splits is the largest power
 // of two s with B * s <= the number of CTA pairs (one round) and s <= k / 64 (a chunk per
-// unit), at least 1.  Measured on a B200 for 64 sequences, k = 2048 (MLA + combine): 1 split
-// 100 us, 2 splits 117 us, 4 splits 151 us, 8 splits 221 us.
+// unit), at least 1.  With one split the kernel writes out and lse itself (no partials, no
+// combine).  Measured on a B200 for 64 sequences, k = 2048 (MLA + combine, the latent-split
+// kernel that preceded the head-split pair): 1 split 100 us, 2 splits 117 us, 4 splits 151 us,
+// 8 splits 221 us.
 int decode_splits(int B, int k) {
   int s = 1;
   while (2 * s <= k / 64 && static_cast<int64_t>(B) * 2 * s <= kMlaClusters) s *= 2;
@@ -423,6 +425,46 @@ dsa_status dsa_indexer_topk_rows(const uint8_t* q_fp8, const float* q_scale, int
   return launch_indexer<kIdxTopk, false>(d_I, H_I, qm, km, p, grid, as_stream(stream));
 }
 
+size_t dsa_decode_select_workspace_size(int32_t B, int32_t max_ctx) {
+  if (B <= 0 || max_ctx <= 0) return 0;
+  const int64_t ld = (static_cast<int64_t>(max_ctx) + 3) / 4 * 4;
+  const int64_t ld16 = ((static_cast<int64_t>(max_ctx) + kSelGroup - 1) / kSelGroup + 3) / 4 * 4;
+  return align256(static_cast<size_t>(B) * ld * 4) + align256(static_cast<size_t>(B) * ld16 * 4);
+}
+
+dsa_status dsa_indexer_topk_decode(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
+                                   const dsa_kv_desc* keys, int32_t B, int32_t H_I, int32_t d_I, int32_t k,
+                                   int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (keys == nullptr || idx_out == nullptr || k <= 0 || B <= 0) return DSA_ERR_INVALID_ARGUMENT;
+  if (keys->kind != DSA_KV_PAGED) return DSA_ERR_UNSUPPORTED;
+  if (workspace == nullptr || !aligned(workspace, 256)) return DSA_ERR_INVALID_ARGUMENT;
+  if (static_cast<int64_t>(B) * kTopkCluster > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+  CUtensorMap qm, km;
+  IndexerParams p;
+  dsa_status st = indexer_common(q_fp8, q_scale, q_scale_heads, w, keys, B, H_I, d_I, &qm, &km, &p);
+  if (st != DSA_OK) return st;
+  if (ws_bytes < dsa_decode_select_workspace_size(B, keys->max_seqlen)) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  // workspace: [scores B x ld fp32][group maxima B x ld16 u32]
+  const int64_t ld = (static_cast<int64_t>(keys->max_seqlen) + 3) / 4 * 4;
+  const int64_t ld16 = ((static_cast<int64_t>(keys->max_seqlen) + kSelGroup - 1) / kSelGroup + 3) / 4 * 4;
+  p.scores = static_cast<float*>(workspace);
+  p.ld = ld;
+  p.row_begin = 0;
+  p.row_end = B;
+  p.gmax = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + align256(static_cast<size_t>(B) * ld * 4));
+  p.ld16 = ld16;
+  cudaStream_t s = as_stream(stream);
+  dim3 grid((keys->max_seqlen + 128 * kDecodeTilesPerCta - 1) / (128 * kDecodeTilesPerCta), B);
+  st = launch_indexer<kIdxScores, true>(d_I, H_I, qm, km, p, grid, s);
+  if (st != DSA_OK) return st;
+  if (cudaFuncSetAttribute(topk_decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmemBytes) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  topk_decode_select_kernel<<<static_cast<unsigned>(B * kTopkCluster), kTopkThreads, kSelSmemBytes, s>>>(
+      p.scores, ld, p.gmax, ld16, keys->context_lens, keys->max_seqlen, k, idx_out);
+  return launch_status();
+}
+
 dsa_status dsa_sparse_mla_prefill_rows(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t H,
                                        int32_t k, float sm_scale, int64_t row_begin, int64_t row_end, void* out,
                                        float* lse, void* stream) {
@@ -547,9 +589,12 @@ dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const
   p.part_o = static_cast<float*>(workspace);
   p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                        align256(static_cast<size_t>(B) * splits * H * kValueDim * 4));
+  p.out = static_cast<__nv_bfloat16*>(out);  // one split: the kernel writes out / lse itself
+  p.lse = lse;
   cudaStream_t s = as_stream(stream);
   dsa_status st = launch_mla_pair<true>(latent->data, q, B, p, static_cast<int64_t>(B) * splits, s);
   if (st != DSA_OK) return st;
+  if (splits == 1) return DSA_OK;
   mla_combine_kernel<<<dim3(H, B), 128, 0, s>>>(p.part_o, p.part_ml, splits, H, static_cast<__nv_bfloat16*>(out), lse);
   return launch_status();
 }
@@ -589,18 +634,14 @@ dsa_status dsa_forward(int32_t mode, const uint8_t* q_fp8, const float* q_scale,
   if (keys->kind != DSA_KV_PAGED || latent->kind != DSA_KV_PAGED) return DSA_ERR_INVALID_ARGUMENT;
   if (workspace == nullptr) return DSA_ERR_INVALID_ARGUMENT;
   if (ws_bytes < need || !aligned(workspace, 256)) return DSA_ERR_WORKSPACE_TOO_SMALL;
-  // workspace: [decode partials][scores B x ld][selection B x k]
+  // workspace: [decode partials][selection workspace: scores, group maxima][selection B x k]
   const int splits = decode_splits(B, k);
   const size_t part = decode_partials_bytes(B, H, splits);
-  const int64_t ld = (static_cast<int64_t>(keys->max_seqlen) + 3) / 4 * 4;
-  float* scores = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + part);
-  int32_t* idx = idx_out != nullptr
-                     ? idx_out
-                     : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + part +
-                                                  align256(static_cast<size_t>(B) * ld * 4));
-  dsa_status st = dsa_indexer_scores(q_fp8, q_scale, q_scale_heads, w, keys, B, H_I, d_I, 0, B, scores, ld, stream);
-  if (st != DSA_OK) return st;
-  st = dsa_topk(scores, ld, B, keys->context_lens, k, idx, stream);
+  const size_t sel = dsa_decode_select_workspace_size(B, keys->max_seqlen);
+  int32_t* idx = idx_out != nullptr ? idx_out
+                                    : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + part + sel);
+  dsa_status st = dsa_indexer_topk_decode(q_fp8, q_scale, q_scale_heads, w, keys, B, H_I, d_I, k, idx,
+                                          static_cast<uint8_t*>(workspace) + part, sel, stream);
   if (st != DSA_OK) return st;
   return dsa_sparse_mla_decode(q, latent, idx, B, H, k, sm_scale, out, lse, workspace, part, stream);
 }
@@ -640,8 +681,7 @@ dsa_status dsa_row_partition(int64_t L, int32_t k, int32_t parts, double indexer
 size_t dsa_workspace_size(int32_t mode, int32_t B, int64_t total_tokens, int32_t max_ctx, int32_t H, int32_t k) {
   if (B <= 0 || k <= 0 || H <= 0) return 0;
   if (mode == DSA_MODE_PREFILL) return align256(static_cast<size_t>(total_tokens > 0 ? total_tokens : 0) * k * 4);
-  const int64_t ld = (static_cast<int64_t>(max_ctx > 0 ? max_ctx : 0) + 3) / 4 * 4;
-  return decode_partials_bytes(B, H, decode_splits(B, k)) + align256(static_cast<size_t>(B) * ld * 4) +
+  return decode_partials_bytes(B, H, decode_splits(B, k)) + dsa_decode_select_workspace_size(B, max_ctx) +
          align256(static_cast<size_t>(B) * k * 4);
 }
 

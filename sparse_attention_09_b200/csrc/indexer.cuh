@@ -52,6 +52,8 @@ struct IndexerParams {
   int32_t tiles_per_cta;      // decode: key tiles per CTA
   float* scores;              // kIdxScores output
   int64_t ld;
+  uint32_t* gmax;             // paged kIdxScores, optional: [rows, ld16] order key of the largest
+  int64_t ld16;               //   score of each 16 consecutive keys (for the decode selection)
   int64_t row_begin, row_end;
   int32_t* idx_out;           // kIdxTopk output [T, k]
   int32_t tok_begin, tok_end; // top-k prefill: token positions [tok_begin, tok_end) of each sequence
@@ -406,7 +408,16 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
             if (gr >= p.row_begin && gr < p.row_end && s < len)
               p.scores[(gr - p.row_begin) * p.ld + s] = s <= t ? score : -INFINITY;
           } else {
-            if (s < len) p.scores[(b - p.row_begin) * p.ld + s] = bad_blk ? -INFINITY : score;
+            const float v = bad_blk ? -INFINITY : score;
+            if (s < len) p.scores[(b - p.row_begin) * p.ld + s] = v;
+            if (p.gmax != nullptr) {  // uniform: every lane takes part in the shuffles
+              // the largest key of the 16 keys of this half-warp (lanes 16h .. 16h+15 hold keys
+              // 16 * (s / 16) ..); keys past the context take no part
+              uint32_t key = s < len ? order_key(v) : 0u;
+#pragma unroll
+              for (int o = 8; o > 0; o >>= 1) key = max(key, __shfl_xor_sync(0xffffffffu, key, o));
+              if ((lane & 15) == 0 && s < len) p.gmax[(b - p.row_begin) * p.ld16 + (s >> 4)] = key;
+            }
           }
         }
       } else {

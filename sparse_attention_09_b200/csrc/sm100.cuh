@@ -22,12 +22,6 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint32_t lane_id() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%laneid;" : "=r"(r));
-  return r;
-}
-
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -113,20 +107,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Same, spinning on the non-blocking probe: for waits on the critical path, where a thread that
-// try_wait suspended can resume well after the phase completes.
-__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
-  const uint32_t a = smem_addr(bar);
-  if (mbar_poll(a, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_poll(a, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
-  }
-}
-
 // Same, with cluster-scope acquire: used where the arrivals come from the peer CTA.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_addr(bar);
@@ -166,31 +146,6 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t local_smem_addr, uint32
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem_addr), "r"(rank));
   return r;
-}
-
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-
-// Asynchronous store into another CTA's shared memory that counts its bytes on that CTA's
-// mbarrier (complete_tx); the storing thread does not wait for it.
-__device__ __forceinline__ void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                                            uint32_t remote_bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                   addr),
-               "r"(a), "r"(b), "r"(c), "r"(d), "r"(remote_bar)
-               : "memory");
-}
-
-__device__ __forceinline__ void st_async_b32(uint32_t addr, uint32_t v, uint32_t remote_bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
-               "r"(remote_bar)
-               : "memory");
 }
 
 // Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into another CTA's, done
@@ -255,15 +210,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t c0,
-                                            int32_t c1, int32_t c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-      "[%5];" ::"r"(smem_addr(dst)),
-      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
-      : "memory");
-}
-
 // ---------------------------------------------------------------------------------------
 // tcgen05: tensor memory
 // ---------------------------------------------------------------------------------------
@@ -301,11 +247,6 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// TMEM address of (lane, column).
-__device__ __forceinline__ uint32_t tmem_addr(uint32_t base, uint32_t lane, uint32_t col) {
-  return base + (lane << 16) + col;
-}
-
 // 32 lanes x 32 bit, 16 consecutive columns per thread.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -324,12 +265,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
-               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-               : "memory");
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -387,16 +322,6 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16.
-__device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // D[tmem] (+)= A[tmem] * B[smem]^T, bf16.
 __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                              uint32_t accumulate) {
@@ -441,50 +366,19 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
-// Issued by one thread of the even CTA of the pair.  A (M/2 rows per CTA) and B (N/2 rows per
-// CTA) are read from the same shared-memory offsets in both CTAs; each CTA's TMEM receives its
-// M/2 rows x N columns of D (for M = 128: columns [0, N/2) on lanes 0-63, [N/2, N) on lanes 64-127).
-__device__ __forceinline__ void umma_bf16_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                                  uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Warp-collective form of the above: every lane passes the same (warp-uniform) operands and one
-// elected lane issues.  Measured on B200 for M = 128, N = 64: 25 cycles per MMA (the shared-memory
-// operand rate) against 45 when one lane builds the descriptors and issues inside a lane branch.
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16, on the CTA pair (cta_group::2): A (M/2 rows per CTA)
+// and B (N/2 rows per CTA) are read from the same shared-memory offsets in both CTAs; each CTA's
+// TMEM receives its M/2 rows x N columns of D (for M = 128: columns [0, N/2) on lanes 0-63,
+// [N/2, N) on lanes 64-127).  Warp-collective, in the even CTA: every lane passes the same
+// (warp-uniform) operands and one elected lane issues.  Measured on B200 for M = 128, N = 64:
+// 25 cycles per MMA (the shared-memory operand rate) against 45 when one lane builds the
+// descriptors and issues inside a lane branch.
 __device__ __forceinline__ void umma_bf16_ss_pair_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                                        uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Same, A from tensor memory (each CTA's 64 rows of A held twice: rows 0-31 on lanes 0-31 and
-// 64-95, rows 32-63 on lanes 32-63 and 96-127; K = 16 bf16 = 8 columns per instruction).
-__device__ __forceinline__ void umma_bf16_ts_pair_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Copies a 64-row x 16-byte slice of a shared-memory matrix (described like an MMA operand) into
-// tensor memory of both CTAs of the pair, rows 0-31 to lanes 0-31 and 64-95, rows 32-63 to lanes
-// 32-63 and 96-127 (the layout of a pair MMA's A operand in tensor memory), 4 columns.  Issued by
-// one elected lane; ordered with the same thread's later tcgen05.mma.
-__device__ __forceinline__ void tmem_cp_pair_64x128b_warp(uint32_t taddr, uint64_t s_desc) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.cp.cta_group::2.64x128b.warpx2::02_13 [%0], %1;\n\t}\n" ::"r"(taddr),
-      "l"(s_desc)
       : "memory");
 }
 
@@ -504,19 +398,6 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mas
 // costlier cluster-scope release (a cluster-wide memory fence per arrival) is not needed.
 __device__ __forceinline__ void mbar_arrive_peer(uint32_t cluster_bar_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar_addr) : "memory");
-}
-
-// Non-blocking probe with cluster-scope acquire (the barrier receives arrivals from the peer).
-__device__ __forceinline__ bool mbar_poll_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
 }
 
 // ---------------------------------------------------------------------------------------

@@ -634,7 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mlap::kThreads, 1)
         break;
       }
       tc_fence_after();
-      if constexpr (!DECODE) {
+      if (!DECODE || p.splits == 1) {  // whole selection in this unit: O / l straight to out
         const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
         __nv_bfloat16* orow = p.out + (un.qrow * p.H + h) * 512 + 128 * kh;
 #pragma unroll 1

@@ -1,12 +1,22 @@
-// Row-wise top-k over fp32 index scores (fine-grained token selection).
+// Row-wise top-k over fp32 index scores (fine-grained token selection: the k largest index
+// scores of a query, ties to the lower key index, indices written ascending).
 //
-// A 4-pass radix select over the order-preserving 32-bit keys of the
-// scores (8 bits per pass, warp-private histograms) finds the key of the k-th largest entry
-// and how many entries equal to it are still needed; an emit pass then walks the row in
-// index order and writes the selected indices with a block-wide scan, so the output is
-// ascending and ties at the boundary go to the lowest indices.  Each thread takes 16
-// consecutive scores per step (four 16-byte loads in flight), so a step covers 8192 scores.
-// A row is handled by a cluster of CTAs (below).
+// Core: a 4-pass radix select over the order-preserving 32-bit keys of the scores (8 bits per
+// pass, warp-private histograms merged over a cluster of CTAs through distributed shared
+// memory) finds the key of the k-th largest entry and how many entries equal to it are still
+// needed; an emit pass then walks the entries in index order and writes the selected indices
+// with a block-wide scan, so the output is ascending and ties at the boundary go to the lowest
+// indices.  A row is handled by a cluster of kTopkCluster CTAs, each taking a contiguous
+// segment of it.  The core reads its entries through a source: a segment of a score row in
+// global memory (dsa_topk), or the candidates a CTA holds in shared memory (decode selection).
+//
+// Decode selection (topk_decode_select_kernel): the paged indexer also writes, per 16 keys,
+// the largest key of the group.  tau = the k-th largest group maximum is a lower bound of the
+// row's k-th largest score: at least k groups have a maximum >= tau and each holds one score
+// >= tau.  One streaming pass keeps the scores >= tau (in index order, in shared memory); for
+// 128K-key rows these are ~2-3K entries instead of 128K, and the exact radix select and the
+// emission run on them.  A row whose candidates overflow a CTA's buffer falls back to the
+// core over the row in global memory, in the same kernel (same result, slower).
 #pragma once
 
 #include "common.cuh"
@@ -17,7 +27,8 @@ namespace dsa {
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkVec = 4;                               // float4 loads per thread per step
-constexpr int kTopkTile = 4 * kTopkVec * kTopkThreads;    // scores per step
+constexpr int kTopkTile = 4 * kTopkVec * kTopkThreads;    // entries per step
+constexpr int kTopkCluster = 4;
 
 // The 16 scores [i0, i0 + 16) of a row of length n (entries past n are not loaded; a row
 // buffer of ld >= n elements, ld % 4 == 0, holds every float4 that starts before n).
@@ -33,96 +44,110 @@ __device__ __forceinline__ void topk_load16(const float* row, int i0, int n, flo
   }
 }
 
-// A cluster of C CTAs per row, each taking a contiguous segment of it
-// (a multiple of 16 scores).  Every radix pass merges the C segment histograms through
-// distributed shared memory, so all CTAs take the same decision; each CTA also counts, from
-// its own histograms, its scores above the final threshold and its scores equal to it.  In
-// the emit pass CTA c writes at the offset of the selected scores of the segments before it,
-// taking as many ties as the row still needs after theirs (ties go to the lowest indices).
 namespace topk_detail {
+
 __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
   return v;
 }
-}  // namespace topk_detail
 
-constexpr int kTopkCluster = 4;
+struct Shared {
+  uint32_t hist[kTopkWarps][256];
+  uint32_t total[2][256];   // this CTA's histogram of a pass (double-buffered: peers read it)
+  uint32_t gtotal[256];     // the row's histogram of the pass
+  int scan_scratch[kTopkWarps];
+  uint32_t s_bin, s_remaining, s_above;
+  uint32_t s_cnt[2];        // this CTA's entries above / equal to the threshold
+};
 
-__global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThreads)
-    topk_rows_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ row_len,
-                             int32_t k, int32_t* __restrict__ idx) {
+// Entries [begin, end) of a score row in global memory; the index of entry i is i.
+struct RowSource {
+  const float* row;
+  int begin, end;
+  bool nan_check;  // report NaN scores (first pass only)
+  __device__ __forceinline__ void load16(int i0, bool first_pass, uint32_t (&key)[16], int32_t (&idx)[16]) const {
+    float f[16];
+    topk_load16(row, i0, end, f);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (nan_check && first_pass && i0 + j < end && is_nan_bits(__float_as_uint(f[j])))
+        record_device_error(DSA_ERR_DEVICE_CHECK);
+      key[j] = order_key(f[j]);
+      idx[j] = i0 + j;
+    }
+  }
+};
+
+// Candidates [0, end) held in shared memory as (order key, index), in index order.
+struct CandSource {
+  const uint32_t* key;
+  const int32_t* idx;
+  int begin, end;
+  __device__ __forceinline__ void load16(int i0, bool, uint32_t (&k)[16], int32_t (&ix)[16]) const {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      uint4 a = make_uint4(0u, 0u, 0u, 0u);
+      int4 b = make_int4(0, 0, 0, 0);
+      if (i0 + 4 * v < end) {  // the buffers are padded to a multiple of 16 entries
+        a = *reinterpret_cast<const uint4*>(key + i0 + 4 * v);
+        b = *reinterpret_cast<const int4*>(idx + i0 + 4 * v);
+      }
+      k[4 * v] = a.x; k[4 * v + 1] = a.y; k[4 * v + 2] = a.z; k[4 * v + 3] = a.w;
+      ix[4 * v] = b.x; ix[4 * v + 1] = b.y; ix[4 * v + 2] = b.z; ix[4 * v + 3] = b.w;
+    }
+  }
+};
+
+// The radix select and ordered emission over the C CTAs of a cluster, each holding the
+// entries [src.begin, src.end) of the row (CTA c's entries precede CTA c+1's in index order).
+// Every CTA of the cluster calls it with the same k; it ends with a cluster barrier, so no CTA
+// leaves while a peer may still read its shared memory.
+template <class Src>
+__device__ void radix_select_emit(const Src& src, int k, int32_t* __restrict__ out, Shared& sh) {
   constexpr int C = kTopkCluster;
-  __shared__ uint32_t hist[kTopkWarps][256];
-  __shared__ uint32_t total[2][256];   // this CTA's histogram of a pass (double-buffered: peers read it)
-  __shared__ uint32_t gtotal[256];     // the row's histogram of the pass
-  __shared__ int scan_scratch[kTopkWarps];
-  __shared__ uint32_t s_bin, s_remaining, s_above;
-  __shared__ uint32_t s_cnt[2];        // this CTA's scores above / equal to the threshold
-
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = dev::cluster_ctarank();
-  const int64_t r = blockIdx.x / C;
-  const float* row = scores + r * ld;
-  int32_t* out = idx + r * static_cast<int64_t>(k);
-  int n = row_len[r];
-  if (n < 0 || n > ld) {  // a row length outside [0, ld] is an input error; the row is clamped
-    if (threadIdx.x == 0 && rank == 0) record_device_error(DSA_ERR_DEVICE_CHECK);
-    n = n < 0 ? 0 : static_cast<int>(ld);
-  }
-
-  if (n <= k) {  // every candidate is selected (the same decision in every CTA of the row)
-    if (rank == 0)
-      for (int i = tid; i < k; i += kTopkThreads) out[i] = i < n ? i : -1;
-    return;
-  }
-  const int per = ((n + C - 1) / C + 15) / 16 * 16;
-  const int seg0 = min(n, static_cast<int>(rank) * per), seg1 = min(n, seg0 + per);
-
   uint32_t prefix = 0, mask = 0, remaining = static_cast<uint32_t>(k);
-  if (tid == 0) s_above = 0u;  // this segment's scores known to be above the threshold
+  if (tid == 0) sh.s_above = 0u;  // this segment's entries known to be above the threshold
 #pragma unroll 1
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int i = tid; i < kTopkWarps * 256; i += kTopkThreads) (&hist[0][0])[i] = 0u;
+    for (int i = tid; i < kTopkWarps * 256; i += kTopkThreads) (&sh.hist[0][0])[i] = 0u;
     __syncthreads();
 #pragma unroll 1
-    for (int base = seg0; base < seg1; base += kTopkTile) {
+    for (int base = src.begin; base < src.end; base += kTopkTile) {
       const int i0 = base + 16 * tid;
-      if (i0 < seg1) {
-        float f[16];
-        topk_load16(row, i0, seg1, f);
+      if (i0 < src.end) {
+        uint32_t key[16];
+        int32_t ix[16];
+        src.load16(i0, pass == 0, key, ix);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          if (i0 + j < seg1) {
-            if (pass == 0 && is_nan_bits(__float_as_uint(f[j]))) record_device_error(DSA_ERR_DEVICE_CHECK);
-            const uint32_t key = order_key(f[j]);
-            if ((key & mask) == prefix) atomicAdd(&hist[warp][(key >> shift) & 255u], 1u);
-          }
-        }
+        for (int j = 0; j < 16; ++j)
+          if (i0 + j < src.end && (key[j] & mask) == prefix) atomicAdd(&sh.hist[warp][(key[j] >> shift) & 255u], 1u);
       }
     }
     __syncthreads();
     if (tid < 256) {
       uint32_t s = 0;
 #pragma unroll
-      for (int w = 0; w < kTopkWarps; ++w) s += hist[w][tid];
-      total[pass & 1][tid] = s;
+      for (int w = 0; w < kTopkWarps; ++w) s += sh.hist[w][tid];
+      sh.total[pass & 1][tid] = s;
     }
     dev::cluster_sync();  // every CTA's histogram of this pass is complete
     if (tid < 256) {
-      const uint32_t a = dev::smem_addr(&total[pass & 1][tid]);
+      const uint32_t a = dev::smem_addr(&sh.total[pass & 1][tid]);
       uint32_t s = 0;
 #pragma unroll
-      for (int c = 0; c < C; ++c) s += topk_detail::ld_cluster_u32(dev::map_to_rank(a, c));
-      gtotal[tid] = s;
+      for (int c = 0; c < C; ++c) s += ld_cluster_u32(dev::map_to_rank(a, c));
+      sh.gtotal[tid] = s;
     }
     __syncthreads();
     if (warp == 0) {
       uint32_t c[8], sum = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        c[j] = gtotal[255 - (8 * lane + j)];
+        c[j] = sh.gtotal[255 - (8 * lane + j)];
         sum += c[j];
       }
       const uint32_t inc = static_cast<uint32_t>(warp_inclusive_scan(static_cast<int>(sum)));
@@ -132,8 +157,8 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           if (acc + c[j] >= remaining) {
-            s_bin = 255u - static_cast<uint32_t>(8 * lane + j);
-            s_remaining = remaining - acc;
+            sh.s_bin = 255u - static_cast<uint32_t>(8 * lane + j);
+            sh.s_remaining = remaining - acc;
             break;
           }
           acc += c[j];
@@ -141,50 +166,50 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
       }
     }
     __syncthreads();
-    const uint32_t bin = s_bin;
-    // this segment's scores of this pass's prefix in bins above the chosen one are above the
+    const uint32_t bin = sh.s_bin;
+    // this segment's entries of this pass's prefix in bins above the chosen one are above the
     // threshold; in the last pass, those in the chosen bin are equal to it
-    if (tid < 256 && static_cast<uint32_t>(tid) > bin) atomicAdd(&s_above, total[pass & 1][tid]);
-    if (pass == 3 && tid == 0) s_cnt[1] = total[pass & 1][bin];
+    if (tid < 256 && static_cast<uint32_t>(tid) > bin) atomicAdd(&sh.s_above, sh.total[pass & 1][tid]);
+    if (pass == 3 && tid == 0) sh.s_cnt[1] = sh.total[pass & 1][bin];
     prefix |= bin << shift;
     mask |= 255u << shift;
-    remaining = s_remaining;
+    remaining = sh.s_remaining;
     __syncthreads();
   }
-  if (tid == 0) s_cnt[0] = s_above;
+  if (tid == 0) sh.s_cnt[0] = sh.s_above;
   dev::cluster_sync();  // the segment counts are published
   // this CTA's output offset and tie quota from the segments before it
   const int need_eq = static_cast<int>(remaining);
   int offset = 0, ties_before = 0;
   for (int c = 0; c < static_cast<int>(rank); ++c) {
-    const int g = static_cast<int>(topk_detail::ld_cluster_u32(dev::map_to_rank(dev::smem_addr(&s_cnt[0]), c)));
-    const int e = static_cast<int>(topk_detail::ld_cluster_u32(dev::map_to_rank(dev::smem_addr(&s_cnt[1]), c)));
+    const int g = static_cast<int>(ld_cluster_u32(dev::map_to_rank(dev::smem_addr(&sh.s_cnt[0]), c)));
+    const int e = static_cast<int>(ld_cluster_u32(dev::map_to_rank(dev::smem_addr(&sh.s_cnt[1]), c)));
     offset += g + min(e, max(0, need_eq - ties_before));
     ties_before += e;
   }
   const int quota = max(0, need_eq - ties_before);  // ties this segment may still take
-  const int my_total = static_cast<int>(s_cnt[0]) + min(static_cast<int>(s_cnt[1]), quota);
+  const int my_total = static_cast<int>(sh.s_cnt[0]) + min(static_cast<int>(sh.s_cnt[1]), quota);
 
   const uint32_t thr = prefix;
   int eq_taken = 0, out_pos = offset;
 #pragma unroll 1
-  for (int base = seg0; base < seg1 && out_pos < offset + my_total; base += kTopkTile) {
+  for (int base = src.begin; base < src.end && out_pos < offset + my_total; base += kTopkTile) {
     const int i0 = base + 16 * tid;
     uint32_t gbits = 0u, ebits = 0u;
-    if (i0 < seg1) {
-      float f[16];
-      topk_load16(row, i0, seg1, f);
+    int32_t ix[16];
+    if (i0 < src.end) {
+      uint32_t key[16];
+      src.load16(i0, false, key, ix);
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        if (i0 + j < seg1) {
-          const uint32_t key = order_key(f[j]);
-          gbits |= static_cast<uint32_t>(key > thr) << j;
-          ebits |= static_cast<uint32_t>(key == thr) << j;
+        if (i0 + j < src.end) {
+          gbits |= static_cast<uint32_t>(key[j] > thr) << j;
+          ebits |= static_cast<uint32_t>(key[j] == thr) << j;
         }
       }
     }
     int tie_total;
-    int tie_rank = eq_taken + block_exclusive_scan<kTopkWarps>(__popc(ebits), scan_scratch, tie_total);
+    int tie_rank = eq_taken + block_exclusive_scan<kTopkWarps>(__popc(ebits), sh.scan_scratch, tie_total);
     uint32_t sbits = gbits;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -194,14 +219,209 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
       }
     }
     int sel_total;
-    int pos = out_pos + block_exclusive_scan<kTopkWarps>(__popc(sbits), scan_scratch, sel_total);
+    int pos = out_pos + block_exclusive_scan<kTopkWarps>(__popc(sbits), sh.scan_scratch, sel_total);
 #pragma unroll
     for (int j = 0; j < 16; ++j)
-      if ((sbits >> j) & 1u) out[pos++] = i0 + j;
+      if ((sbits >> j) & 1u) out[pos++] = ix[j];
     eq_taken += tie_total;
     out_pos += sel_total;
   }
   dev::cluster_sync();  // no CTA leaves while a peer may still read its shared memory
+}
+
+// Row length check shared by the kernels: a length outside [0, cap] is an input error; the
+// row is clamped.
+__device__ __forceinline__ int checked_len(int n, int64_t cap, bool report) {
+  if (n < 0 || n > cap) {
+    if (report) record_device_error(DSA_ERR_DEVICE_CHECK);
+    n = n < 0 ? 0 : static_cast<int>(cap);
+  }
+  return n;
+}
+
+}  // namespace topk_detail
+
+// dsa_topk: one cluster per row over the scores in global memory.
+__global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThreads)
+    topk_rows_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ row_len,
+                             int32_t k, int32_t* __restrict__ idx) {
+  constexpr int C = kTopkCluster;
+  __shared__ topk_detail::Shared sh;
+  const int tid = threadIdx.x;
+  const uint32_t rank = dev::cluster_ctarank();
+  const int64_t r = blockIdx.x / C;
+  int32_t* out = idx + r * static_cast<int64_t>(k);
+  const int n = topk_detail::checked_len(row_len[r], ld, threadIdx.x == 0 && rank == 0);
+  if (n <= k) {  // every candidate is selected (the same decision in every CTA of the row)
+    if (rank == 0)
+      for (int i = tid; i < k; i += kTopkThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  const int per = ((n + C - 1) / C + 15) / 16 * 16;
+  const int seg0 = min(n, static_cast<int>(rank) * per), seg1 = min(n, seg0 + per);
+  topk_detail::radix_select_emit(topk_detail::RowSource{scores + r * ld, seg0, seg1, true}, k, out, sh);
+}
+
+// ---- decode selection ------------------------------------------------------------------------
+constexpr int kSelGroup = 16;     // scores per group maximum (written by the paged indexer)
+constexpr int kSelCap = 8192;     // candidates a CTA holds (key + index: 64 KB of shared memory)
+constexpr int kSelBins = 2048;    // 11-bit digits for the bound on the group maxima
+constexpr int kSelSmemBytes = kSelCap * 8;
+
+namespace topk_detail {
+
+// tau <= the k-th largest of the G group maxima gm[0..G): the 22-bit prefix of that maximum
+// with the low 10 bits cleared (two 11-bit histogram passes).  Every thread of the CTA calls it;
+// `hist` holds kSelBins counters.
+__device__ uint32_t group_max_bound(const uint32_t* __restrict__ gm, int G, int k, uint32_t* hist, Shared& sh) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  uint32_t prefix = 0, mask = 0, remaining = static_cast<uint32_t>(k);
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const int shift = 21 - 11 * pass;
+    for (int i = tid; i < kSelBins; i += kTopkThreads) hist[i] = 0u;
+    __syncthreads();
+#pragma unroll 1
+    for (int base = 0; base < G; base += 4 * kTopkThreads) {
+      const int i = base + 4 * tid;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (i + 3 < G) {
+        v = *reinterpret_cast<const uint4*>(gm + i);
+      } else if (i < G) {
+        v.x = gm[i];
+        if (i + 1 < G) v.y = gm[i + 1];
+        if (i + 2 < G) v.z = gm[i + 2];
+      }
+      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const bool ok = i + j < G && (vv[j] & mask) == prefix;
+        const uint32_t d = ok ? (vv[j] >> shift) & (kSelBins - 1) : 0xFFFFFFFFu;
+        // one atomic per distinct digit of the warp: group maxima share few digits
+        const uint32_t peers = __match_any_sync(0xffffffffu, d);
+        if (ok && (__ffs(peers) - 1) == lane) atomicAdd(&hist[d], static_cast<uint32_t>(__popc(peers)));
+      }
+    }
+    __syncthreads();
+    // the bin of the remaining-th largest, counting from the top bin (4 bins per thread)
+    constexpr int BPT = kSelBins / kTopkThreads;
+    uint32_t c[BPT], sum = 0;
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {
+      c[j] = hist[kSelBins - 1 - (BPT * tid + j)];
+      sum += c[j];
+    }
+    int tot;
+    const uint32_t before = static_cast<uint32_t>(block_exclusive_scan<kTopkWarps>(static_cast<int>(sum), sh.scan_scratch, tot));
+    if (before < remaining && remaining <= before + sum) {
+      uint32_t acc = before;
+#pragma unroll
+      for (int j = 0; j < BPT; ++j) {
+        if (acc + c[j] >= remaining) {
+          sh.s_bin = static_cast<uint32_t>(kSelBins - 1 - (BPT * tid + j));
+          sh.s_remaining = remaining - acc;
+          break;
+        }
+        acc += c[j];
+      }
+    }
+    __syncthreads();
+    prefix |= sh.s_bin << shift;
+    mask |= static_cast<uint32_t>(kSelBins - 1) << shift;
+    remaining = sh.s_remaining;
+    __syncthreads();
+  }
+  return prefix;
+}
+
+}  // namespace topk_detail
+
+// Per-sequence selection after the paged indexer: scores [B, ld] (entries [0, n_b)), gmax
+// [B, ld16] (order key of the largest score of entries [16 g, 16 g + 16) of the row), n_b =
+// min(context_lens[b], max_len).  One cluster of kTopkCluster CTAs per row.
+__global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThreads)
+    topk_decode_select_kernel(const float* __restrict__ scores, int64_t ld, const uint32_t* __restrict__ gmax,
+                              int64_t ld16, const int32_t* __restrict__ context_lens, int32_t max_len, int32_t k,
+                              int32_t* __restrict__ idx) {
+  constexpr int C = kTopkCluster;
+  extern __shared__ uint8_t sel_smem[];
+  uint32_t* cand_key = reinterpret_cast<uint32_t*>(sel_smem);
+  int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_key + kSelCap);
+  __shared__ topk_detail::Shared sh;
+  __shared__ int s_count;
+  const int tid = threadIdx.x;
+  const uint32_t rank = dev::cluster_ctarank();
+  const int64_t r = blockIdx.x / C;
+  int32_t* out = idx + r * static_cast<int64_t>(k);
+  // the indexer reports a context longer than max_len; here it is clamped the same way
+  const int n = topk_detail::checked_len(min(context_lens[r], max_len), ld, threadIdx.x == 0 && rank == 0);
+  if (n <= k) {
+    if (rank == 0)
+      for (int i = tid; i < k; i += kTopkThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  const float* row = scores + r * ld;
+  const int G = (n + kSelGroup - 1) / kSelGroup;
+  // with fewer groups than k the maxima bound nothing: every score is a candidate
+  const uint32_t tau = G >= k ? topk_detail::group_max_bound(gmax + r * ld16, G, k, &sh.hist[0][0], sh) : 0u;
+
+  // one pass over this CTA's segment: the scores >= tau, in index order
+  const int per = ((n + C - 1) / C + 15) / 16 * 16;
+  const int seg0 = min(n, static_cast<int>(rank) * per), seg1 = min(n, seg0 + per);
+  int count = 0;
+#pragma unroll 1
+  for (int base = seg0; base < seg1 && count <= kSelCap; base += kTopkTile) {
+    const int i0 = base + 16 * tid;
+    uint32_t keep = 0u, key[16];
+    if (i0 < seg1) {
+      float f[16];
+      topk_load16(row, i0, seg1, f);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (i0 + j < seg1 && is_nan_bits(__float_as_uint(f[j]))) record_device_error(DSA_ERR_DEVICE_CHECK);
+        key[j] = order_key(f[j]);
+        keep |= static_cast<uint32_t>(i0 + j < seg1 && key[j] >= tau) << j;
+      }
+    }
+    int total;
+    int pos = count + block_exclusive_scan<kTopkWarps>(__popc(keep), sh.scan_scratch, total);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if ((keep >> j) & 1u) {
+        if (pos < kSelCap) {
+          cand_key[pos] = key[j];
+          cand_idx[pos] = i0 + j;
+        }
+        ++pos;
+      }
+    }
+    count += total;
+  }
+  // pad to a multiple of 16 entries (the source loads whole 16-entry groups)
+  if (count <= kSelCap) {
+    const int pad_end = min(kSelCap, (count + 15) / 16 * 16);
+    for (int i = count + tid; i < pad_end; i += kTopkThreads) {
+      cand_key[i] = 0u;
+      cand_idx[i] = -1;
+    }
+  }
+  if (tid == 0) s_count = count;
+  __syncthreads();
+  dev::cluster_sync();  // the candidate counts are published
+  int total = 0;
+  bool overflow = false;
+  for (int c = 0; c < C; ++c) {
+    const int cc = static_cast<int>(topk_detail::ld_cluster_u32(dev::map_to_rank(dev::smem_addr(&s_count), c)));
+    total += min(cc, kSelCap + 1);
+    overflow |= cc > kSelCap;
+  }
+  if (overflow || total < k) {
+    // too many candidates for the buffers (e.g. a tie class of thousands at the boundary):
+    // the exact select over the row in global memory
+    topk_detail::radix_select_emit(topk_detail::RowSource{row, seg0, seg1, true}, k, out, sh);
+  } else {
+    topk_detail::radix_select_emit(topk_detail::CandSource{cand_key, cand_idx, 0, count}, k, out, sh);
+  }
 }
 
 }  // namespace dsa
