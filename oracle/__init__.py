@@ -39,6 +39,15 @@ Parity status per function (what pins it, in ``tests/test_oracle_*.py``):
   head = the softmax of its logits, equal logits = uniform, head-permutation invariance; KL >= 0,
   0 exactly when the scores are log p plus a constant, the gradient sums to 0 and matches
   central finite differences of the loss, and a two-point closed form).
+* ``attention_distribution_dense_token``: pinned (equals the attention weights a library
+  scaled-dot-product attention returns with identity values, averaged over heads; sums to 1;
+  a zero query gives the uniform distribution; two keys of one head give the logistic closed form).
+* ``indexer_backward_query`` / ``indexer_backward``: pinned (every component matches central
+  finite differences of an independently written real-valued forward that itself equals
+  ``indexer_scores_query`` on dequantised codes; closed form for one head and one key; zero
+  where every ReLU is off; planted mistakes -- a dropped ReLU mask, a dropped head weight, a
+  transposed key gradient -- fail the difference check; the sequence form adds key gradients
+  over the queries that selected the key).
 * ``encode_e4m3`` / ``quantize_fp8_rows``: pinned (every finite code round-trips; midpoints
   between neighbouring values go to the even code; saturation and NaN; agreement with torch's
   float8_e4m3fn cast on random values; the per-row scale rule and its error bound).
@@ -60,7 +69,10 @@ from .dsa_oracle import (  # noqa: F401
     sparse_mla_token,
     sparse_mla,
     attention_distribution_token,
+    attention_distribution_dense_token,
     indexer_kl,
+    indexer_backward_query,
+    indexer_backward,
     paged_gather,
     decode_indexer_scores,
     dsa_prefill_rows,

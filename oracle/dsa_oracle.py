@@ -233,6 +233,69 @@ def indexer_kl(p: np.ndarray, scores: np.ndarray):
     return loss, np.exp(logq) - p
 
 
+def attention_distribution_dense_token(q: np.ndarray, latent_prefix: np.ndarray, sm_scale: float):
+    """Target of the dense warm-up stage for one query: the main attention's distribution over
+    the query's whole causal prefix, averaged over heads ([MZ] 二 "两阶段继续预训练", dense
+    warm-up: attention stays dense and the indexer alone is trained, by a KL loss, to match the
+    main attention's output distribution; [36] "DSA 訓練的兩個階段", stage one).
+    Reading: the same aggregation as the sparse stage (mean over heads of the per-head softmax),
+    taken over every preceding token (rows 0..t) instead of the selected set.
+    q: [H, D], latent_prefix: [t+1, D].  Returns float64 [t+1]."""
+    c = np.asarray(latent_prefix, np.float64)
+    logits = float(sm_scale) * (np.asarray(q, np.float64) @ c.T)     # [H, t+1]
+    mx = logits.max(axis=1, keepdims=True)
+    e = np.exp(logits - mx)
+    return (e / e.sum(axis=1, keepdims=True)).mean(axis=0)
+
+
+def indexer_backward_query(q8: np.ndarray, q_scale, w: np.ndarray, k8: np.ndarray, k_scale: np.ndarray,
+                           g: np.ndarray):
+    """Backward of the indexer for one query token ([MZ] 二 "两阶段继续预训练": the indexer is
+    trained by the KL loss alone, with its input detached from the main model's graph).
+
+    Given g[s] = d loss / d I[s] over a set of keys (the KL gradient, q_s - p_s), returns the
+    gradient of sum_s g[s] * I[s] with I[s] = sum_j w[j] * ReLU(q_I[j] . k_I[s]):
+      dw[j]    = sum_s g[s] * ReLU(a[j,s]),                 a[j,s] = q_I[j] . k_I[s]
+      dq_I[j]  = sum_s g[s] * w[j] * [a[j,s] > 0] * k_I[s]
+      dk_I[s]  = g[s] * sum_j w[j] * [a[j,s] > 0] * q_I[j]
+    Readings: the gradient is taken with respect to the dequantised operands q_I =
+    e4m3(q8) * q_scale and k_I = e4m3(k8) * k_scale (the real values the FP8 codes stand for;
+    the quantiser passes it through); ReLU'(0) = 0.
+    q8: [H_I, d_I], q_scale: scalar or [H_I], w: [H_I], k8: [n, d_I], k_scale: [n], g: [n].
+    Returns (dw [H_I], dq [H_I, d_I], dk [n, d_I]), float64."""
+    qs = np.asarray(q_scale, np.float64)
+    q = decode_e4m3(q8) * (qs[:, None] if qs.ndim == 1 else qs)   # [H_I, d_I]
+    k = decode_e4m3(k8) * np.asarray(k_scale, np.float64)[:, None]  # [n, d_I]
+    g = np.asarray(g, np.float64)
+    w = np.asarray(w, np.float64)
+    a = q @ k.T                                                 # [H_I, n]
+    dw = np.maximum(a, 0.0) @ g
+    m = (a > 0.0) * w[:, None] * g[None, :]                     # d loss / d a[j, s]
+    return dw, m @ k, m.T @ q
+
+
+def indexer_backward(q8: np.ndarray, q_scale: np.ndarray, w: np.ndarray, k8: np.ndarray, k_scale: np.ndarray,
+                     idx: np.ndarray, grad: np.ndarray):
+    """Backward of the indexer over one sequence: token t's gradient grad[t, i] = d loss /
+    d I[t, idx[t, i]] on its selected keys (idx -1 padded; in the dense stage the selection is
+    the whole prefix).  Key gradients add up over every query that selected the key.
+    q8: [L, H_I, d_I], q_scale: [L] or [L, H_I], w: [L, H_I], k8: [L, d_I], k_scale: [L],
+    idx / grad: [L, m].  Returns (dw [L, H_I], dq [L, H_I, d_I], dk [L, d_I]), float64."""
+    L, H_I, d_I = q8.shape
+    dw = np.zeros((L, H_I))
+    dq = np.zeros((L, H_I, d_I))
+    dk = np.zeros((k8.shape[0], d_I))
+    for t in range(L):
+        valid = idx[t] >= 0
+        sel = np.asarray(idx[t][valid], np.int64)
+        if sel.size == 0:
+            continue
+        dw[t], dq[t], dks = indexer_backward_query(q8[t], q_scale[t], w[t], k8[sel], k_scale[sel],
+                                                   np.asarray(grad[t], np.float64)[valid])
+        np.add.at(dk, sel, dks)
+    return dw, dq, dk
+
+
 def sparse_mla(q: np.ndarray, latent: np.ndarray, idx: np.ndarray, sm_scale: float, rows=None,
                dv: int = 512):
     """Prefill sparse MLA of one sequence for the given rows; idx [L, k] is -1 padded.
