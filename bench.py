@@ -575,7 +575,46 @@ def run_kl(dsa, inp, idx, cfg, sm):
     res["indexer_kl_gbs"] = T * k * 4 * 4 / (res["indexer_kl_ms"] * 1e-3) / 1e9  # p, scores, idx read; grad written
     res["mean_row_sum_p"] = float(p.sum(dim=1).mean().item())
     assert dsa.dsa_device_error() == 0
-    del p, scores, loss, grad, lse
+    del p, scores, loss
+    torch.cuda.empty_cache()
+
+    # dense warm-up target on the last 1024 query rows of the first sequence (their causal
+    # prefixes are the longest); the sparse forward's lse stands in for the dense one (the
+    # kernel's cost does not depend on its values)
+    L0 = cfg["seqlens"][0]
+    R = min(1024, L0)
+    pd = torch.empty((R, L0), device="cuda")
+    # the indexer backward over every token's selection; the KL gradient is a random stand-in
+    H_I, d_I = cfg["H_I"], cfg["d_I"]
+    keys = dsa.contiguous_desc(inp["k8"], inp["cu_seqlens"], max(inp["seqlens"]), scale=inp["k_scale"])
+    dw = torch.empty((T, H_I), device="cuda")
+    dq = torch.empty((T, H_I, d_I), device="cuda")
+    dkey = torch.empty((T, d_I), device="cuda")
+    grad.normal_()
+    for name, fn, reps in (
+            ("attn_distribution_dense", lambda: dsa.dsa_attn_distribution_dense(
+                inp["q"], lat, lse, nseq, H, L0 - R, L0, sm, pd), 3),
+            ("indexer_backward", lambda: dsa.dsa_indexer_backward(
+                inp["q8"], inp["q_scale"], inp["w"], keys, nseq, H_I, d_I, idx, grad, dw, dq, dkey), 1)):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        res[name + "_ms"] = e0.elapsed_time(e1) / reps
+    dense_pairs = sum(t + 1 for t in range(L0 - R, L0))
+    res["attn_distribution_dense_rows"] = f"rows {L0 - R}..{L0 - 1} of a {L0}-token sequence"
+    res["attn_distribution_dense_tflops"] = dense_pairs * 2 * H * 576 / (res["attn_distribution_dense_ms"] * 1e-3) / 1e12
+    # three fp32 contractions of H_I x d_I per selected (token, key) pair: logits, dq, dk
+    bwd_flops = pairs * H_I * d_I * 2 * 3
+    res["indexer_backward_tflops_fp32"] = bwd_flops / (res["indexer_backward_ms"] * 1e-3) / 1e12
+    # CUDA-core fp32 peak from the unit counts: 148 SMs x 128 FP32 lanes x 2 flops x 1.965 GHz
+    res["indexer_backward_frac_of_fp32_alu"] = res["indexer_backward_tflops_fp32"] / 74.4
+    assert dsa.dsa_device_error() == 0
+    del pd, dw, dq, dkey, grad, lse
     torch.cuda.empty_cache()
     return res
 

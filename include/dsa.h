@@ -311,6 +311,42 @@ dsa_status dsa_indexer_kl(const float* p, const float* scores, const int32_t* id
                           float* loss, float* grad, void* stream);
 
 /*
+ * Dense warm-up target and the indexer backward (the two training stages of the indexer:
+ * "DeepSeek-V3.2 论文解读", section 二, subsection "两阶段继续预训练" -- a dense warm-up in
+ * which attention stays dense and only the indexer learns, by a KL loss towards the main
+ * attention's distribution, then sparse training in which the indexer, its input detached,
+ * still learns from the KL loss alone).
+ *   dsa_attn_distribution_dense: for packed query tokens r in [row_begin, row_end) (position t
+ *     in a sequence of the contiguous latent, cu_seqlens), p_out[(r-row_begin)*ld_p + s] =
+ *     (1/H) sum_h exp(sm_scale * q[r,h,:] . c[s,:] - lse[r,h]) for s <= t and 0 for
+ *     t < s < ld_p: the head-averaged attention distribution over the whole causal prefix.
+ *     q [T, H, 576] bf16, lse [T, H] fp32 natural log of a dense causal attention over the
+ *     prefix (dsa_masked_mla_prefill writes it), ld_p >= latent->max_seqlen; 1 <= H <= 128.
+ *     With p_out, the KL loss and its gradient of the dense stage are dsa_indexer_kl over rows
+ *     of ld_p entries whose idx lists the prefix positions (-1 beyond).
+ *   dsa_indexer_backward: given grad[t*k + i] = d loss / d I[t, idx[t*k + i]] (idx -1 padded,
+ *     as dsa_indexer_kl writes it), writes the gradients of the indexer's inputs, taken with
+ *     respect to the dequantised operands q_I = e4m3(q_fp8) * q_scale and k_I = e4m3(k8) *
+ *     k_scale, through the ReLU (derivative 0 at 0), in fp32:
+ *       dw [T, H_I]:      dw[t,j] = sum_i g_i ReLU(a_j(s_i)),   a_j(s) = q_I[t,j,:] . k_I[s,:]
+ *       dq [T, H_I, d_I]: dq[t,j,:] = sum_i g_i w[t,j] [a_j(s_i) > 0] k_I[s_i,:]
+ *       dk [T, d_I]:      dk[s,:] = sum over (t, i) with idx = s of g_i sum_j w[t,j] [a_j(s) > 0] q_I[t,j,:]
+ *     keys contiguous (cu_seqlens, total_tokens T; queries are the packed tokens); dk is zeroed
+ *     by the call and accumulated with atomic adds (summation order, and so the last bits,
+ *     vary between runs).  Entries outside their sequence (other than -1) are skipped and set
+ *     DSA_ERR_DEVICE_CHECK.  H_I in {4, 64}, d_I in {64, 128}.
+ * Device pointers, caller-owned outputs, asynchronous on `stream`; DSA_ERR_INVALID_ARGUMENT for
+ * NULL / misaligned pointers or ranges outside the arrays, DSA_ERR_UNSUPPORTED outside the
+ * stated shapes.
+ */
+dsa_status dsa_attn_distribution_dense(const void* q, const dsa_kv_desc* latent, const float* lse, int32_t B,
+                                       int32_t H, int64_t row_begin, int64_t row_end, float sm_scale, float* p_out,
+                                       int64_t ld_p, void* stream);
+dsa_status dsa_indexer_backward(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
+                                const dsa_kv_desc* keys, int32_t B, int32_t H_I, int32_t d_I, const int32_t* idx,
+                                const float* grad, int32_t k, float* dw, float* dq, float* dk, void* stream);
+
+/*
  * Self-test of failure detection (no counterpart on the pages): launches a kernel that waits on
  * a barrier nothing completes, with the same bounded-wait scheme as every pipeline wait of this
  * library but a limit of limit_us microseconds (1 .. 2000000); the kernel then records

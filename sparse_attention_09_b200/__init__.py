@@ -36,7 +36,7 @@ EXPORTED = ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_ml
             "dsa_sparse_mla_decode_noalloc", "dsa_quantize_fp8", "dsa_masked_mla_prefill",
             "dsa_indexer_topk_rows", "dsa_sparse_mla_prefill_rows", "dsa_attn_distribution", "dsa_indexer_kl",
             "dsa_selftest_wait_timeout", "dsa_row_partition", "dsa_indexer_topk_decode",
-            "dsa_decode_select_workspace_size")
+            "dsa_decode_select_workspace_size", "dsa_attn_distribution_dense", "dsa_indexer_backward")
 
 
 class KVDesc(ctypes.Structure):
@@ -103,6 +103,10 @@ _lib.dsa_indexer_topk_decode.argtypes = [_P, _P, _I32, _P, _DESC, _I32, _I32, _I
 _lib.dsa_indexer_topk_decode.restype = _I32
 _lib.dsa_decode_select_workspace_size.argtypes = [_I32, _I32]
 _lib.dsa_decode_select_workspace_size.restype = _SZ
+_lib.dsa_attn_distribution_dense.argtypes = [_P, _DESC, _P, _I32, _I32, _I64, _I64, _F32, _P, _I64, _P]
+_lib.dsa_attn_distribution_dense.restype = _I32
+_lib.dsa_indexer_backward.argtypes = [_P, _P, _I32, _P, _DESC, _I32, _I32, _I32, _P, _P, _I32, _P, _P, _P, _P]
+_lib.dsa_indexer_backward.restype = _I32
 
 
 class DSAError(RuntimeError):
@@ -266,6 +270,23 @@ def dsa_forward(mode, q_fp8, q_scale, w, keys: Desc, q, latent: Desc, B, H_I, d_
 
 def dsa_workspace_size(mode, B, total_tokens, max_ctx, H, k) -> int:
     return int(_lib.dsa_workspace_size(int(mode), int(B), int(total_tokens), int(max_ctx), int(H), int(k)))
+
+
+def dsa_attn_distribution_dense(q, latent: Desc, lse, B, H, row_begin, row_end, sm_scale, p_out, stream=None):
+    """p_out [row_end - row_begin, ld]: head-averaged attention over each row's causal prefix."""
+    _check(_lib.dsa_attn_distribution_dense(_ptr(q), latent.ref(), _ptr(lse), int(B), int(H), int(row_begin),
+                                            int(row_end), float(sm_scale), _ptr(p_out), p_out.stride(0),
+                                            _stream(stream)), "dsa_attn_distribution_dense")
+    return p_out
+
+
+def dsa_indexer_backward(q_fp8, q_scale, w, keys: Desc, B, H_I, d_I, idx, grad, dw, dq, dk, stream=None):
+    """Gradients of the indexer's inputs (dw [T, H_I], dq [T, H_I, d_I], dk [T, d_I], fp32) from
+    d loss / d I on each token's entries (idx / grad [T, k])."""
+    _check(_lib.dsa_indexer_backward(_ptr(q_fp8), _ptr(q_scale), _q_scale_heads(q_scale, H_I), _ptr(w), keys.ref(),
+                                     int(B), int(H_I), int(d_I), _ptr(idx), _ptr(grad), idx.shape[1], _ptr(dw),
+                                     _ptr(dq), _ptr(dk), _stream(stream)), "dsa_indexer_backward")
+    return dw, dq, dk
 
 
 def dsa_decode_select_workspace_size(B, max_ctx) -> int:

@@ -4,6 +4,10 @@
 // distribution is aligned to by the KL loss in the sparse training stage ("DeepSeek-V3.2
 // 论文解读", section 二: the indexer is trained with a KL loss towards the main attention).
 //
+// Dense mode (the dense warm-up stage's target): the same over every row of the token's causal
+// prefix, p[t, s] for s <= t (the entries are the prefix positions themselves, no selection
+// list), with lse from a dense (masked) attention forward; p rows hold ld entries, zero past t.
+//
 // One CTA per SM walks tokens.  Per CTA: warps 0-3 turn logits into probabilities and reduce
 // them over heads (thread h = head h = TMEM lane h), warps 4-5 gather the selected latent rows
 // (all 576 dims, cp.async into 9 blocks of 64 dims with the 128-byte swizzle), warp 6 issues
@@ -17,14 +21,16 @@
 namespace dsa {
 
 struct ProbsParams {
-  const __nv_bfloat16* q;     // [rows, H, 576]
-  const int32_t* idx;         // [rows, k]
-  const float* lse;           // [rows, H] natural log
+  const __nv_bfloat16* q;     // [rows, H, 576] (dense: [T, H, 576], packed tokens)
+  const int32_t* idx;         // [rows, k] (sparse mode)
+  const float* lse;           // [rows, H] natural log (dense: [T, H])
   const int32_t* cu_seqlens;  // [B+1]
   int32_t B, H, k;
-  int64_t rows;
+  int64_t rows;               // units: sparse, rows of q / idx / p; dense, tokens row0 .. row0+rows-1
+  int64_t row0;               // dense: packed token of unit 0
+  int64_t ld;                 // dense: entries per row of p
   float scale_log2;           // sm_scale * log2(e)
-  float* p;                   // [rows, k]
+  float* p;                   // [rows, k] (dense: [rows, ld])
 };
 
 namespace probs {
@@ -72,6 +78,7 @@ __device__ __forceinline__ float lane_transpose_sum(float (&v)[32]) {
 }
 }  // namespace probs
 
+template <bool DENSE>
 __global__ void __launch_bounds__(probs::kThreads, 1)
     attn_probs_kernel(const __nv_bfloat16* __restrict__ latent, const ProbsParams p) {
   using namespace dev;
@@ -117,14 +124,32 @@ __global__ void __launch_bounds__(probs::kThreads, 1)
     seq_start = p.cu_seqlens[lo];
     seq_len = p.cu_seqlens[lo + 1] - seq_start;
   };
-  // chunks up to the last valid entry of the row (every role computes the same, warp-wide)
+  // chunks up to the last valid entry of the row (every role computes the same, warp-wide);
+  // dense: up to the token's own position t
   auto unit_chunks = [&](int64_t u) {
-    const int32_t* row = p.idx + u * p.k;
-    int last = -1;
-    for (int j = lane; j < p.k; j += 32)
-      if (row[j] >= 0) last = j;
-    last = __reduce_max_sync(0xffffffffu, last);
-    return last < 0 ? 1 : last / kChunk + 1;
+    if constexpr (DENSE) {
+      int seq_start, seq_len;
+      seq_of(u + p.row0, seq_start, seq_len);
+      return static_cast<int>(u + p.row0 - seq_start) / kChunk + 1;
+    } else {
+      const int32_t* row = p.idx + u * p.k;
+      int last = -1;
+      for (int j = lane; j < p.k; j += 32)
+        if (row[j] >= 0) last = j;
+      last = __reduce_max_sync(0xffffffffu, last);
+      return last < 0 ? 1 : last / kChunk + 1;
+    }
+  };
+  // entry j of a unit's row: its latent row position (and whether it is valid)
+  auto entry = [&](int64_t u, int t, int seq_len, int j, bool& valid) {
+    if constexpr (DENSE) {
+      valid = j <= t;
+      return j;
+    } else {
+      const int v = p.idx[u * p.k + j];
+      valid = v >= 0 && v < seq_len;
+      return v;
+    }
   };
 
   if (warp >= 4 && warp < kMmaWarp) {
@@ -136,9 +161,9 @@ __global__ void __launch_bounds__(probs::kThreads, 1)
     bool ok = true;
     for (int64_t u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
       int seq_start, seq_len;
-      seq_of(u, seq_start, seq_len);
+      seq_of(DENSE ? u + p.row0 : u, seq_start, seq_len);
+      const int t = DENSE ? static_cast<int>(u + p.row0 - seq_start) : 0;
       const int c1 = unit_chunks(u);
-      const int32_t* row = p.idx + u * p.k;
       for (int c = 0; c < c1; ++c, ++g) {
         const int stage = static_cast<int>(g % kStages);
         if (!mbar_wait(&bar_kvempty[stage], ((g / kStages) & 1u) ^ 1u)) {
@@ -146,8 +171,8 @@ __global__ void __launch_bounds__(probs::kThreads, 1)
           ok = false;
           break;
         }
-        const int v = row[c * kChunk + 32 * pw + lane];
-        const bool valid = v >= 0 && v < seq_len;
+        bool valid;
+        const int v = entry(u, t, seq_len, c * kChunk + 32 * pw + lane, valid);
         const int prow = seq_start + (valid ? v : 0);  // masked rows still copy a real row
         const uint32_t st = smem_addr(sKV + stage * kStageBytes);
 #pragma unroll 8
@@ -205,7 +230,7 @@ __global__ void __launch_bounds__(probs::kThreads, 1)
     const int h = tid;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     auto load_q = [&](int64_t u) {
-      const __nv_bfloat16* qr = p.q + (u * p.H + h) * 576;
+      const __nv_bfloat16* qr = p.q + ((DENSE ? u + p.row0 : u) * p.H + h) * 576;
       const bool real = h < p.H;
 #pragma unroll 1
       for (int c0 = 0; c0 < 288; c0 += 48) {
@@ -233,15 +258,19 @@ __global__ void __launch_bounds__(probs::kThreads, 1)
     for (int64_t u = blockIdx.x; u < nunits; u += gridDim.x) {
       const int c1 = unit_chunks(u);
       int seq_start, seq_len;
-      seq_of(u, seq_start, seq_len);
-      const float lse2 = h < p.H ? p.lse[u * p.H + h] * 1.4426950408889634f : INFINITY;
-      const int32_t* irow = p.idx + u * p.k;
-      float* prow = p.p + u * p.k;
+      const int64_t gq = DENSE ? u + p.row0 : u;  // row of q and lse
+      seq_of(gq, seq_start, seq_len);
+      const int t = DENSE ? static_cast<int>(gq - seq_start) : 0;
+      const float lse2 = h < p.H ? p.lse[gq * p.H + h] * 1.4426950408889634f : INFINITY;
+      const int64_t row_len = DENSE ? p.ld : p.k;
+      float* prow = p.p + u * row_len;
       for (int c = 0; c < c1; ++c, ++g) {
         const int b = static_cast<int>(g & 1u);
         // which of the chunk's 64 entries are valid: read here from the selection row (every
         // warp the same), so the mask needs no hand-over from the gather warps
-        const int e0 = irow[c * kChunk + lane], e1 = irow[c * kChunk + 32 + lane];
+        bool v0, v1;
+        entry(u, t, seq_len, c * kChunk + lane, v0);
+        entry(u, t, seq_len, c * kChunk + 32 + lane, v1);
         bool ok = mbar_wait(&bar_sfull[b], (g >> 1) & 1u);
         if (sm_any(!ok)) {
           aborted = true;
@@ -253,8 +282,8 @@ __global__ void __launch_bounds__(probs::kThreads, 1)
         tmem_ld32(lane_base + kColS + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
         tmem_wait_ld();
         reg_fence(sr);
-        const uint64_t vmask = static_cast<uint64_t>(__ballot_sync(0xffffffffu, e0 >= 0 && e0 < seq_len)) |
-                               (static_cast<uint64_t>(__ballot_sync(0xffffffffu, e1 >= 0 && e1 < seq_len)) << 32);
+        const uint64_t vmask = static_cast<uint64_t>(__ballot_sync(0xffffffffu, v0)) |
+                               (static_cast<uint64_t>(__ballot_sync(0xffffffffu, v1)) << 32);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_sfree[b]);
@@ -274,13 +303,13 @@ __global__ void __launch_bounds__(probs::kThreads, 1)
         s_red[g & 1u][warp][lane] = half[0];
         s_red[g & 1u][warp][32 + lane] = half[1];
         sm_sync();
-        if (tid < kChunk) {
+        if (tid < kChunk && c * kChunk + tid < row_len) {  // a dense row may end inside the chunk
           const float s = (s_red[g & 1u][0][tid] + s_red[g & 1u][1][tid]) + (s_red[g & 1u][2][tid] + s_red[g & 1u][3][tid]);
           prow[c * kChunk + tid] = s * inv_h;
         }
       }
       if (aborted) break;
-      for (int j = c1 * kChunk + tid; j < p.k; j += 128) prow[j] = 0.f;  // past the last valid entry
+      for (int64_t j = c1 * kChunk + tid; j < row_len; j += 128) prow[j] = 0.f;  // past the last valid entry
     }
     if (aborted) record_device_error(DSA_ERR_TIMEOUT);
   }

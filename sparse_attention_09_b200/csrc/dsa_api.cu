@@ -14,6 +14,7 @@
 #include "indexer.cuh"
 #include "quantize.cuh"
 #include "attn_probs.cuh"
+#include "indexer_bwd.cuh"
 #include "indexer_kl.cuh"
 #include "selftest.cuh"
 #include "sparse_mla.cuh"
@@ -291,12 +292,90 @@ dsa_status dsa_attn_distribution(const void* q, const dsa_kv_desc* latent, const
   p.scale_log2 = sm_scale * 1.4426950408889634f;
   p.p = p_out;
   const int smem = probs::kSmemBytes + 1024;
-  if (cudaFuncSetAttribute(attn_probs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(attn_probs_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return DSA_ERR_CUDA;
   const int64_t grid = p.rows < 148 ? p.rows : 148;
-  attn_probs_kernel<<<static_cast<unsigned>(grid), probs::kThreads, smem, as_stream(stream)>>>(
+  attn_probs_kernel<false><<<static_cast<unsigned>(grid), probs::kThreads, smem, as_stream(stream)>>>(
       static_cast<const __nv_bfloat16*>(latent->data), p);
   return launch_status();
+}
+
+dsa_status dsa_attn_distribution_dense(const void* q, const dsa_kv_desc* latent, const float* lse, int32_t B,
+                                       int32_t H, int64_t row_begin, int64_t row_end, float sm_scale, float* p_out,
+                                       int64_t ld_p, void* stream) {
+  if (latent == nullptr || row_begin < 0 || row_end < row_begin) return DSA_ERR_INVALID_ARGUMENT;
+  if (row_end == row_begin) return DSA_OK;
+  if (q == nullptr || latent->data == nullptr || lse == nullptr || p_out == nullptr || B <= 0)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (latent->kind != DSA_KV_CONTIGUOUS || latent->cu_seqlens == nullptr || latent->total_tokens <= 0)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (row_end > latent->total_tokens || ld_p < latent->max_seqlen) return DSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(latent->data, 16)) return DSA_ERR_INVALID_ARGUMENT;
+  if (H < 1 || H > 128) return DSA_ERR_UNSUPPORTED;
+  ProbsParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.lse = lse;
+  p.cu_seqlens = latent->cu_seqlens;
+  p.B = B;
+  p.H = H;
+  p.rows = row_end - row_begin;
+  p.row0 = row_begin;
+  p.ld = ld_p;
+  p.scale_log2 = sm_scale * 1.4426950408889634f;
+  p.p = p_out;
+  const int smem = probs::kSmemBytes + 1024;
+  if (cudaFuncSetAttribute(attn_probs_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  const int64_t grid = p.rows < 148 ? p.rows : 148;
+  attn_probs_kernel<true><<<static_cast<unsigned>(grid), probs::kThreads, smem, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(latent->data), p);
+  return launch_status();
+}
+
+dsa_status dsa_indexer_backward(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
+                                const dsa_kv_desc* keys, int32_t B, int32_t H_I, int32_t d_I, const int32_t* idx,
+                                const float* grad, int32_t k, float* dw, float* dq, float* dk, void* stream) {
+  if (keys == nullptr || k <= 0 || B <= 0) return DSA_ERR_INVALID_ARGUMENT;
+  if (keys->kind != DSA_KV_CONTIGUOUS) return DSA_ERR_UNSUPPORTED;
+  if (q_fp8 == nullptr || q_scale == nullptr || w == nullptr || keys->data == nullptr || keys->scale == nullptr ||
+      keys->cu_seqlens == nullptr || keys->total_tokens <= 0 || idx == nullptr || grad == nullptr || dw == nullptr ||
+      dq == nullptr || dk == nullptr)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (q_scale_heads != 1 && q_scale_heads != H_I) return DSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(keys->data, 4) || !aligned(dk, 16)) return DSA_ERR_INVALID_ARGUMENT;
+  if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED;
+  IdxBwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q8 = q_fp8;
+  p.q_scale = q_scale;
+  p.q_scale_heads = q_scale_heads;
+  p.w = w;
+  p.k8 = static_cast<const uint8_t*>(keys->data);
+  p.k_scale = keys->scale;
+  p.cu_seqlens = keys->cu_seqlens;
+  p.B = B;
+  p.idx = idx;
+  p.grad = grad;
+  p.k = k;
+  p.rows = keys->total_tokens;
+  p.dw = dw;
+  p.dq = dq;
+  p.dk = dk;
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemsetAsync(dk, 0, static_cast<size_t>(keys->total_tokens) * d_I * sizeof(float), s) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  auto launch = [&](auto kern, int smem) -> dsa_status {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    const int64_t grid = p.rows < 2 * 148 ? p.rows : 2 * 148;
+    kern<<<static_cast<unsigned>(grid), ibwd::kThreads, smem, s>>>(p);
+    return launch_status();
+  };
+  if (H_I == 64 && d_I == 128) return launch(indexer_backward_kernel<64, 128>, ibwd::Layout<64, 128>::kSmemBytes);
+  if (H_I == 64 && d_I == 64) return launch(indexer_backward_kernel<64, 64>, ibwd::Layout<64, 64>::kSmemBytes);
+  if (H_I == 4 && d_I == 128) return launch(indexer_backward_kernel<4, 128>, ibwd::Layout<4, 128>::kSmemBytes);
+  return launch(indexer_backward_kernel<4, 64>, ibwd::Layout<4, 64>::kSmemBytes);
 }
 
 dsa_status dsa_indexer_kl(const float* p, const float* scores, const int32_t* idx, int64_t rows, int32_t k,

@@ -99,15 +99,28 @@ struct CandSource {
   }
 };
 
-// The radix select and ordered emission over the C CTAs of a cluster, each holding the
-// entries [src.begin, src.end) of the row (CTA c's entries precede CTA c+1's in index order).
-// Every CTA of the cluster calls it with the same k; it ends with a cluster barrier, so no CTA
-// leaves while a peer may still read its shared memory.
-template <class Src>
+// Barrier over the C CTAs that share a row (C = 1: the CTA alone).
+template <int C>
+__device__ __forceinline__ void row_sync() {
+  if constexpr (C == 1) __syncthreads();
+  else dev::cluster_sync();
+}
+
+// A shared-memory word of CTA c of the row's cluster (C = 1: this CTA's own).
+template <int C>
+__device__ __forceinline__ uint32_t row_ld(const uint32_t* local, int c) {
+  if constexpr (C == 1) return *reinterpret_cast<const volatile uint32_t*>(local);
+  else return ld_cluster_u32(dev::map_to_rank(dev::smem_addr(local), static_cast<uint32_t>(c)));
+}
+
+// The radix select and ordered emission over the C CTAs of a cluster (or one CTA, C = 1), each
+// holding the entries [src.begin, src.end) of the row (CTA c's entries precede CTA c+1's in
+// index order).  Every CTA of the cluster calls it with the same k; it ends with a barrier over
+// the C CTAs, so no CTA leaves while a peer may still read its shared memory.
+template <int C, class Src>
 __device__ void radix_select_emit(const Src& src, int k, int32_t* __restrict__ out, Shared& sh) {
-  constexpr int C = kTopkCluster;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t rank = dev::cluster_ctarank();
+  const uint32_t rank = C == 1 ? 0u : dev::cluster_ctarank();
   uint32_t prefix = 0, mask = 0, remaining = static_cast<uint32_t>(k);
   if (tid == 0) sh.s_above = 0u;  // this segment's entries known to be above the threshold
 #pragma unroll 1
@@ -134,12 +147,11 @@ __device__ void radix_select_emit(const Src& src, int k, int32_t* __restrict__ o
       for (int w = 0; w < kTopkWarps; ++w) s += sh.hist[w][tid];
       sh.total[pass & 1][tid] = s;
     }
-    dev::cluster_sync();  // every CTA's histogram of this pass is complete
+    row_sync<C>();  // every CTA's histogram of this pass is complete
     if (tid < 256) {
-      const uint32_t a = dev::smem_addr(&sh.total[pass & 1][tid]);
       uint32_t s = 0;
 #pragma unroll
-      for (int c = 0; c < C; ++c) s += ld_cluster_u32(dev::map_to_rank(a, c));
+      for (int c = 0; c < C; ++c) s += row_ld<C>(&sh.total[pass & 1][tid], c);
       sh.gtotal[tid] = s;
     }
     __syncthreads();
@@ -177,13 +189,13 @@ __device__ void radix_select_emit(const Src& src, int k, int32_t* __restrict__ o
     __syncthreads();
   }
   if (tid == 0) sh.s_cnt[0] = sh.s_above;
-  dev::cluster_sync();  // the segment counts are published
+  row_sync<C>();  // the segment counts are published
   // this CTA's output offset and tie quota from the segments before it
   const int need_eq = static_cast<int>(remaining);
   int offset = 0, ties_before = 0;
   for (int c = 0; c < static_cast<int>(rank); ++c) {
-    const int g = static_cast<int>(ld_cluster_u32(dev::map_to_rank(dev::smem_addr(&sh.s_cnt[0]), c)));
-    const int e = static_cast<int>(ld_cluster_u32(dev::map_to_rank(dev::smem_addr(&sh.s_cnt[1]), c)));
+    const int g = static_cast<int>(row_ld<C>(&sh.s_cnt[0], c));
+    const int e = static_cast<int>(row_ld<C>(&sh.s_cnt[1], c));
     offset += g + min(e, max(0, need_eq - ties_before));
     ties_before += e;
   }
@@ -226,7 +238,7 @@ __device__ void radix_select_emit(const Src& src, int k, int32_t* __restrict__ o
     eq_taken += tie_total;
     out_pos += sel_total;
   }
-  dev::cluster_sync();  // no CTA leaves while a peer may still read its shared memory
+  row_sync<C>();  // no CTA leaves while a peer may still read its shared memory
 }
 
 // Row length check shared by the kernels: a length outside [0, cap] is an input error; the
@@ -259,86 +271,105 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
   }
   const int per = ((n + C - 1) / C + 15) / 16 * 16;
   const int seg0 = min(n, static_cast<int>(rank) * per), seg1 = min(n, seg0 + per);
-  topk_detail::radix_select_emit(topk_detail::RowSource{scores + r * ld, seg0, seg1, true}, k, out, sh);
+  topk_detail::radix_select_emit<C>(topk_detail::RowSource{scores + r * ld, seg0, seg1, true}, k, out, sh);
 }
 
 // ---- decode selection ------------------------------------------------------------------------
-constexpr int kSelGroup = 16;     // scores per group maximum (written by the paged indexer)
-constexpr int kSelCap = 8192;     // candidates a CTA holds (key + index: 64 KB of shared memory)
-constexpr int kSelBins = 2048;    // 11-bit digits for the bound on the group maxima
+constexpr int kSelGroup = 16;       // scores per group maximum (written by the paged indexer)
+constexpr int kSelCap = 8192;       // candidates of a row (key + index: 64 KB of shared memory)
+constexpr int kSelBits = 12;        // digit of the one-pass bound on the group maxima
+constexpr int kSelBins = 1 << kSelBits;
+constexpr int kSelPerThread = 32;   // scores a thread filters per step
 constexpr int kSelSmemBytes = kSelCap * 8;
 
 namespace topk_detail {
 
-// tau <= the k-th largest of the G group maxima gm[0..G): the 22-bit prefix of that maximum
-// with the low 10 bits cleared (two 11-bit histogram passes).  Every thread of the CTA calls it;
-// `hist` holds kSelBins counters.
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// tau <= the k-th largest of the G group maxima gm[0..G): the top 12 bits of that maximum,
+// low bits cleared (one histogram pass).  Every thread of the CTA calls it; `hist` holds
+// kSelBins counters.
 __device__ uint32_t group_max_bound(const uint32_t* __restrict__ gm, int G, int k, uint32_t* hist, Shared& sh) {
+  constexpr int shift = 32 - kSelBits;
   const int tid = threadIdx.x, lane = tid & 31;
-  uint32_t prefix = 0, mask = 0, remaining = static_cast<uint32_t>(k);
+  for (int i = tid; i < kSelBins; i += kTopkThreads) hist[i] = 0u;
+  __syncthreads();
+  // 4 x 4 maxima per thread per step, every load of a step issued before the first use
+  constexpr int V = 4;
 #pragma unroll 1
-  for (int pass = 0; pass < 2; ++pass) {
-    const int shift = 21 - 11 * pass;
-    for (int i = tid; i < kSelBins; i += kTopkThreads) hist[i] = 0u;
-    __syncthreads();
-#pragma unroll 1
-    for (int base = 0; base < G; base += 4 * kTopkThreads) {
-      const int i = base + 4 * tid;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  for (int base = 0; base < G; base += 4 * V * kTopkThreads) {
+    uint32_t vv[4 * V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const int i = base + 4 * (v * kTopkThreads + tid);
+      uint4 x = make_uint4(0u, 0u, 0u, 0u);
       if (i + 3 < G) {
-        v = *reinterpret_cast<const uint4*>(gm + i);
+        x = *reinterpret_cast<const uint4*>(gm + i);
       } else if (i < G) {
-        v.x = gm[i];
-        if (i + 1 < G) v.y = gm[i + 1];
-        if (i + 2 < G) v.z = gm[i + 2];
+        x.x = gm[i];
+        if (i + 1 < G) x.y = gm[i + 1];
+        if (i + 2 < G) x.z = gm[i + 2];
       }
-      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+      vv[4 * v] = x.x;
+      vv[4 * v + 1] = x.y;
+      vv[4 * v + 2] = x.z;
+      vv[4 * v + 3] = x.w;
+    }
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const bool ok = i + j < G && (vv[j] & mask) == prefix;
-        const uint32_t d = ok ? (vv[j] >> shift) & (kSelBins - 1) : 0xFFFFFFFFu;
+        const bool ok = base + 4 * (v * kTopkThreads + tid) + j < G;
+        const uint32_t d = ok ? vv[4 * v + j] >> shift : 0xFFFFFFFFu;
         // one atomic per distinct digit of the warp: group maxima share few digits
         const uint32_t peers = __match_any_sync(0xffffffffu, d);
         if (ok && (__ffs(peers) - 1) == lane) atomicAdd(&hist[d], static_cast<uint32_t>(__popc(peers)));
       }
     }
-    __syncthreads();
-    // the bin of the remaining-th largest, counting from the top bin (4 bins per thread)
-    constexpr int BPT = kSelBins / kTopkThreads;
-    uint32_t c[BPT], sum = 0;
+  }
+  __syncthreads();
+  // the bin of the k-th largest, counting from the top bin (BPT bins per thread)
+  constexpr int BPT = kSelBins / kTopkThreads;
+  uint32_t c[BPT], sum = 0;
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    c[j] = hist[kSelBins - 1 - (BPT * tid + j)];
+    sum += c[j];
+  }
+  int tot;
+  const uint32_t before =
+      static_cast<uint32_t>(block_exclusive_scan<kTopkWarps>(static_cast<int>(sum), sh.scan_scratch, tot));
+  const uint32_t want = static_cast<uint32_t>(k);
+  if (before < want && want <= before + sum) {
+    uint32_t acc = before;
 #pragma unroll
     for (int j = 0; j < BPT; ++j) {
-      c[j] = hist[kSelBins - 1 - (BPT * tid + j)];
-      sum += c[j];
-    }
-    int tot;
-    const uint32_t before = static_cast<uint32_t>(block_exclusive_scan<kTopkWarps>(static_cast<int>(sum), sh.scan_scratch, tot));
-    if (before < remaining && remaining <= before + sum) {
-      uint32_t acc = before;
-#pragma unroll
-      for (int j = 0; j < BPT; ++j) {
-        if (acc + c[j] >= remaining) {
-          sh.s_bin = static_cast<uint32_t>(kSelBins - 1 - (BPT * tid + j));
-          sh.s_remaining = remaining - acc;
-          break;
-        }
-        acc += c[j];
+      if (acc + c[j] >= want) {
+        sh.s_bin = static_cast<uint32_t>(kSelBins - 1 - (BPT * tid + j));
+        break;
       }
+      acc += c[j];
     }
-    __syncthreads();
-    prefix |= sh.s_bin << shift;
-    mask |= static_cast<uint32_t>(kSelBins - 1) << shift;
-    remaining = sh.s_remaining;
-    __syncthreads();
   }
-  return prefix;
+  __syncthreads();
+  const uint32_t tau = sh.s_bin << shift;
+  __syncthreads();
+  return tau;
 }
 
 }  // namespace topk_detail
 
 // Per-sequence selection after the paged indexer: scores [B, ld] (entries [0, n_b)), gmax
 // [B, ld16] (order key of the largest score of entries [16 g, 16 g + 16) of the row), n_b =
-// min(context_lens[b], max_len).  One cluster of kTopkCluster CTAs per row.
+// min(context_lens[b], max_len).  One cluster of kTopkCluster CTAs per row:
+//   1. every CTA computes tau from the row's group maxima (the same value in each);
+//   2. every CTA filters its quarter of the row: the scores >= tau, in index order, into its
+//      own shared memory;
+//   3. the CTAs publish their counts; unless the row's candidates exceed kSelCap, CTAs 1..3
+//      append theirs to CTA 0's buffer, and CTA 0 alone runs the exact select and emission.
+// With more than kSelCap candidates the cluster runs the full radix select over the row.
 __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThreads)
     topk_decode_select_kernel(const float* __restrict__ scores, int64_t ld, const uint32_t* __restrict__ gmax,
                               int64_t ld16, const int32_t* __restrict__ context_lens, int32_t max_len, int32_t k,
@@ -348,7 +379,7 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
   uint32_t* cand_key = reinterpret_cast<uint32_t*>(sel_smem);
   int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_key + kSelCap);
   __shared__ topk_detail::Shared sh;
-  __shared__ int s_count;
+  __shared__ uint32_t s_count;
   const int tid = threadIdx.x;
   const uint32_t rank = dev::cluster_ctarank();
   const int64_t r = blockIdx.x / C;
@@ -362,34 +393,41 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
   }
   const float* row = scores + r * ld;
   const int G = (n + kSelGroup - 1) / kSelGroup;
-  // with fewer groups than k the maxima bound nothing: every score is a candidate
+  // 1. with fewer groups than k the maxima bound nothing: every score is a candidate
   const uint32_t tau = G >= k ? topk_detail::group_max_bound(gmax + r * ld16, G, k, &sh.hist[0][0], sh) : 0u;
 
-  // one pass over this CTA's segment: the scores >= tau, in index order
+  // 2. this CTA's segment: the scores >= tau, in index order (kSelPerThread consecutive
+  // scores per thread per step)
   const int per = ((n + C - 1) / C + 15) / 16 * 16;
   const int seg0 = min(n, static_cast<int>(rank) * per), seg1 = min(n, seg0 + per);
   int count = 0;
 #pragma unroll 1
-  for (int base = seg0; base < seg1 && count <= kSelCap; base += kTopkTile) {
-    const int i0 = base + 16 * tid;
-    uint32_t keep = 0u, key[16];
-    if (i0 < seg1) {
-      float f[16];
-      topk_load16(row, i0, seg1, f);
+  for (int base = seg0; base < seg1 && count <= kSelCap; base += kSelPerThread * kTopkThreads) {
+    const int i0 = base + kSelPerThread * tid;
+    float f[kSelPerThread];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (i0 + j < seg1 && is_nan_bits(__float_as_uint(f[j]))) record_device_error(DSA_ERR_DEVICE_CHECK);
-        key[j] = order_key(f[j]);
-        keep |= static_cast<uint32_t>(i0 + j < seg1 && key[j] >= tau) << j;
-      }
+    for (int v = 0; v < kSelPerThread / 4; ++v) {
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i0 + 4 * v < seg1) x = *reinterpret_cast<const float4*>(row + i0 + 4 * v);
+      f[4 * v] = x.x;
+      f[4 * v + 1] = x.y;
+      f[4 * v + 2] = x.z;
+      f[4 * v + 3] = x.w;
+    }
+    uint32_t keep = 0u;
+#pragma unroll
+    for (int j = 0; j < kSelPerThread; ++j) {
+      const bool in = i0 + j < seg1;
+      if (in && is_nan_bits(__float_as_uint(f[j]))) record_device_error(DSA_ERR_DEVICE_CHECK);
+      keep |= static_cast<uint32_t>(in && order_key(f[j]) >= tau) << j;
     }
     int total;
     int pos = count + block_exclusive_scan<kTopkWarps>(__popc(keep), sh.scan_scratch, total);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < kSelPerThread; ++j) {
       if ((keep >> j) & 1u) {
         if (pos < kSelCap) {
-          cand_key[pos] = key[j];
+          cand_key[pos] = order_key(f[j]);
           cand_idx[pos] = i0 + j;
         }
         ++pos;
@@ -397,31 +435,37 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
     }
     count += total;
   }
-  // pad to a multiple of 16 entries (the source loads whole 16-entry groups)
-  if (count <= kSelCap) {
-    const int pad_end = min(kSelCap, (count + 15) / 16 * 16);
-    for (int i = count + tid; i < pad_end; i += kTopkThreads) {
-      cand_key[i] = 0u;
-      cand_idx[i] = -1;
-    }
-  }
-  if (tid == 0) s_count = count;
-  __syncthreads();
-  dev::cluster_sync();  // the candidate counts are published
-  int total = 0;
-  bool overflow = false;
+  if (tid == 0) s_count = static_cast<uint32_t>(min(count, kSelCap + 1));
+  dev::cluster_sync();  // 3. the counts are published and every CTA's candidates are written
+  int total = 0, offset = 0;
   for (int c = 0; c < C; ++c) {
     const int cc = static_cast<int>(topk_detail::ld_cluster_u32(dev::map_to_rank(dev::smem_addr(&s_count), c)));
-    total += min(cc, kSelCap + 1);
-    overflow |= cc > kSelCap;
+    if (c < static_cast<int>(rank)) offset += cc;
+    total += cc;
   }
-  if (overflow || total < k) {
-    // too many candidates for the buffers (e.g. a tie class of thousands at the boundary):
-    // the exact select over the row in global memory
-    topk_detail::radix_select_emit(topk_detail::RowSource{row, seg0, seg1, true}, k, out, sh);
-  } else {
-    topk_detail::radix_select_emit(topk_detail::CandSource{cand_key, cand_idx, 0, count}, k, out, sh);
+  if (total > kSelCap || total < k) {
+    // too many candidates for one buffer (e.g. a tie class of thousands at the boundary):
+    // the exact select over the row in global memory, on the whole cluster
+    topk_detail::radix_select_emit<C>(topk_detail::RowSource{row, seg0, seg1, true}, k, out, sh);
+    return;
   }
+  if (rank != 0) {  // append this CTA's candidates to CTA 0's buffer, after those of CTAs < rank
+    const uint32_t kdst = dev::map_to_rank(dev::smem_addr(cand_key), 0u);
+    const uint32_t idst = dev::map_to_rank(dev::smem_addr(cand_idx), 0u);
+    for (int i = tid; i < count; i += kTopkThreads) {
+      topk_detail::st_cluster_u32(kdst + 4u * static_cast<uint32_t>(offset + i), cand_key[i]);
+      topk_detail::st_cluster_u32(idst + 4u * static_cast<uint32_t>(offset + i), static_cast<uint32_t>(cand_idx[i]));
+    }
+  }
+  dev::cluster_sync();  // CTA 0 holds the row's candidates; the others are done
+  if (rank != 0) return;
+  // pad to a multiple of 16 entries (the source loads whole 16-entry groups)
+  for (int i = total + tid; i < min(kSelCap, (total + 15) / 16 * 16); i += kTopkThreads) {
+    cand_key[i] = 0u;
+    cand_idx[i] = -1;
+  }
+  __syncthreads();
+  topk_detail::radix_select_emit<1>(topk_detail::CandSource{cand_key, cand_idx, 0, total}, k, out, sh);
 }
 
 }  // namespace dsa
