@@ -336,8 +336,8 @@ dsa_status dsa_indexer_kl(const float* p, const float* scores, const int32_t* id
  *     vary between runs).  Entries outside their sequence (other than -1) are skipped and set
  *     DSA_ERR_DEVICE_CHECK.  H_I in {4, 64}, d_I in {64, 128}.
  * Device pointers, caller-owned outputs, asynchronous on `stream`; DSA_ERR_INVALID_ARGUMENT for
- * NULL / misaligned pointers or ranges outside the arrays, DSA_ERR_UNSUPPORTED outside the
- * stated shapes.
+ * NULL / misaligned pointers (dq and dk 16-byte aligned) or ranges outside the arrays,
+ * DSA_ERR_UNSUPPORTED outside the stated shapes.
  */
 dsa_status dsa_attn_distribution_dense(const void* q, const dsa_kv_desc* latent, const float* lse, int32_t B,
                                        int32_t H, int64_t row_begin, int64_t row_end, float sm_scale, float* p_out,

@@ -343,7 +343,7 @@ dsa_status dsa_indexer_backward(const uint8_t* q_fp8, const float* q_scale, int3
       dq == nullptr || dk == nullptr)
     return DSA_ERR_INVALID_ARGUMENT;
   if (q_scale_heads != 1 && q_scale_heads != H_I) return DSA_ERR_INVALID_ARGUMENT;
-  if (!aligned(keys->data, 4) || !aligned(dk, 16)) return DSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(keys->data, 4) || !aligned(dk, 16) || !aligned(dq, 16)) return DSA_ERR_INVALID_ARGUMENT;
   if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED;
   IdxBwdParams p;
   std::memset(&p, 0, sizeof(p));
@@ -372,8 +372,8 @@ dsa_status dsa_indexer_backward(const uint8_t* q_fp8, const float* q_scale, int3
     kern<<<static_cast<unsigned>(grid), ibwd::kThreads, smem, s>>>(p);
     return launch_status();
   };
-  if (H_I == 64 && d_I == 128) return launch(indexer_backward_kernel<64, 128>, ibwd::Layout<64, 128>::kSmemBytes);
-  if (H_I == 64 && d_I == 64) return launch(indexer_backward_kernel<64, 64>, ibwd::Layout<64, 64>::kSmemBytes);
+  if (H_I == 64 && d_I == 128) return launch(indexer_backward_h64_kernel<128>, ibwd::Layout64<128>::kSmemBytes);
+  if (H_I == 64 && d_I == 64) return launch(indexer_backward_h64_kernel<64>, ibwd::Layout64<64>::kSmemBytes);
   if (H_I == 4 && d_I == 128) return launch(indexer_backward_kernel<4, 128>, ibwd::Layout<4, 128>::kSmemBytes);
   return launch(indexer_backward_kernel<4, 64>, ibwd::Layout<4, 64>::kSmemBytes);
 }

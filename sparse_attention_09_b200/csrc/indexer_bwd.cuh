@@ -199,4 +199,208 @@ __global__ void __launch_bounds__(ibwd::kThreads) indexer_backward_kernel(const 
   }
 }
 
+// The same computation for 64 heads, register-blocked: every shared-memory load is a 16-byte
+// vector that feeds 8 (phase A) or 16-32 (phases B, C) fused multiply-adds.
+//   A: thread (jb, sb) -> heads 2jb, 2jb+1 and keys sb + 8i (i < 4): 8 logits;
+//   B: thread (jq, dq) -> heads 4jq..4jq+3, dims 4dq + 64c: dq accumulators in registers;
+//   C: thread (sq, dq) -> keys 2sq, 2sq+1, dims 4dq + 64c: the chunk's dk rows.
+// Rows of q_I and k_I are padded by 4 floats, so the 8 lanes that read 8 consecutive key rows
+// (phase A) or heads 2 apart hit distinct banks.
+namespace ibwd {
+template <int D_I>
+struct Layout64 {
+  static constexpr int kQS = D_I + 4, kKS = D_I + 4;
+  static constexpr int kFloats = 64 * kQS + kKC * kKS + 2 * 64 * kKC + 64 + 64 + kKC;
+  static constexpr int kSmemBytes = 4 * kFloats + 4 * kKC;
+};
+
+__device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc) {
+  return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
+}
+}  // namespace ibwd
+
+template <int D_I>
+__global__ void __launch_bounds__(ibwd::kThreads) indexer_backward_h64_kernel(const IdxBwdParams p) {
+  using namespace ibwd;
+  using Lay = Layout64<D_I>;
+  constexpr int H_I = 64, QS = Lay::kQS, KS = Lay::kKS, D4 = D_I / 4, NC = D_I / 64;
+  extern __shared__ __align__(16) float ibwd_smem[];
+  float* sQ = ibwd_smem;                       // [64][QS]
+  float* sK = sQ + 64 * QS;                    // [kKC][KS]
+  float* sM = sK + kKC * KS;                   // [64][kKC]  M[j][s]
+  float* sMT = sM + 64 * kKC;                  // [kKC][64]  M[j][s] transposed
+  float* sW = sMT + kKC * 64;                  // [64]
+  float* sDW = sW + 64;                        // [64]
+  float* sG = sDW + 64;                        // [kKC]
+  int* sV = reinterpret_cast<int*>(sG + kKC);  // [kKC]
+  __shared__ int s_last[kThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int jb = tid >> 3, sb = tid & 7;       // phase A
+  const int jq = tid >> 4, dq4 = tid & 15;     // phase B (and sq = jq in phase C)
+
+  for (int64_t u = blockIdx.x; u < p.rows; u += gridDim.x) {
+    int lo = 0, hi = p.B;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (p.cu_seqlens[mid] <= u) lo = mid;
+      else hi = mid;
+    }
+    const int seq_start = p.cu_seqlens[lo], seq_len = p.cu_seqlens[lo + 1] - seq_start;
+    for (int e = tid; e < H_I * D_I; e += kThreads) {
+      const int j = e / D_I, d = e % D_I;
+      const float sc = p.q_scale[p.q_scale_heads == 1 ? u : u * H_I + j];
+      sQ[j * QS + d] = e4m3_to_f32(p.q8[u * H_I * D_I + e]) * sc;
+    }
+    if (tid < H_I) {
+      sW[tid] = p.w[u * H_I + tid];
+      sDW[tid] = 0.f;
+    }
+    float dq[4][NC][4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+#pragma unroll
+      for (int c = 0; c < NC; ++c)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dq[h][c][e] = 0.f;
+    int last = -1;
+    for (int i = tid; i < p.k; i += kThreads)
+      if (p.idx[u * p.k + i] >= 0) last = i;
+    last = __reduce_max_sync(0xffffffffu, last);
+    if (lane == 0) s_last[warp] = last;
+    __syncthreads();
+    last = -1;
+#pragma unroll
+    for (int i = 0; i < kThreads / 32; ++i) last = max(last, s_last[i]);
+    const int nchunks = (last + kKC) / kKC;
+
+    for (int c0 = 0; c0 < nchunks; ++c0) {
+      if (tid < kKC) {
+        const int i = c0 * kKC + tid;
+        const int v = i < p.k ? p.idx[u * p.k + i] : -1;
+        const bool valid = v >= 0 && v < seq_len;
+        if (!valid && v != -1) record_device_error(DSA_ERR_DEVICE_CHECK);
+        sV[tid] = valid ? seq_start + v : -1;
+        sG[tid] = valid ? p.grad[u * p.k + i] : 0.f;
+      }
+      __syncthreads();
+      for (int e = tid; e < kKC * D4; e += kThreads) {
+        const int s = e / D4, d = 4 * (e % D4);
+        const int row = sV[s];
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (row >= 0) {
+          const uint32_t codes = *reinterpret_cast<const uint32_t*>(p.k8 + static_cast<int64_t>(row) * D_I + d);
+          const float ks = p.k_scale[row];
+          x = make_float4(e4m3_to_f32(static_cast<uint8_t>(codes)) * ks, e4m3_to_f32(static_cast<uint8_t>(codes >> 8)) * ks,
+                          e4m3_to_f32(static_cast<uint8_t>(codes >> 16)) * ks,
+                          e4m3_to_f32(static_cast<uint8_t>(codes >> 24)) * ks);
+        }
+        *reinterpret_cast<float4*>(sK + s * KS + d) = x;
+      }
+      __syncthreads();
+      // (A) logits of heads 2jb, 2jb+1 at keys sb + 8i
+      {
+        float a[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) a[h][i] = 0.f;
+#pragma unroll 4
+        for (int d4 = 0; d4 < D4; ++d4) {
+          const float4 q0 = *reinterpret_cast<const float4*>(sQ + (2 * jb) * QS + 4 * d4);
+          const float4 q1 = *reinterpret_cast<const float4*>(sQ + (2 * jb + 1) * QS + 4 * d4);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 kk = *reinterpret_cast<const float4*>(sK + (sb + 8 * i) * KS + 4 * d4);
+            a[0][i] = dot4(q0, kk, a[0][i]);
+            a[1][i] = dot4(q1, kk, a[1][i]);
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int j = 2 * jb + h;
+          const float wj = sW[j];
+          float part = 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int s = sb + 8 * i;
+            const float gs = sG[s];
+            const float m = a[h][i] > 0.f ? wj * gs : 0.f;
+            sM[j * kKC + s] = m;
+            sMT[s * 64 + j] = m;
+            part = fmaf(fmaxf(a[h][i], 0.f), gs, part);
+          }
+          // the 8 lanes of this head pair (same jb) hold its 32 keys
+          part += __shfl_xor_sync(0xffffffffu, part, 1);
+          part += __shfl_xor_sync(0xffffffffu, part, 2);
+          part += __shfl_xor_sync(0xffffffffu, part, 4);
+          if (sb == 0) sDW[j] += part;
+        }
+      }
+      __syncthreads();
+      // (B) dq[4jq + h, 4dq4 + 64c + e] += sum_s M[j,s] k_I[s, d]
+#pragma unroll 4
+      for (int s = 0; s < kKC; ++s) {
+        const float4 m4 = *reinterpret_cast<const float4*>(sMT + s * 64 + 4 * jq);
+        const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          const float4 kk = *reinterpret_cast<const float4*>(sK + s * KS + 4 * dq4 + 64 * c);
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            dq[h][c][0] = fmaf(mm[h], kk.x, dq[h][c][0]);
+            dq[h][c][1] = fmaf(mm[h], kk.y, dq[h][c][1]);
+            dq[h][c][2] = fmaf(mm[h], kk.z, dq[h][c][2]);
+            dq[h][c][3] = fmaf(mm[h], kk.w, dq[h][c][3]);
+          }
+        }
+      }
+      // (C) dk rows of keys 2jq, 2jq+1: sum_j M[j,s] q_I[j, d]
+      {
+        float acc[2][NC][4];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int c = 0; c < NC; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[r][c][e] = 0.f;
+#pragma unroll 4
+        for (int j = 0; j < H_I; ++j) {
+          const float2 m2 = *reinterpret_cast<const float2*>(sM + j * kKC + 2 * jq);
+#pragma unroll
+          for (int c = 0; c < NC; ++c) {
+            const float4 qq = *reinterpret_cast<const float4*>(sQ + j * QS + 4 * dq4 + 64 * c);
+            acc[0][c][0] = fmaf(m2.x, qq.x, acc[0][c][0]);
+            acc[0][c][1] = fmaf(m2.x, qq.y, acc[0][c][1]);
+            acc[0][c][2] = fmaf(m2.x, qq.z, acc[0][c][2]);
+            acc[0][c][3] = fmaf(m2.x, qq.w, acc[0][c][3]);
+            acc[1][c][0] = fmaf(m2.y, qq.x, acc[1][c][0]);
+            acc[1][c][1] = fmaf(m2.y, qq.y, acc[1][c][1]);
+            acc[1][c][2] = fmaf(m2.y, qq.z, acc[1][c][2]);
+            acc[1][c][3] = fmaf(m2.y, qq.w, acc[1][c][3]);
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int row = sV[2 * jq + r];
+          if (row < 0) continue;
+#pragma unroll
+          for (int c = 0; c < NC; ++c)
+            atomicAdd(reinterpret_cast<float4*>(p.dk + static_cast<int64_t>(row) * D_I + 4 * dq4 + 64 * c),
+                      make_float4(acc[r][c][0], acc[r][c][1], acc[r][c][2], acc[r][c][3]));
+        }
+      }
+      __syncthreads();  // sK, sM, sMT, sV and sG are rewritten by the next chunk
+    }
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+#pragma unroll
+      for (int c = 0; c < NC; ++c)
+        *reinterpret_cast<float4*>(p.dq + (u * H_I + 4 * jq + h) * D_I + 4 * dq4 + 64 * c) =
+            make_float4(dq[h][c][0], dq[h][c][1], dq[h][c][2], dq[h][c][3]);
+    __syncthreads();
+    if (tid < H_I) p.dw[u * H_I + tid] = sDW[tid];
+    __syncthreads();  // sQ, sW and sDW are rewritten by the next token
+  }
+}
+
 }  // namespace dsa

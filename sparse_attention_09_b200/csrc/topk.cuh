@@ -293,7 +293,7 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
 // kSelBins counters.
 __device__ uint32_t group_max_bound(const uint32_t* __restrict__ gm, int G, int k, uint32_t* hist, Shared& sh) {
   constexpr int shift = 32 - kSelBits;
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x;
   for (int i = tid; i < kSelBins; i += kTopkThreads) hist[i] = 0u;
   __syncthreads();
   // 4 x 4 maxima per thread per step, every load of a step issued before the first use
@@ -321,11 +321,9 @@ __device__ uint32_t group_max_bound(const uint32_t* __restrict__ gm, int G, int 
     for (int v = 0; v < V; ++v) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const bool ok = base + 4 * (v * kTopkThreads + tid) + j < G;
-        const uint32_t d = ok ? vv[4 * v + j] >> shift : 0xFFFFFFFFu;
-        // one atomic per distinct digit of the warp: group maxima share few digits
-        const uint32_t peers = __match_any_sync(0xffffffffu, d);
-        if (ok && (__ffs(peers) - 1) == lane) atomicAdd(&hist[d], static_cast<uint32_t>(__popc(peers)));
+        // plain shared-memory increments: warp-aggregating them with __match_any_sync measured
+        // several times slower on B200 than the same-address serialisation it saves
+        if (base + 4 * (v * kTopkThreads + tid) + j < G) atomicAdd(&hist[vv[4 * v + j] >> shift], 1u);
       }
     }
   }

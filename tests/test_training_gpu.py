@@ -193,5 +193,6 @@ def test_indexer_backward_reports_and_skips_entries_outside_the_sequence():
     assert err == dsa.DSA_OK
     got, err = run(bad)
     assert err == dsa.DSA_ERR_DEVICE_CHECK
-    for g, r in zip(got, ref):
-        assert torch.allclose(g, r, rtol=1e-5, atol=1e-6)
+    # dw and dq: the same per-token arithmetic, bit for bit; dk: atomic adds in any order
+    assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1])
+    assert (got[2] - ref[2]).abs().max() <= 1e-5 * ref[2].abs().max()
