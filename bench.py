@@ -386,7 +386,9 @@ def run_profile_case(args, dsa, sm):
                      rows gathered for its 2048 selected entries, as for every row of the run).
       decode_8x128k  8 sequences at contexts drawn from [122880, 131072]: the fused decode
                      selection (paged indexer scan + selection kernel), sparse MLA decode and
-                     the combine.
+                     the combine (8 splits per sequence).
+      decode_64      the bench's decode workload (64 sequences, contexts U[8192, 131072]), the
+                     same calls (one split per sequence: no combine).
       indexer_128k   the whole fused indexer + top-k launch of the L=131072 prefill (the bench's
                      own call and launch shape) with only the indexer's operands on the device
                      (~2.3 GB): its per-launch DRAM bytes need no scaling.
@@ -416,9 +418,12 @@ def run_profile_case(args, dsa, sm):
         torch.cuda.synchronize()
         out.update(rows=R, L=L, indexer_topk_ms=evs[0].elapsed_time(evs[1]),
                    sparse_mla_ms=evs[1].elapsed_time(evs[2]))
-    elif args.profile_case == "decode_8x128k":
-        B = 8
-        d = synth.decode_inputs(B=B, ctx_lo=122880, ctx_hi=131072, H_I=64, d_I=128, H=128, seed=31, device="cuda")
+    elif args.profile_case in ("decode_8x128k", "decode_64"):
+        if args.profile_case == "decode_64":
+            d = synth.decode_inputs(device="cuda", **dict(synth.WORKLOADS[DECODE]))
+        else:
+            d = synth.decode_inputs(B=8, ctx_lo=122880, ctx_hi=131072, H_I=64, d_I=128, H=128, seed=31, device="cuda")
+        B = d["B"]
         keys = dsa.paged_desc(d["kcache8"], d["block_table"], d["ctx"], d["max_ctx"], scale=d["kscale_cache"])
         lat = dsa.paged_desc(d["latent_cache"], d["block_table"], d["ctx"], d["max_ctx"])
         idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
@@ -871,7 +876,8 @@ def main():
     ap.add_argument("--workload", default=PREFILL, choices=[w for w, c in synth.WORKLOADS.items() if c["kind"] == "prefill"],
                     help="prefill workload of the timed step (the headline is prefill_128k; smaller ones are for profiling)")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--profile-case", choices=["rows_128k", "decode_8x128k", "indexer_128k", "mla_quarters_128k"], default=None,
+    ap.add_argument("--profile-case", choices=["rows_128k", "decode_8x128k", "decode_64", "indexer_128k",
+                                                  "mla_quarters_128k"], default=None,
                     help="run one small case of the kernels for a counter capture and exit")
     ap.add_argument("--idx-ms", type=float, default=142.0,
                     help="--strong: measured time of the fused indexer top-k over the whole sequence")

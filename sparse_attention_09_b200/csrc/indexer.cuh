@@ -315,8 +315,8 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
       }
       const bool ok = mbar_wait(&bar_accfull[acc], aph);
       if (!ok) record_device_error(DSA_ERR_TIMEOUT);
-      // top-k mode takes the abort decision at its per-tile group vote below (one barrier per
-      // tile); reading a stale accumulator before it is harmless
+      // top-k mode takes the abort decision at its group vote below (one barrier per two
+      // tiles); reading a stale accumulator before it is harmless
       if (MODE == kIdxScores && sel::gany(G, !ok)) {
         aborted = true;
         break;
@@ -439,9 +439,11 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
             kmax[tt] = max(kmax[tt], key);
           }
           wcnt[tt] += __popc(m);
-          need_cut |= wcnt[tt] > Q - 32;  // the next tile could add 32 more to this region
+          // the group votes after every second tile, and the two tiles after a vote add at most
+          // 64 entries to a region: cut a token when one of its regions holds more than Q - 64
+          need_cut |= wcnt[tt] > Q - 64;
         }
-        if (sel::gany(G, need_cut || !ok)) {
+        if ((it & 1) && sel::gany(G, need_cut || !ok)) {
           if (sel::gany(G, !ok)) {
             aborted = true;
             break;
@@ -454,8 +456,8 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
 #pragma unroll
           for (int tt = 0; tt < TPG; ++tt) {
             const int tok = tg0 + tt;
-            const bool full = s_cnt[tok][0] > Q - 32 || s_cnt[tok][1] > Q - 32 || s_cnt[tok][2] > Q - 32 ||
-                              s_cnt[tok][3] > Q - 32;
+            const bool full = s_cnt[tok][0] > Q - 64 || s_cnt[tok][1] > Q - 64 || s_cnt[tok][2] > Q - 64 ||
+                              s_cnt[tok][3] > Q - 64;
             if (full) {  // uniform over the group
               uint32_t lo, hi;
               sel::group_minmax(G, s_sel[g], kmin[tt], kmax[tt], lo, hi);

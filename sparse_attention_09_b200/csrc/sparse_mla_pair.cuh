@@ -49,8 +49,9 @@
 //     softmax warps, an index ring and a fixed issue order of the two products.
 //
 // The same kernel serves decode: a work item is then (sequence, split of its selection) over a
-// paged latent cache, and the unnormalised partial result (O, M, l) goes to a workspace that a
-// small kernel merges by log-sum-exp.
+// paged latent cache.  A split selection's unnormalised partial results (O, M, l) go to a
+// workspace that a small kernel merges by log-sum-exp; an unsplit one is written as out / lse
+// directly, as in prefill.
 #pragma once
 
 #include "common.cuh"

@@ -277,9 +277,8 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
 // ---- decode selection ------------------------------------------------------------------------
 constexpr int kSelGroup = 16;       // scores per group maximum (written by the paged indexer)
 constexpr int kSelCap = 8192;       // candidates of a row (key + index: 64 KB of shared memory)
-constexpr int kSelBits = 12;        // digit of the one-pass bound on the group maxima
-constexpr int kSelBins = 1 << kSelBits;
-constexpr int kSelPerThread = 32;   // scores a thread filters per step
+constexpr int kSelBuckets = 4096;   // linear buckets over the group maxima's key range
+constexpr int kSelDigit = 11;       // radix digit of the exact select over the candidates
 constexpr int kSelSmemBytes = kSelCap * 8;
 
 namespace topk_detail {
@@ -288,73 +287,170 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-// tau <= the k-th largest of the G group maxima gm[0..G): the top 12 bits of that maximum,
-// low bits cleared (one histogram pass).  Every thread of the CTA calls it; `hist` holds
-// kSelBins counters.
-__device__ uint32_t group_max_bound(const uint32_t* __restrict__ gm, int G, int k, uint32_t* hist, Shared& sh) {
-  constexpr int shift = 32 - kSelBits;
+// Block-wide reductions of one uint32 per thread (every thread receives the result).
+template <class Op>
+__device__ __forceinline__ uint32_t block_reduce_u32(uint32_t v, uint32_t* scratch, Op op) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();  // scratch is free
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  v = scratch[0];
+#pragma unroll
+  for (int w = 1; w < kTopkWarps; ++w) v = op(v, scratch[w]);
+  return v;
+}
+struct MinOp { __device__ uint32_t operator()(uint32_t a, uint32_t b) const { return min(a, b); } };
+struct MaxOp { __device__ uint32_t operator()(uint32_t a, uint32_t b) const { return max(a, b); } };
+struct AndOp { __device__ uint32_t operator()(uint32_t a, uint32_t b) const { return a & b; } };
+struct OrOp { __device__ uint32_t operator()(uint32_t a, uint32_t b) const { return a | b; } };
+
+// Finds, counting from the top bin of hist[0..kBins), the bin where the count reaches `want`;
+// returns it and sets `above` to the count in the bins above it.  Every thread calls it.
+template <int kBins>
+__device__ __forceinline__ int find_bin_from_top(const uint32_t* hist, uint32_t want, uint32_t& above, Shared& sh) {
+  constexpr int BPT = kBins / kTopkThreads;
   const int tid = threadIdx.x;
-  for (int i = tid; i < kSelBins; i += kTopkThreads) hist[i] = 0u;
-  __syncthreads();
-  // 4 x 4 maxima per thread per step, every load of a step issued before the first use
-  constexpr int V = 4;
-#pragma unroll 1
-  for (int base = 0; base < G; base += 4 * V * kTopkThreads) {
-    uint32_t vv[4 * V];
-#pragma unroll
-    for (int v = 0; v < V; ++v) {
-      const int i = base + 4 * (v * kTopkThreads + tid);
-      uint4 x = make_uint4(0u, 0u, 0u, 0u);
-      if (i + 3 < G) {
-        x = *reinterpret_cast<const uint4*>(gm + i);
-      } else if (i < G) {
-        x.x = gm[i];
-        if (i + 1 < G) x.y = gm[i + 1];
-        if (i + 2 < G) x.z = gm[i + 2];
-      }
-      vv[4 * v] = x.x;
-      vv[4 * v + 1] = x.y;
-      vv[4 * v + 2] = x.z;
-      vv[4 * v + 3] = x.w;
-    }
-#pragma unroll
-    for (int v = 0; v < V; ++v) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        // plain shared-memory increments: warp-aggregating them with __match_any_sync measured
-        // several times slower on B200 than the same-address serialisation it saves
-        if (base + 4 * (v * kTopkThreads + tid) + j < G) atomicAdd(&hist[vv[4 * v + j] >> shift], 1u);
-      }
-    }
-  }
-  __syncthreads();
-  // the bin of the k-th largest, counting from the top bin (BPT bins per thread)
-  constexpr int BPT = kSelBins / kTopkThreads;
   uint32_t c[BPT], sum = 0;
 #pragma unroll
   for (int j = 0; j < BPT; ++j) {
-    c[j] = hist[kSelBins - 1 - (BPT * tid + j)];
+    c[j] = hist[kBins - 1 - (BPT * tid + j)];
     sum += c[j];
   }
   int tot;
   const uint32_t before =
       static_cast<uint32_t>(block_exclusive_scan<kTopkWarps>(static_cast<int>(sum), sh.scan_scratch, tot));
-  const uint32_t want = static_cast<uint32_t>(k);
   if (before < want && want <= before + sum) {
     uint32_t acc = before;
 #pragma unroll
     for (int j = 0; j < BPT; ++j) {
       if (acc + c[j] >= want) {
-        sh.s_bin = static_cast<uint32_t>(kSelBins - 1 - (BPT * tid + j));
+        sh.s_bin = static_cast<uint32_t>(kBins - 1 - (BPT * tid + j));
+        sh.s_above = acc;
         break;
       }
       acc += c[j];
     }
   }
   __syncthreads();
-  const uint32_t tau = sh.s_bin << shift;
+  const int bin = static_cast<int>(sh.s_bin);
+  above = sh.s_above;
   __syncthreads();
-  return tau;
+  return bin;
+}
+
+// tau <= the k-th largest of the G group maxima gm[0..G) (G >= k).  The maxima's key range
+// [lo, hi] is mapped linearly onto kSelBuckets buckets (any monotone map keeps the order; a
+// linear one spreads the maxima, which crowd a few exponent bins, over many buckets); tau is
+// the lower edge of the bucket below the one holding the k-th largest, so float rounding of
+// the map cannot put tau above it.  Every thread of the CTA calls it; `hist` holds
+// kSelBuckets counters.
+__device__ uint32_t group_max_bound(const uint32_t* __restrict__ gm, int G, int k, uint32_t* hist, Shared& sh) {
+  const int tid = threadIdx.x;
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int i = tid; i < G; i += kTopkThreads) {
+    const uint32_t v = gm[i];
+    lo = min(lo, v);
+    hi = max(hi, v);
+  }
+  lo = block_reduce_u32(lo, reinterpret_cast<uint32_t*>(sh.scan_scratch), MinOp{});
+  hi = block_reduce_u32(hi, reinterpret_cast<uint32_t*>(sh.scan_scratch), MaxOp{});
+  if (hi == lo) return lo;  // every maximum is equal: all G >= k groups reach it
+  const float inv = static_cast<float>(kSelBuckets) / (static_cast<float>(hi - lo) + 1.f);
+  for (int i = tid; i < kSelBuckets; i += kTopkThreads) hist[i] = 0u;
+  __syncthreads();
+  for (int i = tid; i < G; i += kTopkThreads) {
+    const int b = static_cast<int>(static_cast<float>(gm[i] - lo) * inv);
+    atomicAdd(&hist[b < kSelBuckets ? b : kSelBuckets - 1], 1u);
+  }
+  __syncthreads();
+  uint32_t above;
+  const int b = find_bin_from_top<kSelBuckets>(hist, static_cast<uint32_t>(k), above, sh);
+  const float edge = static_cast<float>(b - 1) / inv;  // one bucket of margin for the rounding
+  return edge <= 0.f ? lo : lo + static_cast<uint32_t>(edge);
+}
+
+}  // namespace topk_detail
+
+namespace topk_detail {
+
+// Exact top-k of the n <= kSelCap candidates (order key, index) that this CTA holds in index
+// order, written ascending to out[0..k) (n >= k).  The k-th largest key comes from radix
+// passes of kSelDigit bits that start below the candidates' common key prefix (the candidates
+// of a row share their leading bits, which would put them all in one bin of a fixed-position
+// digit); ties at it go to the lowest indices.  Every thread of the CTA calls it.
+__device__ void cand_select_emit(const uint32_t* __restrict__ key, const int32_t* __restrict__ idx, int n, int k,
+                                 int32_t* __restrict__ out, uint32_t* hist, Shared& sh) {
+  constexpr int kBins = 1 << kSelDigit;
+  const int tid = threadIdx.x;
+  uint32_t a = 0xFFFFFFFFu, o = 0u;
+  for (int i = tid; i < n; i += kTopkThreads) {
+    a &= key[i];
+    o |= key[i];
+  }
+  a = block_reduce_u32(a, reinterpret_cast<uint32_t*>(sh.scan_scratch), AndOp{});
+  o = block_reduce_u32(o, reinterpret_cast<uint32_t*>(sh.scan_scratch), OrOp{});
+  const int common = (a ^ o) == 0u ? 32 : __clz(a ^ o);  // leading bits every candidate shares
+  uint32_t mask = common == 0 ? 0u : (0xFFFFFFFFu << (32 - common));
+  uint32_t prefix = a & mask;
+  uint32_t rem = static_cast<uint32_t>(k);  // entries still to take at or below the prefix
+  int pos = 32 - common;
+#pragma unroll 1
+  while (pos > 0) {
+    const int d = pos < kSelDigit ? pos : kSelDigit;
+    const int shift = pos - d;
+    const uint32_t dmask = (1u << d) - 1u;
+    for (int i = tid; i < kBins; i += kTopkThreads) hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n; i += kTopkThreads) {
+      const uint32_t kk = key[i];
+      if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & dmask], 1u);
+    }
+    __syncthreads();
+    uint32_t above;
+    const uint32_t bin = static_cast<uint32_t>(find_bin_from_top<kBins>(hist, rem, above, sh));
+    prefix |= bin << shift;
+    mask |= dmask << shift;
+    rem -= above;
+    pos = shift;
+  }
+  // prefix is the k-th largest key; rem of the keys equal to it are taken (the lowest indices)
+  const uint32_t thr = prefix;
+  const int quota = static_cast<int>(rem);
+  int eq_taken = 0, out_pos = 0;
+#pragma unroll 1
+  for (int base = 0; base < n; base += 4 * kTopkThreads) {
+    const int i0 = base + 4 * tid;
+    uint32_t gbits = 0u, ebits = 0u;
+    int32_t ix[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (i0 + j < n) {
+        const uint32_t kk = key[i0 + j];
+        ix[j] = idx[i0 + j];
+        gbits |= static_cast<uint32_t>(kk > thr) << j;
+        ebits |= static_cast<uint32_t>(kk == thr) << j;
+      }
+    }
+    int tie_total;
+    int tie_rank = eq_taken + block_exclusive_scan<kTopkWarps>(__popc(ebits), sh.scan_scratch, tie_total);
+    uint32_t sbits = gbits;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if ((ebits >> j) & 1u) {
+        if (tie_rank < quota) sbits |= 1u << j;
+        ++tie_rank;
+      }
+    }
+    int sel_total;
+    int p = out_pos + block_exclusive_scan<kTopkWarps>(__popc(sbits), sh.scan_scratch, sel_total);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if ((sbits >> j) & 1u) out[p++] = ix[j];
+    eq_taken += tie_total;
+    out_pos += sel_total;
+  }
 }
 
 }  // namespace topk_detail
@@ -363,10 +459,11 @@ __device__ uint32_t group_max_bound(const uint32_t* __restrict__ gm, int G, int 
 // [B, ld16] (order key of the largest score of entries [16 g, 16 g + 16) of the row), n_b =
 // min(context_lens[b], max_len).  One cluster of kTopkCluster CTAs per row:
 //   1. every CTA computes tau from the row's group maxima (the same value in each);
-//   2. every CTA filters its quarter of the row: the scores >= tau, in index order, into its
-//      own shared memory;
-//   3. the CTAs publish their counts; unless the row's candidates exceed kSelCap, CTAs 1..3
-//      append theirs to CTA 0's buffer, and CTA 0 alone runs the exact select and emission.
+//   2. every CTA splits its quarter of the row into 16 warp slices and counts, with coalesced
+//      16-byte loads, the scores >= tau of each slice;
+//   3. the CTAs exchange their counts; unless the row's candidates exceed kSelCap, every warp
+//      reads its slice again and writes its candidates, in index order, straight into CTA 0's
+//      buffer at its offset (distributed shared memory), and CTA 0 alone selects and emits.
 // With more than kSelCap candidates the cluster runs the full radix select over the row.
 __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThreads)
     topk_decode_select_kernel(const float* __restrict__ scores, int64_t ld, const uint32_t* __restrict__ gmax,
@@ -378,7 +475,8 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
   int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_key + kSelCap);
   __shared__ topk_detail::Shared sh;
   __shared__ uint32_t s_count;
-  const int tid = threadIdx.x;
+  __shared__ int s_wcount[kTopkWarps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = dev::cluster_ctarank();
   const int64_t r = blockIdx.x / C;
   int32_t* out = idx + r * static_cast<int64_t>(k);
@@ -394,47 +492,34 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
   // 1. with fewer groups than k the maxima bound nothing: every score is a candidate
   const uint32_t tau = G >= k ? topk_detail::group_max_bound(gmax + r * ld16, G, k, &sh.hist[0][0], sh) : 0u;
 
-  // 2. this CTA's segment: the scores >= tau, in index order (kSelPerThread consecutive
-  // scores per thread per step)
+  // 2. this CTA's segment, in 16 warp slices of whole 128-score steps (a float4 per lane)
   const int per = ((n + C - 1) / C + 15) / 16 * 16;
   const int seg0 = min(n, static_cast<int>(rank) * per), seg1 = min(n, seg0 + per);
-  int count = 0;
-#pragma unroll 1
-  for (int base = seg0; base < seg1 && count <= kSelCap; base += kSelPerThread * kTopkThreads) {
-    const int i0 = base + kSelPerThread * tid;
-    float f[kSelPerThread];
+  const int wlen = ((seg1 - seg0 + kTopkWarps - 1) / kTopkWarps + 127) / 128 * 128;
+  const int w0 = min(seg1, seg0 + warp * wlen), w1 = min(seg1, w0 + wlen);
+  int wcount = 0;
+  for (int i = w0 + 4 * lane; i < w1; i += 128) {
+    const float4 x = *reinterpret_cast<const float4*>(row + i);  // ld >= n, ld % 4 == 0
+    const float f[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-    for (int v = 0; v < kSelPerThread / 4; ++v) {
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (i0 + 4 * v < seg1) x = *reinterpret_cast<const float4*>(row + i0 + 4 * v);
-      f[4 * v] = x.x;
-      f[4 * v + 1] = x.y;
-      f[4 * v + 2] = x.z;
-      f[4 * v + 3] = x.w;
-    }
-    uint32_t keep = 0u;
-#pragma unroll
-    for (int j = 0; j < kSelPerThread; ++j) {
-      const bool in = i0 + j < seg1;
-      if (in && is_nan_bits(__float_as_uint(f[j]))) record_device_error(DSA_ERR_DEVICE_CHECK);
-      keep |= static_cast<uint32_t>(in && order_key(f[j]) >= tau) << j;
-    }
-    int total;
-    int pos = count + block_exclusive_scan<kTopkWarps>(__popc(keep), sh.scan_scratch, total);
-#pragma unroll
-    for (int j = 0; j < kSelPerThread; ++j) {
-      if ((keep >> j) & 1u) {
-        if (pos < kSelCap) {
-          cand_key[pos] = order_key(f[j]);
-          cand_idx[pos] = i0 + j;
-        }
-        ++pos;
+    for (int j = 0; j < 4; ++j) {
+      if (i + j < w1) {
+        if (is_nan_bits(__float_as_uint(f[j]))) record_device_error(DSA_ERR_DEVICE_CHECK);
+        wcount += order_key(f[j]) >= tau ? 1 : 0;
       }
     }
-    count += total;
   }
-  if (tid == 0) s_count = static_cast<uint32_t>(min(count, kSelCap + 1));
-  dev::cluster_sync();  // 3. the counts are published and every CTA's candidates are written
+  wcount = __reduce_add_sync(0xffffffffu, wcount);
+  if (lane == 0) s_wcount[warp] = wcount;
+  __syncthreads();
+  int woff = 0, ccount = 0;
+#pragma unroll
+  for (int w = 0; w < kTopkWarps; ++w) {
+    woff += w < warp ? s_wcount[w] : 0;
+    ccount += s_wcount[w];
+  }
+  if (tid == 0) s_count = static_cast<uint32_t>(ccount);
+  dev::cluster_sync();  // 3. the counts are published
   int total = 0, offset = 0;
   for (int c = 0; c < C; ++c) {
     const int cc = static_cast<int>(topk_detail::ld_cluster_u32(dev::map_to_rank(dev::smem_addr(&s_count), c)));
@@ -444,26 +529,42 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
   if (total > kSelCap || total < k) {
     // too many candidates for one buffer (e.g. a tie class of thousands at the boundary):
     // the exact select over the row in global memory, on the whole cluster
-    topk_detail::radix_select_emit<C>(topk_detail::RowSource{row, seg0, seg1, true}, k, out, sh);
+    topk_detail::radix_select_emit<C>(topk_detail::RowSource{row, seg0, seg1, false}, k, out, sh);
     return;
   }
-  if (rank != 0) {  // append this CTA's candidates to CTA 0's buffer, after those of CTAs < rank
+  {  // this warp's candidates, in index order, into CTA 0's buffer at offset + woff
     const uint32_t kdst = dev::map_to_rank(dev::smem_addr(cand_key), 0u);
     const uint32_t idst = dev::map_to_rank(dev::smem_addr(cand_idx), 0u);
-    for (int i = tid; i < count; i += kTopkThreads) {
-      topk_detail::st_cluster_u32(kdst + 4u * static_cast<uint32_t>(offset + i), cand_key[i]);
-      topk_detail::st_cluster_u32(idst + 4u * static_cast<uint32_t>(offset + i), static_cast<uint32_t>(cand_idx[i]));
+    uint32_t at = static_cast<uint32_t>(offset + woff);
+    for (int i = w0 + 4 * lane; i - 4 * lane < w1; i += 128) {  // whole-warp steps
+      uint32_t kk[4];
+      uint32_t keep = 0u;
+      if (i < w1) {
+        const float4 x = *reinterpret_cast<const float4*>(row + i);
+        kk[0] = order_key(x.x);
+        kk[1] = order_key(x.y);
+        kk[2] = order_key(x.z);
+        kk[3] = order_key(x.w);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) keep |= static_cast<uint32_t>(i + j < w1 && kk[j] >= tau) << j;
+      }
+      const int cnt = __popc(keep);
+      const int incl = warp_inclusive_scan(cnt);
+      uint32_t p = at + static_cast<uint32_t>(incl - cnt);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if ((keep >> j) & 1u) {
+          topk_detail::st_cluster_u32(kdst + 4u * p, kk[j]);
+          topk_detail::st_cluster_u32(idst + 4u * p, static_cast<uint32_t>(i + j));
+          ++p;
+        }
+      }
+      at += static_cast<uint32_t>(__shfl_sync(0xffffffffu, incl, 31));
     }
   }
   dev::cluster_sync();  // CTA 0 holds the row's candidates; the others are done
   if (rank != 0) return;
-  // pad to a multiple of 16 entries (the source loads whole 16-entry groups)
-  for (int i = total + tid; i < min(kSelCap, (total + 15) / 16 * 16); i += kTopkThreads) {
-    cand_key[i] = 0u;
-    cand_idx[i] = -1;
-  }
-  __syncthreads();
-  topk_detail::radix_select_emit<1>(topk_detail::CandSource{cand_key, cand_idx, 0, total}, k, out, sh);
+  topk_detail::cand_select_emit(cand_key, cand_idx, total, k, out, &sh.hist[0][0], sh);
 }
 
 }  // namespace dsa
