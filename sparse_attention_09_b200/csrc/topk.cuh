@@ -279,6 +279,7 @@ constexpr int kSelGroup = 16;       // scores per group maximum (written by the 
 constexpr int kSelCap = 8192;       // candidates of a row (key + index: 64 KB of shared memory)
 constexpr int kSelBuckets = 4096;   // linear buckets over the group maxima's key range
 constexpr int kSelDigit = 11;       // radix digit of the exact select over the candidates
+constexpr int kSelBatch = 8;        // 128-score steps a warp loads before using them
 constexpr int kSelSmemBytes = kSelCap * 8;
 
 namespace topk_detail {
@@ -347,12 +348,43 @@ __device__ __forceinline__ int find_bin_from_top(const uint32_t* hist, uint32_t 
 // the map cannot put tau above it.  Every thread of the CTA calls it; `hist` holds
 // kSelBuckets counters.
 __device__ uint32_t group_max_bound(const uint32_t* __restrict__ gm, int G, int k, uint32_t* hist, Shared& sh) {
+  constexpr int V = 4;  // 16-byte loads per thread per step, all issued before the first use
   const int tid = threadIdx.x;
   uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  for (int i = tid; i < G; i += kTopkThreads) {
-    const uint32_t v = gm[i];
-    lo = min(lo, v);
-    hi = max(hi, v);
+  // every load of a step is issued before any is used; a row of up to 8192 maxima (128K keys)
+  // is one step, held in registers for both uses below
+  uint32_t vv[4 * V];
+  auto load_step = [&](int base) {
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const int i = base + 4 * (v * kTopkThreads + tid);
+      uint4 x = make_uint4(0u, 0u, 0u, 0u);
+      if (i + 3 < G) {
+        x = *reinterpret_cast<const uint4*>(gm + i);
+      } else if (i < G) {
+        x.x = gm[i];
+        if (i + 1 < G) x.y = gm[i + 1];
+        if (i + 2 < G) x.z = gm[i + 2];
+      }
+      vv[4 * v] = x.x;
+      vv[4 * v + 1] = x.y;
+      vv[4 * v + 2] = x.z;
+      vv[4 * v + 3] = x.w;
+    }
+  };
+  auto valid = [&](int base, int v, int j) { return base + 4 * (v * kTopkThreads + tid) + j < G; };
+  constexpr int STEP = 4 * V * kTopkThreads;
+#pragma unroll 1
+  for (int base = 0; base < G; base += STEP) {
+    load_step(base);
+#pragma unroll
+    for (int v = 0; v < V; ++v)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (valid(base, v, j)) {
+          lo = min(lo, vv[4 * v + j]);
+          hi = max(hi, vv[4 * v + j]);
+        }
   }
   lo = block_reduce_u32(lo, reinterpret_cast<uint32_t*>(sh.scan_scratch), MinOp{});
   hi = block_reduce_u32(hi, reinterpret_cast<uint32_t*>(sh.scan_scratch), MaxOp{});
@@ -360,9 +392,17 @@ __device__ uint32_t group_max_bound(const uint32_t* __restrict__ gm, int G, int 
   const float inv = static_cast<float>(kSelBuckets) / (static_cast<float>(hi - lo) + 1.f);
   for (int i = tid; i < kSelBuckets; i += kTopkThreads) hist[i] = 0u;
   __syncthreads();
-  for (int i = tid; i < G; i += kTopkThreads) {
-    const int b = static_cast<int>(static_cast<float>(gm[i] - lo) * inv);
-    atomicAdd(&hist[b < kSelBuckets ? b : kSelBuckets - 1], 1u);
+#pragma unroll 1
+  for (int base = 0; base < G; base += STEP) {
+    if (G > STEP) load_step(base);  // one step: the maxima are still in registers
+#pragma unroll
+    for (int v = 0; v < V; ++v)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (valid(base, v, j)) {
+          const int b = static_cast<int>(static_cast<float>(vv[4 * v + j] - lo) * inv);
+          atomicAdd(&hist[b < kSelBuckets ? b : kSelBuckets - 1], 1u);
+        }
   }
   __syncthreads();
   uint32_t above;
@@ -465,7 +505,7 @@ __device__ void cand_select_emit(const uint32_t* __restrict__ key, const int32_t
 //      reads its slice again and writes its candidates, in index order, straight into CTA 0's
 //      buffer at its offset (distributed shared memory), and CTA 0 alone selects and emits.
 // With more than kSelCap candidates the cluster runs the full radix select over the row.
-__global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThreads)
+__global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThreads, 2)
     topk_decode_select_kernel(const float* __restrict__ scores, int64_t ld, const uint32_t* __restrict__ gmax,
                               int64_t ld16, const int32_t* __restrict__ context_lens, int32_t max_len, int32_t k,
                               int32_t* __restrict__ idx) {
@@ -497,15 +537,27 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
   const int seg0 = min(n, static_cast<int>(rank) * per), seg1 = min(n, seg0 + per);
   const int wlen = ((seg1 - seg0 + kTopkWarps - 1) / kTopkWarps + 127) / 128 * 128;
   const int w0 = min(seg1, seg0 + warp * wlen), w1 = min(seg1, w0 + wlen);
+  // a warp reads its slice in batches of kSelBatch 128-score steps, every load of a batch
+  // issued before the first is used (coalesced: a step is 512 contiguous bytes)
   int wcount = 0;
-  for (int i = w0 + 4 * lane; i < w1; i += 128) {
-    const float4 x = *reinterpret_cast<const float4*>(row + i);  // ld >= n, ld % 4 == 0
-    const float f[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll 1
+  for (int b0 = w0; b0 < w1; b0 += 128 * kSelBatch) {
+    float4 x[kSelBatch];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (i + j < w1) {
-        if (is_nan_bits(__float_as_uint(f[j]))) record_device_error(DSA_ERR_DEVICE_CHECK);
-        wcount += order_key(f[j]) >= tau ? 1 : 0;
+    for (int m = 0; m < kSelBatch; ++m) {
+      const int i = b0 + 128 * m + 4 * lane;
+      x[m] = i < w1 ? *reinterpret_cast<const float4*>(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);  // ld >= n, ld % 4 == 0
+    }
+#pragma unroll
+    for (int m = 0; m < kSelBatch; ++m) {
+      const int i = b0 + 128 * m + 4 * lane;
+      const float f[4] = {x[m].x, x[m].y, x[m].z, x[m].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (i + j < w1) {
+          if (is_nan_bits(__float_as_uint(f[j]))) record_device_error(DSA_ERR_DEVICE_CHECK);
+          wcount += order_key(f[j]) >= tau ? 1 : 0;
+        }
       }
     }
   }
@@ -536,30 +588,34 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
     const uint32_t kdst = dev::map_to_rank(dev::smem_addr(cand_key), 0u);
     const uint32_t idst = dev::map_to_rank(dev::smem_addr(cand_idx), 0u);
     uint32_t at = static_cast<uint32_t>(offset + woff);
-    for (int i = w0 + 4 * lane; i - 4 * lane < w1; i += 128) {  // whole-warp steps
-      uint32_t kk[4];
-      uint32_t keep = 0u;
-      if (i < w1) {
-        const float4 x = *reinterpret_cast<const float4*>(row + i);
-        kk[0] = order_key(x.x);
-        kk[1] = order_key(x.y);
-        kk[2] = order_key(x.z);
-        kk[3] = order_key(x.w);
+#pragma unroll 1
+    for (int b0 = w0; b0 < w1; b0 += 128 * kSelBatch) {  // warp-uniform
+      float4 x[kSelBatch];
+#pragma unroll
+      for (int m = 0; m < kSelBatch; ++m) {
+        const int i = b0 + 128 * m + 4 * lane;
+        x[m] = i < w1 ? *reinterpret_cast<const float4*>(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int m = 0; m < kSelBatch; ++m) {
+        const int i = b0 + 128 * m + 4 * lane;
+        const uint32_t kk[4] = {order_key(x[m].x), order_key(x[m].y), order_key(x[m].z), order_key(x[m].w)};
+        uint32_t keep = 0u;
 #pragma unroll
         for (int j = 0; j < 4; ++j) keep |= static_cast<uint32_t>(i + j < w1 && kk[j] >= tau) << j;
-      }
-      const int cnt = __popc(keep);
-      const int incl = warp_inclusive_scan(cnt);
-      uint32_t p = at + static_cast<uint32_t>(incl - cnt);
+        const int cnt = __popc(keep);
+        const int incl = warp_inclusive_scan(cnt);
+        uint32_t p = at + static_cast<uint32_t>(incl - cnt);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if ((keep >> j) & 1u) {
-          topk_detail::st_cluster_u32(kdst + 4u * p, kk[j]);
-          topk_detail::st_cluster_u32(idst + 4u * p, static_cast<uint32_t>(i + j));
-          ++p;
+        for (int j = 0; j < 4; ++j) {
+          if ((keep >> j) & 1u) {
+            topk_detail::st_cluster_u32(kdst + 4u * p, kk[j]);
+            topk_detail::st_cluster_u32(idst + 4u * p, static_cast<uint32_t>(i + j));
+            ++p;
+          }
         }
+        at += static_cast<uint32_t>(__shfl_sync(0xffffffffu, incl, 31));
       }
-      at += static_cast<uint32_t>(__shfl_sync(0xffffffffu, incl, 31));
     }
   }
   dev::cluster_sync();  // CTA 0 holds the row's candidates; the others are done
