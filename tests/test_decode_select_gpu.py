@@ -1,6 +1,6 @@
 """The fused decode selection (dsa_indexer_topk_decode): paged indexer, then the per-sequence
-top-k that reads each score row once and keeps only the scores at or above the k-th largest
-16-key group maximum.
+top-k that reads only the 16-key groups whose maximum reaches the k-th largest group maximum
+and keeps their scores at or above it.
 
 The selection must equal the oracle's top-k (ties to the lower position, ascending) of the
 GPU's own scores bit for bit: dsa_indexer_scores runs the same kernel and fp32 arithmetic, and
@@ -10,8 +10,8 @@ cover every path of the selection kernel:
   - fewer 16-key groups than k (the group maxima bound nothing; every score is a candidate);
   - the group-maximum bound with its candidates held on chip, at 128K keys;
   - a tie class straddling the k-th position whose members fit on chip;
-  - a tie class of tens of thousands (the on-chip buffers overflow: the full radix select
-    over the row in global memory runs instead)."""
+  - a tie class of tens of thousands (the on-chip candidate buffer overflows: the full radix
+    select over the row in global memory runs instead)."""
 import numpy as np
 import pytest
 import torch
@@ -20,11 +20,10 @@ import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
-CAP = 8192          # candidates one CTA of the selection holds
-CLUSTER = 4         # CTAs per sequence
+CAP = 8192          # candidates the selection holds on chip per row
 
 
-def _run(d, k, max_ctx=None):
+def _run(d, k, max_ctx=None, scan_reports=True):
     import sparse_attention_09_b200 as dsa
     B = d["B"]
     max_ctx = d["max_ctx"] if max_ctx is None else max_ctx
@@ -36,7 +35,8 @@ def _run(d, k, max_ctx=None):
     ld = (max_ctx + 3) // 4 * 4
     S = torch.full((B, ld), float("nan"), device="cuda")
     dsa.dsa_indexer_scores(d["q8"], d["q_scale"], d["w"], keys, B, 64, 128, 0, B, S)
-    assert dsa.dsa_device_error() == err   # the scan reports what the fused call reported
+    # the scan alone reports what the fused call reported (NaN scores only the selection does)
+    assert dsa.dsa_device_error() == (err if scan_reports else dsa.DSA_OK)
     return idx.cpu().numpy(), S.cpu().numpy(), err
 
 
@@ -96,7 +96,7 @@ def test_scores_behind_the_selection_match_oracle():
 @pytest.mark.parametrize("patterns,ctx", [(32, [131072, 100000, 90000]), (3, [131072, 120000])])
 def test_tie_classes_at_the_boundary(patterns, ctx):
     """32 patterns: the top class (~2.8-4K keys) holds the k-th position and fits on chip;
-    3 patterns: the top class (~40K keys) overflows a CTA's buffer (full radix select)."""
+    3 patterns: the top class (~40K keys) overflows the candidate buffer (full radix select)."""
     k = 2048
     d = _patterned(synth.decode_inputs(B=len(ctx), ctx_lo=1, ctx_hi=131072, H_I=64, d_I=128, H=16,
                                        seed=70 + patterns, device="cuda", ctx=ctx), patterns, seed=patterns)
@@ -109,16 +109,15 @@ def test_tie_classes_at_the_boundary(patterns, ctx):
         kth = np.sort(row)[::-1][k - 1]
         above, tied = int((row > kth).sum()), int((row == kth).sum())
         assert above < k < above + tied, "the k-th position must fall inside a tie class"
-        per = ((n + CLUSTER - 1) // CLUSTER + 15) // 16 * 16   # a CTA's segment of the row
-        seg_top = [int((row[c * per:(c + 1) * per] >= kth).sum()) for c in range(CLUSTER)]
-        if patterns == 3:   # a segment holds more of the class than a CTA's buffer
-            assert max(seg_top) > CAP
+        if patterns == 3:   # the candidates (at least the whole tie class) exceed the buffer
+            assert above + tied > CAP
         else:
             assert above + tied <= CAP
 
 
 def test_all_equal_scores_select_the_first_k_positions():
-    """w = 0: every score is 0.  Contexts below 16k keep every score on chip; 128K overflows."""
+    """w = 0: every score is 0.  Below 16k keys every score is a candidate and fits on chip;
+    at 32K and 128K every group passes the bound and the candidates overflow."""
     k = 2048
     ctx = [5000, 32768, 131072]
     d = synth.decode_inputs(B=3, ctx_lo=1, ctx_hi=131072, H_I=64, d_I=128, H=16, seed=80, device="cuda", ctx=ctx)
@@ -152,3 +151,18 @@ def test_blocks_outside_the_pool_score_minus_inf_and_are_not_selected():
     assert np.isneginf(S[0, 6400:6464]).all() and np.isneginf(S[1, :64]).all()
     _check(idx, S, [60000, 40000], k)
     assert not ((idx[0] >= 6400) & (idx[0] < 6464)).any() and not ((idx[1] >= 0) & (idx[1] < 64)).any()
+
+
+def test_nan_score_is_reported():
+    """A NaN key scale makes a NaN score; its group counts as passing the bound, so the
+    selection reads it and reports DSA_ERR_DEVICE_CHECK."""
+    import sparse_attention_09_b200 as dsa
+    d = synth.decode_inputs(B=2, ctx_lo=1, ctx_hi=60000, H_I=64, d_I=128, H=16, seed=83, device="cuda",
+                            ctx=[60000, 40000])
+    blk = int(d["block_table"][1, 300].item())   # sequence 1, position 300 * 64 + 5
+    d["kscale_cache"] = d["kscale_cache"].clone()
+    d["kscale_cache"][blk, 5] = float("nan")
+    idx, S, err = _run(d, 2048, scan_reports=False)
+    assert err == dsa.DSA_ERR_DEVICE_CHECK
+    assert np.isnan(S[1, 300 * 64 + 5])
+    _check(idx[:1], S[:1], [60000], 2048)   # the other sequence is untouched
