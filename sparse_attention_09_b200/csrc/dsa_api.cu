@@ -517,6 +517,7 @@ dsa_status dsa_indexer_topk_decode(const uint8_t* q_fp8, const float* q_scale, i
   if (keys == nullptr || idx_out == nullptr || k <= 0 || B <= 0) return DSA_ERR_INVALID_ARGUMENT;
   if (keys->kind != DSA_KV_PAGED) return DSA_ERR_UNSUPPORTED;
   if (workspace == nullptr || !aligned(workspace, 256)) return DSA_ERR_INVALID_ARGUMENT;
+  if (static_cast<int64_t>(B) * kTopkCluster > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
   CUtensorMap qm, km;
   IndexerParams p;
   dsa_status st = indexer_common(q_fp8, q_scale, q_scale_heads, w, keys, B, H_I, d_I, &qm, &km, &p);
@@ -538,7 +539,7 @@ dsa_status dsa_indexer_topk_decode(const uint8_t* q_fp8, const float* q_scale, i
   if (cudaFuncSetAttribute(topk_decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmemBytes) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
-  topk_decode_select_kernel<<<static_cast<unsigned>(B), kTopkThreads, kSelSmemBytes, s>>>(
+  topk_decode_select_kernel<<<static_cast<unsigned>(B * kTopkCluster), kTopkThreads, kSelSmemBytes, s>>>(
       p.scores, ld, p.gmax, ld16, keys->context_lens, keys->max_seqlen, k, idx_out);
   return launch_status();
 }

@@ -412,9 +412,8 @@ __global__ void __launch_bounds__(IdxGroups<TOK>::kThreads, 1)
             if (s < len) p.scores[(b - p.row_begin) * p.ld + s] = v;
             if (p.gmax != nullptr) {  // uniform: every lane takes part in the shuffles
               // the largest key of the 16 keys of this half-warp (lanes 16h .. 16h+15 hold keys
-              // 16 * (s / 16) ..); keys past the context take no part; a NaN score counts as the
-              // largest key, so that the selection reads (and reports) its group
-              uint32_t key = s < len ? (is_nan_bits(__float_as_uint(v)) ? 0xFFFFFFFFu : order_key(v)) : 0u;
+              // 16 * (s / 16) ..); keys past the context take no part
+              uint32_t key = s < len ? order_key(v) : 0u;
 #pragma unroll
               for (int o = 8; o > 0; o >>= 1) key = max(key, __shfl_xor_sync(0xffffffffu, key, o));
               if ((lane & 15) == 0 && s < len) p.gmax[(b - p.row_begin) * p.ld16 + (s >> 4)] = key;

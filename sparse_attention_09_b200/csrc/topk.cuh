@@ -6,17 +6,17 @@
 // memory) finds the key of the k-th largest entry and how many entries equal to it are still
 // needed; an emit pass then walks the entries in index order and writes the selected indices
 // with a block-wide scan, so the output is ascending and ties at the boundary go to the lowest
-// indices.  A row is handled by a cluster of kTopkCluster CTAs, each taking a contiguous
-// segment of it.  The core reads its entries through a source: a segment of a score row in
-// global memory (dsa_topk), or the candidates a CTA holds in shared memory (decode selection).
+// indices.  The core reads its entries through a source (a segment of a score row in global
+// memory, or candidates in shared memory) and is generic over the CTAs that share a row.
+// dsa_topk runs it on a cluster of kTopkCluster CTAs per row.
 //
 // Decode selection (topk_decode_select_kernel): the paged indexer also writes, per 16 keys,
 // the largest key of the group.  tau = the k-th largest group maximum is a lower bound of the
 // row's k-th largest score: at least k groups have a maximum >= tau and each holds one score
-// >= tau.  One streaming pass keeps the scores >= tau (in index order, in shared memory); for
-// 128K-key rows these are ~2-3K entries instead of 128K, and the exact radix select and the
-// emission run on them.  A row whose candidates overflow a CTA's buffer falls back to the
-// core over the row in global memory, in the same kernel (same result, slower).
+// >= tau.  The row's scores >= tau (~2-3K of a 128K-key row) are gathered, in index order, into
+// one CTA's shared memory, where the exact k-th largest is found and the selection emitted.
+// A row whose candidates overflow that buffer takes the core over the row in global memory, in
+// the same kernel (same result, slower).
 #pragma once
 
 #include "common.cuh"
@@ -277,14 +277,18 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
 // ---- decode selection ------------------------------------------------------------------------
 constexpr int kSelGroup = 16;       // scores per group maximum (written by the paged indexer)
 constexpr int kSelCap = 8192;       // candidates of a row (key + index: 64 KB of shared memory)
-constexpr int kSelGroupCap = 8192;  // groups whose maximum reaches tau (32 KB of shared memory)
 constexpr int kSelBuckets = 4096;   // linear buckets over the group maxima's key range
 constexpr int kSelCandBuckets = 2048;  // linear buckets over the candidates' key range
-constexpr int kSelRankMax = 2048;   // boundary-bucket members ranked directly (O(m^2))
+constexpr int kSelRankMax = 512;    // boundary-bucket members ranked directly (O(m^2))
 constexpr int kSelDigit = 11;       // radix digit of the fallback select over the candidates
-constexpr int kSelSmemBytes = kSelCap * 8 + kSelGroupCap * 4;
+constexpr int kSelBatch = 8;        // 128-score steps a warp loads before using them
+constexpr int kSelSmemBytes = kSelCap * 8;
 
 namespace topk_detail {
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 
 // Block-wide reductions of one uint32 per thread (every thread receives the result).
 template <class Op>
@@ -345,18 +349,12 @@ __device__ __forceinline__ int find_bin_from_top(const uint32_t* hist, uint32_t 
 // the lower edge of the bucket below the one holding the k-th largest, so float rounding of
 // the map cannot put tau above it.  Every thread of the CTA calls it; `hist` holds
 // kSelBuckets counters.
-// The groups whose maximum reaches tau, in index order, into grp[0..np) (np > cap: overflow,
-// grp incomplete).  tau <= the k-th largest of the G group maxima gm[0..G) (G >= k): the maxima's
-// key range [lo, hi] is mapped linearly onto kSelBuckets buckets (any monotone map keeps the
-// order; a linear one spreads the maxima, which crowd a few exponent bins, over many buckets),
-// and tau is the lower edge of the bucket below the one holding the k-th largest, so float
-// rounding of the map cannot put tau above it.  Every thread of the CTA calls it; `hist` holds
-// kSelBuckets counters.
-__device__ int passing_groups(const uint32_t* __restrict__ gm, int G, int k, uint32_t* hist, Shared& sh,
-                              int32_t* grp, int cap, uint32_t& tau) {
+__device__ uint32_t group_max_bound(const uint32_t* __restrict__ gm, int G, int k, uint32_t* hist, Shared& sh) {
   constexpr int V = 4;  // 16-byte loads per thread per step, all issued before the first use
-  constexpr int STEP = 4 * V * kTopkThreads;
   const int tid = threadIdx.x;
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  // every load of a step is issued before any is used; a row of up to 8192 maxima (128K keys)
+  // is one step, held in registers for both uses below
   uint32_t vv[4 * V];
   auto load_step = [&](int base) {
 #pragma unroll
@@ -376,9 +374,8 @@ __device__ int passing_groups(const uint32_t* __restrict__ gm, int G, int k, uin
       vv[4 * v + 3] = x.w;
     }
   };
-  auto at = [&](int base, int v, int j) { return base + 4 * (v * kTopkThreads + tid) + j; };
-  // a row of up to 8192 maxima (128K keys) is one step, held in registers for all three uses
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  auto valid = [&](int base, int v, int j) { return base + 4 * (v * kTopkThreads + tid) + j < G; };
+  constexpr int STEP = 4 * V * kTopkThreads;
 #pragma unroll 1
   for (int base = 0; base < G; base += STEP) {
     load_step(base);
@@ -386,59 +383,34 @@ __device__ int passing_groups(const uint32_t* __restrict__ gm, int G, int k, uin
     for (int v = 0; v < V; ++v)
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        if (at(base, v, j) < G) {
+        if (valid(base, v, j)) {
           lo = min(lo, vv[4 * v + j]);
           hi = max(hi, vv[4 * v + j]);
         }
   }
   lo = block_reduce_u32(lo, reinterpret_cast<uint32_t*>(sh.scan_scratch), MinOp{});
   hi = block_reduce_u32(hi, reinterpret_cast<uint32_t*>(sh.scan_scratch), MaxOp{});
-  if (hi == lo) {
-    tau = lo;  // every maximum is equal: all G >= k groups reach it
-  } else {
-    const float inv = static_cast<float>(kSelBuckets) / (static_cast<float>(hi - lo) + 1.f);
-    for (int i = tid; i < kSelBuckets; i += kTopkThreads) hist[i] = 0u;
-    __syncthreads();
-#pragma unroll 1
-    for (int base = 0; base < G; base += STEP) {
-      if (G > STEP) load_step(base);
-#pragma unroll
-      for (int v = 0; v < V; ++v)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (at(base, v, j) < G) {
-            const int b = static_cast<int>(static_cast<float>(vv[4 * v + j] - lo) * inv);
-            atomicAdd(&hist[b < kSelBuckets ? b : kSelBuckets - 1], 1u);
-          }
-    }
-    __syncthreads();
-    uint32_t above;
-    const int b = find_bin_from_top<kSelBuckets>(hist, static_cast<uint32_t>(k), above, sh);
-    const float edge = static_cast<float>(b - 1) / inv;  // one bucket of margin for the rounding
-    tau = edge <= 0.f ? lo : lo + static_cast<uint32_t>(edge);
-  }
-  // the passing groups, in index order (value order within a step is (v, thread, j))
-  int np = 0;
+  if (hi == lo) return lo;  // every maximum is equal: all G >= k groups reach it
+  const float inv = static_cast<float>(kSelBuckets) / (static_cast<float>(hi - lo) + 1.f);
+  for (int i = tid; i < kSelBuckets; i += kTopkThreads) hist[i] = 0u;
+  __syncthreads();
 #pragma unroll 1
   for (int base = 0; base < G; base += STEP) {
-    if (G > STEP) load_step(base);
+    if (G > STEP) load_step(base);  // one step: the maxima are still in registers
 #pragma unroll
-    for (int v = 0; v < V; ++v) {
-      uint32_t pass = 0u;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) pass |= static_cast<uint32_t>(at(base, v, j) < G && vv[4 * v + j] >= tau) << j;
-      int tot;
-      int p = np + block_exclusive_scan<kTopkWarps>(__popc(pass), sh.scan_scratch, tot);
+    for (int v = 0; v < V; ++v)
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        if ((pass >> j) & 1u) {
-          if (p < cap) grp[p] = at(base, v, j);
-          ++p;
+        if (valid(base, v, j)) {
+          const int b = static_cast<int>(static_cast<float>(vv[4 * v + j] - lo) * inv);
+          atomicAdd(&hist[b < kSelBuckets ? b : kSelBuckets - 1], 1u);
         }
-      np += tot;
-    }
   }
-  return np;
+  __syncthreads();
+  uint32_t above;
+  const int b = find_bin_from_top<kSelBuckets>(hist, static_cast<uint32_t>(k), above, sh);
+  const float edge = static_cast<float>(b - 1) / inv;  // one bucket of margin for the rounding
+  return edge <= 0.f ? lo : lo + static_cast<uint32_t>(edge);
 }
 
 }  // namespace topk_detail
@@ -597,107 +569,130 @@ __device__ void cand_select_emit(const uint32_t* __restrict__ key, const int32_t
 
 // Per-sequence selection after the paged indexer: scores [B, ld] (entries [0, n_b)), gmax
 // [B, ld16] (order key of the largest score of entries [16 g, 16 g + 16) of the row), n_b =
-// min(context_lens[b], max_len).  One CTA per row:
-//   1. tau from the row's group maxima, and the groups whose maximum reaches it (in index
-//      order): only they can hold a score >= tau (about k of the n/16 groups);
-//   2. the 16 scores of each such group (one thread per group, 64 contiguous bytes; the next
-//      round's loads issued before this round is used), keeping the scores >= tau in index
-//      order in shared memory;
-//   3. the exact select over those candidates and the ascending emission.
-// A row whose passing groups or candidates overflow the buffers takes the full radix select
-// over the row in global memory.
-__global__ void __launch_bounds__(kTopkThreads)
+// min(context_lens[b], max_len).  One cluster of kTopkCluster CTAs per row:
+//   1. every CTA computes tau from the row's group maxima (the same value in each);
+//   2. every CTA splits its quarter of the row into 16 warp slices and counts, with coalesced
+//      16-byte loads, the scores >= tau of each slice;
+//   3. the CTAs exchange their counts; unless the row's candidates exceed kSelCap, every warp
+//      reads its slice again and writes its candidates, in index order, straight into CTA 0's
+//      buffer at its offset (distributed shared memory), and CTA 0 alone selects and emits.
+// With more than kSelCap candidates the cluster runs the full radix select over the row.
+__global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThreads, 2)
     topk_decode_select_kernel(const float* __restrict__ scores, int64_t ld, const uint32_t* __restrict__ gmax,
                               int64_t ld16, const int32_t* __restrict__ context_lens, int32_t max_len, int32_t k,
                               int32_t* __restrict__ idx) {
+  constexpr int C = kTopkCluster;
   extern __shared__ uint8_t sel_smem[];
   uint32_t* cand_key = reinterpret_cast<uint32_t*>(sel_smem);
   int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_key + kSelCap);
-  int32_t* grp = cand_idx + kSelCap;
   __shared__ topk_detail::Shared sh;
-  const int tid = threadIdx.x;
-  const int64_t r = blockIdx.x;
+  __shared__ uint32_t s_count;
+  __shared__ int s_wcount[kTopkWarps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t rank = dev::cluster_ctarank();
+  const int64_t r = blockIdx.x / C;
   int32_t* out = idx + r * static_cast<int64_t>(k);
   // the indexer reports a context longer than max_len; here it is clamped the same way
-  const int n = topk_detail::checked_len(min(context_lens[r], max_len), ld, threadIdx.x == 0);
+  const int n = topk_detail::checked_len(min(context_lens[r], max_len), ld, threadIdx.x == 0 && rank == 0);
   if (n <= k) {
-    for (int i = tid; i < k; i += kTopkThreads) out[i] = i < n ? i : -1;
+    if (rank == 0)
+      for (int i = tid; i < k; i += kTopkThreads) out[i] = i < n ? i : -1;
     return;
   }
   const float* row = scores + r * ld;
   const int G = (n + kSelGroup - 1) / kSelGroup;
-  uint32_t tau = 0u;
-  int np;
-  if (G >= k) {
-    np = topk_detail::passing_groups(gmax + r * ld16, G, k, &sh.hist[0][0], sh, grp, kSelGroupCap, tau);
-  } else {  // fewer groups than k: the maxima bound nothing, every score is a candidate
-    for (int g = tid; g < G; g += kTopkThreads) grp[g] = g;
-    np = G;
-    __syncthreads();
-  }
-  // 2. the passing groups' scores >= tau, in index order
-  int count = 0;
-  if (np <= kSelGroupCap) {
-    float4 cur[4], nxt[4];
-    auto load = [&](int round, float4(&x)[4]) {
-      const int j = round * kTopkThreads + tid;
-      const int g = j < np ? grp[j] : -1;
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const int i = 16 * g + 4 * v;
-        x[v] = g >= 0 && i < n ? *reinterpret_cast<const float4*>(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    };
-    const int rounds = (np + kTopkThreads - 1) / kTopkThreads;
-    if (rounds > 0) load(0, cur);
+  // 1. with fewer groups than k the maxima bound nothing: every score is a candidate
+  const uint32_t tau = G >= k ? topk_detail::group_max_bound(gmax + r * ld16, G, k, &sh.hist[0][0], sh) : 0u;
+
+  // 2. this CTA's segment, in 16 warp slices of whole 128-score steps (a float4 per lane)
+  const int per = ((n + C - 1) / C + 15) / 16 * 16;
+  const int seg0 = min(n, static_cast<int>(rank) * per), seg1 = min(n, seg0 + per);
+  const int wlen = ((seg1 - seg0 + kTopkWarps - 1) / kTopkWarps + 127) / 128 * 128;
+  const int w0 = min(seg1, seg0 + warp * wlen), w1 = min(seg1, w0 + wlen);
+  // a warp reads its slice in batches of kSelBatch 128-score steps, every load of a batch
+  // issued before the first is used (coalesced: a step is 512 contiguous bytes)
+  int wcount = 0;
 #pragma unroll 1
-    for (int rd = 0; rd < rounds; ++rd) {
-      if (rd + 1 < rounds) load(rd + 1, nxt);
-      const int j = rd * kTopkThreads + tid;
-      const int g = j < np ? grp[j] : -1;
-      uint32_t keep = 0u;
+  for (int b0 = w0; b0 < w1; b0 += 128 * kSelBatch) {
+    float4 x[kSelBatch];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const float f[4] = {cur[v].x, cur[v].y, cur[v].z, cur[v].w};
+    for (int m = 0; m < kSelBatch; ++m) {
+      const int i = b0 + 128 * m + 4 * lane;
+      x[m] = i < w1 ? *reinterpret_cast<const float4*>(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);  // ld >= n, ld % 4 == 0
+    }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 16 * g + 4 * v + e;
-          const bool in = g >= 0 && i < n;
-          if (in && is_nan_bits(__float_as_uint(f[e]))) record_device_error(DSA_ERR_DEVICE_CHECK);
-          keep |= static_cast<uint32_t>(in && order_key(f[e]) >= tau) << (4 * v + e);
+    for (int m = 0; m < kSelBatch; ++m) {
+      const int i = b0 + 128 * m + 4 * lane;
+      const float f[4] = {x[m].x, x[m].y, x[m].z, x[m].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (i + j < w1) {
+          if (is_nan_bits(__float_as_uint(f[j]))) record_device_error(DSA_ERR_DEVICE_CHECK);
+          wcount += order_key(f[j]) >= tau ? 1 : 0;
         }
       }
-      int total;
-      int p = count + block_exclusive_scan<kTopkWarps>(__popc(keep), sh.scan_scratch, total);
+    }
+  }
+  wcount = __reduce_add_sync(0xffffffffu, wcount);
+  if (lane == 0) s_wcount[warp] = wcount;
+  __syncthreads();
+  int woff = 0, ccount = 0;
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const float f[4] = {cur[v].x, cur[v].y, cur[v].z, cur[v].w};
+  for (int w = 0; w < kTopkWarps; ++w) {
+    woff += w < warp ? s_wcount[w] : 0;
+    ccount += s_wcount[w];
+  }
+  if (tid == 0) s_count = static_cast<uint32_t>(ccount);
+  dev::cluster_sync();  // 3. the counts are published
+  int total = 0, offset = 0;
+  for (int c = 0; c < C; ++c) {
+    const int cc = static_cast<int>(topk_detail::ld_cluster_u32(dev::map_to_rank(dev::smem_addr(&s_count), c)));
+    if (c < static_cast<int>(rank)) offset += cc;
+    total += cc;
+  }
+  if (total > kSelCap || total < k) {
+    // too many candidates for one buffer (e.g. a tie class of thousands at the boundary):
+    // the exact select over the row in global memory, on the whole cluster
+    topk_detail::radix_select_emit<C>(topk_detail::RowSource{row, seg0, seg1, false}, k, out, sh);
+    return;
+  }
+  {  // this warp's candidates, in index order, into CTA 0's buffer at offset + woff
+    const uint32_t kdst = dev::map_to_rank(dev::smem_addr(cand_key), 0u);
+    const uint32_t idst = dev::map_to_rank(dev::smem_addr(cand_idx), 0u);
+    uint32_t at = static_cast<uint32_t>(offset + woff);
+#pragma unroll 1
+    for (int b0 = w0; b0 < w1; b0 += 128 * kSelBatch) {  // warp-uniform
+      float4 x[kSelBatch];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if ((keep >> (4 * v + e)) & 1u) {
-            if (p < kSelCap) {
-              cand_key[p] = order_key(f[e]);
-              cand_idx[p] = 16 * g + 4 * v + e;
-            }
+      for (int m = 0; m < kSelBatch; ++m) {
+        const int i = b0 + 128 * m + 4 * lane;
+        x[m] = i < w1 ? *reinterpret_cast<const float4*>(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int m = 0; m < kSelBatch; ++m) {
+        const int i = b0 + 128 * m + 4 * lane;
+        const uint32_t kk[4] = {order_key(x[m].x), order_key(x[m].y), order_key(x[m].z), order_key(x[m].w)};
+        uint32_t keep = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) keep |= static_cast<uint32_t>(i + j < w1 && kk[j] >= tau) << j;
+        const int cnt = __popc(keep);
+        const int incl = warp_inclusive_scan(cnt);
+        uint32_t p = at + static_cast<uint32_t>(incl - cnt);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if ((keep >> j) & 1u) {
+            topk_detail::st_cluster_u32(kdst + 4u * p, kk[j]);
+            topk_detail::st_cluster_u32(idst + 4u * p, static_cast<uint32_t>(i + j));
             ++p;
           }
         }
+        at += static_cast<uint32_t>(__shfl_sync(0xffffffffu, incl, 31));
       }
-      count += total;
-#pragma unroll
-      for (int v = 0; v < 4; ++v) cur[v] = nxt[v];
     }
   }
-  if (np > kSelGroupCap || count > kSelCap || count < k) {
-    // too many groups or candidates for the buffers (e.g. a tie class of thousands at the
-    // boundary): the exact select over the row in global memory
-    __syncthreads();
-    topk_detail::radix_select_emit<1>(topk_detail::RowSource{row, 0, n, true}, k, out, sh);
-    return;
-  }
-  __syncthreads();
-  // 3. the exact select over the candidates and the emission
-  topk_detail::cand_select_emit(cand_key, cand_idx, count, k, out, &sh.hist[0][0], sh);
+  dev::cluster_sync();  // CTA 0 holds the row's candidates; the others are done
+  if (rank != 0) return;
+  topk_detail::cand_select_emit(cand_key, cand_idx, total, k, out, &sh.hist[0][0], sh);
 }
 
 }  // namespace dsa
