@@ -64,7 +64,7 @@ constexpr int kIdxStages = 4;      // key-tile ring depth, scores mode
 constexpr int kIdxStagesTopk = 3;  // fused top-k mode (the candidate sets need the SMEM)
 constexpr int kIdxCapMax = 4096;   // candidate capacity per token, fused top-k mode
 constexpr int kIdxTok = 4;            // prefill query tokens per CTA
-constexpr int kDecodeTilesPerCta = 16;  // decode: 2048 keys per CTA
+constexpr int kDecodeTilesPerCta = 32;  // decode: 4096 keys per CTA (measured: 16 -> 32 tiles, -3 % at 64 x ~71K keys, -12 % at 8 x ~127K)
 
 template <int D_I, int H_I, int TOK, int MODE, bool PAGED>
 dsa_status launch_indexer_t(const CUtensorMap& qm, const CUtensorMap& km, const IndexerParams& p, dim3 grid,
