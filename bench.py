@@ -355,7 +355,12 @@ def run_ours(args, world, rank, local):
         cpu = {"value": len(rows) / secs, "unit": "tokens/s", "cores": blas_threads(), "host_cores": os.cpu_count(),
                "kind": "oracle",
                "sample": f"{len(rows)} query rows of the L=131072 prefill (full causal prefix each: indexer, "
-                         f"top-k, attention), {secs:.1f} s"}
+                         f"top-k, attention), {secs:.1f} s",
+               "extrapolation": f"the whole L=131072 prefill at this rate: about {L * secs / len(rows) / 3600:.1f} h "
+                                f"(the rows are drawn uniformly over the sequence, so their mean cost is that of "
+                                f"an average row; estimate, not measured)"}
+        if args.cpu_c2_full:
+            cpu["c2_full"] = oracle_prefill_full(dict(synth.WORKLOADS["prefill_8k"]), sm)
 
     if rank == 0:
         line = {
@@ -708,17 +713,43 @@ def run_decode(args, dsa, sm, peaks):
 
 def oracle_decode_sample(d, k, sm, nseq):
     """The oracle's decode step (paged indexer over the whole context, top-k, sparse MLA) on the
-    first nseq sequences of the decode workload, timed on the host; tokens/s = nseq / time."""
+    first nseq sequences of the decode workload (all 64 by default: the step in full), timed on
+    the host, one sequence at a time (its host copy is made outside the timed region);
+    tokens/s = nseq / time."""
     import oracle
-    seqs = [synth.decode_seq_numpy(d, b) for b in range(nseq)]
-    t0 = time.perf_counter()
-    for s in seqs:
-        oracle.dsa_decode(s, k, sm)
-    secs = time.perf_counter() - t0
-    ctx = [int(d["ctx_host"][b]) for b in range(nseq)]
+    secs = 0.0
+    for b in range(nseq):
+        seq = synth.decode_seq_numpy(d, b)
+        t0 = time.perf_counter()
+        oracle.dsa_decode(seq, k, sm)
+        secs += time.perf_counter() - t0
+        del seq
+    full = nseq == d["B"]
+    ctx = sum(int(d["ctx_host"][b]) for b in range(nseq))
     return {"value": nseq / secs, "unit": "tokens/s", "cores": blas_threads(), "host_cores": os.cpu_count(),
             "kind": "oracle",
-            "sample": f"{nseq} of the 64 decode sequences (contexts {ctx}), one decode token each, {secs:.1f} s"}
+            "sample": (f"the whole decode step: all {nseq} sequences" if full else f"{nseq} of the {d['B']} sequences")
+                      + f" ({ctx} context keys), one decode token each, {secs:.1f} s"}
+
+
+def oracle_prefill_full(cfg, sm, block=512):
+    """The oracle on every query row of a prefill workload (prefill_8k: L=8192), in row blocks of
+    `block` rows to bound host memory; tokens/s = L / time (host copies outside the timed region)."""
+    import oracle
+    inp = synth.prefill_inputs(device="cuda", **cfg)
+    L, k = cfg["seqlens"][0], cfg["k"]
+    secs = 0.0
+    for r0 in range(0, L, block):
+        rows = list(range(r0, min(L, r0 + block)))
+        seq = synth.seq_slice_numpy(inp, 0, rows=rows)
+        t0 = time.perf_counter()
+        oracle.dsa_prefill_rows(seq, k, sm, rows)
+        secs += time.perf_counter() - t0
+        del seq
+    del inp
+    torch.cuda.empty_cache()
+    return {"value": L / secs, "unit": "tokens/s", "cores": blas_threads(), "host_cores": os.cpu_count(),
+            "kind": "oracle", "sample": f"the whole L={L} prefill (prefill_8k), every query row, {secs:.1f} s"}
 
 
 def run_e2e(args, dsa, inp, cfg, sm, n_blocks=32):
@@ -871,7 +902,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-rows", type=int, default=256)
-    ap.add_argument("--cpu-decode-seqs", type=int, default=4)
+    ap.add_argument("--cpu-decode-seqs", type=int, default=64,
+                    help="decode sequences the oracle baseline runs (64 = the whole decode_64 step)")
+    ap.add_argument("--cpu-c2-full", action="store_true",
+                    help="also time the oracle on the whole prefill_8k workload (about two minutes of CPU)")
     ap.add_argument("--ref-rows", type=int, default=2)
     ap.add_argument("--workload", default=PREFILL, choices=[w for w, c in synth.WORKLOADS.items() if c["kind"] == "prefill"],
                     help="prefill workload of the timed step (the headline is prefill_128k; smaller ones are for profiling)")
