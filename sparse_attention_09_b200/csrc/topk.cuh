@@ -290,6 +290,15 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
+// The float whose order key is `key` (the inverse of order_key on its image); for a key whose
+// inverse would be a NaN pattern, the infinity on its side, so that !(f < result) holds for
+// every score f with order_key(f) >= key (a superset of them, never fewer).
+__device__ __forceinline__ float key_floor_float(uint32_t key) {
+  if (key > 0xFF800000u) return INFINITY;   // above order_key(+inf): positive NaN patterns
+  if (key < 0x007FFFFFu) return -INFINITY;  // below order_key(-inf): negative NaN patterns
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
 // Block-wide reductions of one uint32 per thread (every thread receives the result).
 template <class Op>
 __device__ __forceinline__ uint32_t block_reduce_u32(uint32_t v, uint32_t* scratch, Op op) {
@@ -610,7 +619,11 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
   const int wlen = ((seg1 - seg0 + kTopkWarps - 1) / kTopkWarps + 127) / 128 * 128;
   const int w0 = min(seg1, seg0 + warp * wlen), w1 = min(seg1, w0 + wlen);
   // a warp reads its slice in batches of kSelBatch 128-score steps, every load of a batch
-  // issued before the first is used (coalesced: a step is 512 contiguous bytes)
+  // issued before the first is used (coalesced: a step is 512 contiguous bytes).  A score is a
+  // candidate when !(score < tf), tf the float whose order key is tau: one compare per score,
+  // the same set as order_key(score) >= tau for every non-NaN score, and a NaN score is always
+  // a candidate (it is reported when the candidates are written).
+  const float tf = topk_detail::key_floor_float(tau);
   int wcount = 0;
 #pragma unroll 1
   for (int b0 = w0; b0 < w1; b0 += 128 * kSelBatch) {
@@ -622,14 +635,13 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
     }
 #pragma unroll
     for (int m = 0; m < kSelBatch; ++m) {
-      const int i = b0 + 128 * m + 4 * lane;
-      const float f[4] = {x[m].x, x[m].y, x[m].z, x[m].w};
+      const int lim = w1 - (b0 + 128 * m + 4 * lane);  // scores of this float4 inside the slice
+      if (lim >= 4) {
+        wcount += (x[m].x < tf ? 0 : 1) + (x[m].y < tf ? 0 : 1) + (x[m].z < tf ? 0 : 1) + (x[m].w < tf ? 0 : 1);
+      } else if (lim > 0) {
+        const float f[4] = {x[m].x, x[m].y, x[m].z, x[m].w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (i + j < w1) {
-          if (is_nan_bits(__float_as_uint(f[j]))) record_device_error(DSA_ERR_DEVICE_CHECK);
-          wcount += order_key(f[j]) >= tau ? 1 : 0;
-        }
+        for (int j = 0; j < 4; ++j) wcount += (j < lim && !(f[j] < tf)) ? 1 : 0;
       }
     }
   }
@@ -653,7 +665,7 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
   if (total > kSelCap || total < k) {
     // too many candidates for one buffer (e.g. a tie class of thousands at the boundary):
     // the exact select over the row in global memory, on the whole cluster
-    topk_detail::radix_select_emit<C>(topk_detail::RowSource{row, seg0, seg1, false}, k, out, sh);
+    topk_detail::radix_select_emit<C>(topk_detail::RowSource{row, seg0, seg1, true}, k, out, sh);
     return;
   }
   {  // this warp's candidates, in index order, into CTA 0's buffer at offset + woff
@@ -671,17 +683,19 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThre
 #pragma unroll
       for (int m = 0; m < kSelBatch; ++m) {
         const int i = b0 + 128 * m + 4 * lane;
-        const uint32_t kk[4] = {order_key(x[m].x), order_key(x[m].y), order_key(x[m].z), order_key(x[m].w)};
+        const float f[4] = {x[m].x, x[m].y, x[m].z, x[m].w};
+        const int lim = w1 - i;
         uint32_t keep = 0u;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) keep |= static_cast<uint32_t>(i + j < w1 && kk[j] >= tau) << j;
+        for (int j = 0; j < 4; ++j) keep |= static_cast<uint32_t>(j < lim && !(f[j] < tf)) << j;
         const int cnt = __popc(keep);
         const int incl = warp_inclusive_scan(cnt);
         uint32_t p = at + static_cast<uint32_t>(incl - cnt);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           if ((keep >> j) & 1u) {
-            topk_detail::st_cluster_u32(kdst + 4u * p, kk[j]);
+            if (is_nan_bits(__float_as_uint(f[j]))) record_device_error(DSA_ERR_DEVICE_CHECK);
+            topk_detail::st_cluster_u32(kdst + 4u * p, order_key(f[j]));
             topk_detail::st_cluster_u32(idst + 4u * p, static_cast<uint32_t>(i + j));
             ++p;
           }
