@@ -61,15 +61,18 @@ bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint6
 
 // ---- lightning indexer -------------------------------------------------------------------
 constexpr int kIdxStages = 4;      // key-tile ring depth, scores mode
-constexpr int kIdxStagesTopk = 3;  // fused top-k mode (the candidate sets need the SMEM)
-constexpr int kIdxCapMax = 4096;   // candidate capacity per token, fused top-k mode
+// Fused top-k mode: the candidate sets need the shared memory.  Up to 128K keys (d_I = 128) the
+// key ring has 2 stages and a token holds up to 4608 candidates; longer sequences need the
+// third stage for the emission bitmap (which reuses the ring) and hold 4096.  Measured at
+// L = 131072: 130.9 ms against 135.4 ms with 3 stages and 4096 (fewer streaming cuts).
+constexpr int kIdxStagesTopkShort = 2, kIdxCapShort = 4608, kIdxCapExtraShort = 2560;
+constexpr int kIdxStagesTopkLong = 3, kIdxCapLong = 4096, kIdxCapExtraLong = 1024;
 constexpr int kIdxTok = 4;            // prefill query tokens per CTA
 constexpr int kDecodeTilesPerCta = 32;  // decode: 4096 keys per CTA (measured: 16 -> 32 tiles, -3 % at 64 x ~71K keys, -12 % at 8 x ~127K)
 
-template <int D_I, int H_I, int TOK, int MODE, bool PAGED>
-dsa_status launch_indexer_t(const CUtensorMap& qm, const CUtensorMap& km, const IndexerParams& p, dim3 grid,
+template <int D_I, int H_I, int TOK, int MODE, bool PAGED, int STAGES>
+dsa_status launch_indexer_s(const CUtensorMap& qm, const CUtensorMap& km, const IndexerParams& p, dim3 grid,
                             cudaStream_t s) {
-  constexpr int STAGES = MODE == kIdxTopk ? kIdxStagesTopk : kIdxStages;
   auto kern = indexer_kernel<D_I, H_I, TOK, MODE, PAGED, STAGES>;
   const int smem = indexer_smem_bytes<D_I, H_I, TOK, MODE, STAGES>(p.cap) + 1024;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -78,20 +81,57 @@ dsa_status launch_indexer_t(const CUtensorMap& qm, const CUtensorMap& km, const 
   return launch_status();
 }
 
+// Scores mode: kIdxStages; fused top-k mode: the ring depth `stages` (2 or 3, see above).
+template <int D_I, int H_I, int TOK, int MODE, bool PAGED>
+dsa_status launch_indexer_t(const CUtensorMap& qm, const CUtensorMap& km, const IndexerParams& p, dim3 grid,
+                            cudaStream_t s, int stages) {
+  if constexpr (MODE == kIdxTopk) {
+    if (stages == kIdxStagesTopkShort)
+      return launch_indexer_s<D_I, H_I, TOK, MODE, PAGED, kIdxStagesTopkShort>(qm, km, p, grid, s);
+    return launch_indexer_s<D_I, H_I, TOK, MODE, PAGED, kIdxStagesTopkLong>(qm, km, p, grid, s);
+  } else {
+    return launch_indexer_s<D_I, H_I, TOK, MODE, PAGED, kIdxStages>(qm, km, p, grid, s);
+  }
+}
+
+// Ring depth and candidate capacity of the fused top-k for sequences of up to max_seqlen keys
+// (the final ascending emission uses a bitmap of the causal prefix inside the key ring, half of
+// it per epilogue group); DSA_ERR_UNSUPPORTED when the bitmap does not fit three stages.
+dsa_status topk_config(int d_I, int max_seqlen, int k, int* stages, int* cap) {
+  const int64_t bitmap_bytes = (static_cast<int64_t>(max_seqlen) + 31) / 32 * 4;
+  const int64_t stage_bytes = 128 * static_cast<int64_t>(d_I);
+  if (max_seqlen > (1 << 24)) return DSA_ERR_UNSUPPORTED;
+  int extra, cmax;
+  if (bitmap_bytes <= kIdxStagesTopkShort * stage_bytes / 2) {
+    *stages = kIdxStagesTopkShort;
+    extra = kIdxCapExtraShort;
+    cmax = kIdxCapShort;
+  } else if (bitmap_bytes <= kIdxStagesTopkLong * stage_bytes / 2) {
+    *stages = kIdxStagesTopkLong;
+    extra = kIdxCapExtraLong;
+    cmax = kIdxCapLong;
+  } else {
+    return DSA_ERR_UNSUPPORTED;
+  }
+  *cap = k + extra < 2 * k ? 2 * k : k + extra;
+  if (*cap > cmax) *cap = cmax;
+  return DSA_OK;
+}
+
 template <int MODE, bool PAGED>
 dsa_status launch_indexer(int d_I, int H_I, const CUtensorMap& qm, const CUtensorMap& km, const IndexerParams& p,
-                          dim3 grid, cudaStream_t s) {
+                          dim3 grid, cudaStream_t s, int stages = 0) {
   constexpr int TOK = PAGED ? 1 : kIdxTok;
   if constexpr (PAGED) {
     if (H_I != 64) return DSA_ERR_UNSUPPORTED;
-    if (d_I == 128) return launch_indexer_t<128, 64, TOK, MODE, PAGED>(qm, km, p, grid, s);
-    if (d_I == 64) return launch_indexer_t<64, 64, TOK, MODE, PAGED>(qm, km, p, grid, s);
+    if (d_I == 128) return launch_indexer_t<128, 64, TOK, MODE, PAGED>(qm, km, p, grid, s, stages);
+    if (d_I == 64) return launch_indexer_t<64, 64, TOK, MODE, PAGED>(qm, km, p, grid, s, stages);
     return DSA_ERR_UNSUPPORTED;
   } else {
-    if (d_I == 128 && H_I == 64) return launch_indexer_t<128, 64, TOK, MODE, PAGED>(qm, km, p, grid, s);
-  if (d_I == 64 && H_I == 64) return launch_indexer_t<64, 64, TOK, MODE, PAGED>(qm, km, p, grid, s);
-  if (d_I == 128 && H_I == 4) return launch_indexer_t<128, 4, TOK, MODE, PAGED>(qm, km, p, grid, s);
-  if (d_I == 64 && H_I == 4) return launch_indexer_t<64, 4, TOK, MODE, PAGED>(qm, km, p, grid, s);
+    if (d_I == 128 && H_I == 64) return launch_indexer_t<128, 64, TOK, MODE, PAGED>(qm, km, p, grid, s, stages);
+  if (d_I == 64 && H_I == 64) return launch_indexer_t<64, 64, TOK, MODE, PAGED>(qm, km, p, grid, s, stages);
+  if (d_I == 128 && H_I == 4) return launch_indexer_t<128, 4, TOK, MODE, PAGED>(qm, km, p, grid, s, stages);
+  if (d_I == 64 && H_I == 4) return launch_indexer_t<64, 4, TOK, MODE, PAGED>(qm, km, p, grid, s, stages);
   return DSA_ERR_UNSUPPORTED;
   }
 }
@@ -463,17 +503,13 @@ dsa_status dsa_indexer_topk(const uint8_t* q_fp8, const float* q_scale, int32_t 
   IndexerParams p;
   dsa_status st = indexer_common(q_fp8, q_scale, q_scale_heads, w, keys, B, H_I, d_I, &qm, &km, &p);
   if (st != DSA_OK) return st;
-  // the final ascending emission uses a bitmap of the causal prefix inside the key ring
-  const int64_t bitmap_bytes = (static_cast<int64_t>(keys->max_seqlen) + 31) / 32 * 4;
-  // (each of the two epilogue groups of a CTA has half of the key ring for its bitmap)
-  if (bitmap_bytes > static_cast<int64_t>(kIdxStagesTopk) * 128 * d_I / 2 || keys->max_seqlen > (1 << 24))
-    return DSA_ERR_UNSUPPORTED;
+  int stages;
+  st = topk_config(d_I, keys->max_seqlen, k, &stages, &p.cap);
+  if (st != DSA_OK) return st;
   p.idx_out = idx_out;
   p.k = k;
-  p.cap = k + 1024 < 2 * k ? 2 * k : k + 1024;
-  if (p.cap > kIdxCapMax) p.cap = kIdxCapMax;
   dim3 grid((keys->max_seqlen + kIdxTok - 1) / kIdxTok, B);
-  return launch_indexer<kIdxTopk, false>(d_I, H_I, qm, km, p, grid, as_stream(stream));
+  return launch_indexer<kIdxTopk, false>(d_I, H_I, qm, km, p, grid, as_stream(stream), stages);
 }
 
 dsa_status dsa_indexer_topk_rows(const uint8_t* q_fp8, const float* q_scale, int32_t q_scale_heads, const float* w,
@@ -490,18 +526,16 @@ dsa_status dsa_indexer_topk_rows(const uint8_t* q_fp8, const float* q_scale, int
   dsa_status st = indexer_common(q_fp8, q_scale, q_scale_heads, w, keys, 1, H_I, d_I, &qm, &km, &p,
                                  row_end - row_begin);
   if (st != DSA_OK) return st;
-  const int64_t bitmap_bytes = (static_cast<int64_t>(keys->max_seqlen) + 31) / 32 * 4;
-  if (bitmap_bytes > static_cast<int64_t>(kIdxStagesTopk) * 128 * d_I / 2 || keys->max_seqlen > (1 << 24))
-    return DSA_ERR_UNSUPPORTED;
+  int stages;
+  st = topk_config(d_I, keys->max_seqlen, k, &stages, &p.cap);
+  if (st != DSA_OK) return st;
   p.idx_out = idx_out;
   p.k = k;
-  p.cap = k + 1024 < 2 * k ? 2 * k : k + 1024;
-  if (p.cap > kIdxCapMax) p.cap = kIdxCapMax;
   p.tok_begin = static_cast<int32_t>(row_begin);
   p.tok_end = static_cast<int32_t>(row_end);
   p.q_row0 = row_begin;
   dim3 grid(static_cast<unsigned>((row_end - row_begin + kIdxTok - 1) / kIdxTok), 1);
-  return launch_indexer<kIdxTopk, false>(d_I, H_I, qm, km, p, grid, as_stream(stream));
+  return launch_indexer<kIdxTopk, false>(d_I, H_I, qm, km, p, grid, as_stream(stream), stages);
 }
 
 size_t dsa_decode_select_workspace_size(int32_t B, int32_t max_ctx) {

@@ -68,7 +68,7 @@ struct Cands {
   uint32_t* key;  // [4 * Q]
   int32_t* idx;   // [4 * Q]
   int* cnt;       // [4] fill count of each region (valid at cut points)
-  int Q;          // region capacity (<= 1024)
+  int Q;          // region capacity (<= 1152)
 };
 
 __device__ __forceinline__ int total_count(const Cands& C) { return C.cnt[0] + C.cnt[1] + C.cnt[2] + C.cnt[3]; }
@@ -130,12 +130,12 @@ __device__ __forceinline__ void group_minmax(const Group& G, Scratch& S, uint32_
 // would serialise the rounds).
 template <class Keep>
 __device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S, Keep keep) {
-  constexpr int kMaxRounds = 32;  // Q <= 1024 = 32 lanes x 32 rounds
+  constexpr int kMaxRounds = 36;  // Q <= 1152 = 32 lanes x 36 rounds
   const int w = G.warp(), lane = G.lane();
   const int c = C.cnt[w];
   uint32_t key[kMaxRounds];
   int32_t id[kMaxRounds];
-  uint32_t keepbits = 0u;  // bit r: this lane keeps its entry of round r
+  uint64_t keepbits = 0u;  // bit r: this lane keeps its entry of round r
 #pragma unroll
   for (int r = 0; r < kMaxRounds; ++r) {
     const int i = r * 32 + lane;
@@ -144,10 +144,10 @@ __device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S
     if (i < c) {
       key[r] = C.key[w * C.Q + i];
       id[r] = C.idx[w * C.Q + i];
-      if (keep(key[r], id[r])) keepbits |= 1u << r;
+      if (keep(key[r], id[r])) keepbits |= 1ull << r;
     }
   }
-  const int wcount = __reduce_add_sync(0xffffffffu, __popc(keepbits));
+  const int wcount = __reduce_add_sync(0xffffffffu, __popcll(keepbits));
   int total;
   int base = gscan(G, lane == 0 ? wcount : 0, S.scan, total);  // its barriers order reads before writes
   base = __shfl_sync(0xffffffffu, base, 0);
@@ -156,7 +156,7 @@ __device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S
 #pragma unroll
   for (int r = 0; r < kMaxRounds; ++r) {
     if (r * 32 >= c) break;
-    const bool k = (keepbits >> r) & 1u;
+    const bool k = (keepbits >> r) & 1ull;
     const uint32_t m = __ballot_sync(0xffffffffu, k);
     if (k) {
       const uint32_t p = static_cast<uint32_t>(base) + static_cast<uint32_t>(__popc(m & below));

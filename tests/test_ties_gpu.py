@@ -1,8 +1,9 @@
 """The fused indexer top-k under heavy ties, on rows far longer than its candidate capacity.
 
 The method keeps the top-k = 2048 scores per query with ties going to the lower index.  The
-fused kernel streams each row through a bounded candidate set (capacity max(2k, k + 1024), at
-most 4096) and cuts it to a superset of the current top k whenever it fills; when the boundary
+fused kernel streams each row through a bounded candidate set (for sequences of up to 128K keys:
+capacity max(2k, k + 2560), at most 4608) and cuts it to a superset of the current top k whenever
+it fills; when the boundary
 bucket holds many equal keys the cut splits them by index.  These inputs make that happen on
 most rows: every key is one of three e4m3 patterns, so a row's scores take three values and the
 k-th position falls inside a tied class of thousands; a quarter of the rows have w = 0, so all
@@ -37,7 +38,8 @@ def _three_level_inputs(seqlens, seed):
 
 
 def _capacity(k):
-    return min(max(2 * k, k + 1024), 4096)
+    """Candidates per token of the fused top-k for sequences of at most 128K keys (d_I = 128)."""
+    return min(max(2 * k, k + 2560), 4608)
 
 
 def _straddles(row, m):
@@ -122,3 +124,18 @@ def test_fused_topk_three_level_ties_2x32k_sampled(k):
             if t + 1 > _capacity(k) and _straddles(row.astype(np.float64), m):
                 straddle += 1
     assert straddle > 20, f"only {straddle} sampled rows split a tied class past the candidate capacity"
+
+
+@pytest.mark.parametrize("d_I,L", [(64, 66000), (64, 65536)])
+def test_fused_topk_both_ring_configurations(d_I, L):
+    """Up to 2^16 keys at d_I = 64 (2^17 at d_I = 128) the fused top-k runs a 2-stage key ring
+    with 4608 candidates per token; one key more and it takes the 3-stage ring with 4096 (the
+    emission bitmap needs the third stage).  Both give the oracle's top-k of the GPU scores."""
+    k = 512
+    inp = synth.exact_prefill_inputs([L], 4, d_I, 16, seed=L % 97, device="cuda", small_scores=True)
+    idx = indexer_topk(inp, k).cpu().numpy()
+    rows = [0, k - 1, k, 3000, 40000, L - 2, L - 1]
+    for t in rows:
+        S = indexer_scores(inp, row_begin=t, row_end=t + 1)[0].cpu().numpy()
+        exp = oracle.topk_rows(S[None, : t + 1], np.array([t + 1]), k)[0]
+        assert np.array_equal(idx[t], exp), f"row {t}"
