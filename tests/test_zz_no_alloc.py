@@ -8,6 +8,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 from helpers import assert_attention_close
 
@@ -64,8 +65,8 @@ def test_noalloc_decode_rejects_sizes_beyond_its_scratch():
 
 def test_noalloc_decode_size_edge_at_128_heads():
     """At H = 128 the partials of B = 127 sequences (one split each) fit the scratch array and
-    B = 128 do not: the last size that fits runs and equals the workspace call, the first that
-    does not is refused before any launch."""
+    B = 128 do not: the last size that fits runs, equals the workspace call and agrees with the
+    oracle on sampled sequences; the first that does not is refused before any launch."""
     import sparse_attention_09_b200 as dsa
     B, k = 127, 2048
     d = synth.decode_inputs(B=B, ctx_lo=1, ctx_hi=2500, H_I=64, d_I=128, H=128, seed=31, device="cuda")
@@ -88,6 +89,12 @@ def test_noalloc_decode_size_edge_at_128_heads():
     assert st == dsa.DSA_OK, dsa.dsa_status_string(st)
     assert dsa.dsa_device_error() == 0
     assert torch.equal(out, ref)  # the same kernels on the same inputs
+    for b in (0, 63, B - 1):        # and the oracle on the selected latent rows
+        seq = synth.decode_seq_numpy(d, b)
+        lat = oracle.paged_gather(seq["latent_cache"], seq["block_table"], seq["ctx"])
+        sel = idx[b].cpu().numpy()
+        want, _ = oracle.sparse_mla_token(seq["q"], lat, sel[sel >= 0], sm)
+        assert_attention_close(out[b].float().cpu().numpy(), want, f"seq {b}")
     poison = out.clone()
     st = dsa._lib.dsa_sparse_mla_decode_noalloc(ctypes.c_void_p(d["q"].data_ptr()), latent.ref(),
                                                 ctypes.c_void_p(idx.data_ptr()), B + 1, 128, k, ctypes.c_float(sm),
