@@ -47,6 +47,11 @@ def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
+# fp32 lane operations per second (one op per lane and cycle): 148 SMs x 128 lanes x 1.965 GHz;
+# an FMA counts 2 flops, so the fp32 FMA peak is twice this in FLOP/s
+FP32_LANE_OPS_T = 148 * 128 * 1.965e9 / 1e12
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -327,6 +332,12 @@ def run_ours(args, world, rank, local):
     }
     for kk in kernels.values():
         kk["frac"] = kk["tflops"] / kk["peak_tflops"]
+    # the indexer epilogue's own floor: ReLU and the weighted head sum, 2*H_I ops per causal pair,
+    # against one fp32 op per lane and cycle (148 SMs x 128 lanes x 1.965 GHz = 37.2 T ops/s)
+    alu_ops = idx_flops / cfg["d_I"]
+    kernels["indexer_topk"]["epilogue_alu"] = {
+        "ops": alu_ops, "tops": alu_ops / (idx_ms * 1e-3) / 1e12, "peak_tops": FP32_LANE_OPS_T,
+        "frac": alu_ops / (idx_ms * 1e-3) / 1e12 / FP32_LANE_OPS_T}
     dom = max(kernels, key=lambda n: kernels[n]["ms"])
     dk = kernels[dom]
     traffic = profile_traffic(dom)
@@ -359,6 +370,7 @@ def run_ours(args, world, rank, local):
                "extrapolation": f"the whole L=131072 prefill at this rate: about {L * secs / len(rows) / 3600:.1f} h "
                                 f"(the rows are drawn uniformly over the sequence, so their mean cost is that of "
                                 f"an average row; estimate, not measured)"}
+        cpu["c1_full"] = oracle_prefill_full(dict(synth.WORKLOADS["tiny_256"]), sm)   # a few seconds
         if args.cpu_c2_full:
             cpu["c2_full"] = oracle_prefill_full(dict(synth.WORKLOADS["prefill_8k"]), sm)
 
@@ -622,7 +634,7 @@ def run_kl(dsa, inp, idx, cfg, sm):
     bwd_flops = pairs * H_I * d_I * 2 * 3
     res["indexer_backward_tflops_fp32"] = bwd_flops / (res["indexer_backward_ms"] * 1e-3) / 1e12
     # CUDA-core fp32 peak from the unit counts: 148 SMs x 128 FP32 lanes x 2 flops x 1.965 GHz
-    res["indexer_backward_frac_of_fp32_alu"] = res["indexer_backward_tflops_fp32"] / 74.4
+    res["indexer_backward_frac_of_fp32_alu"] = res["indexer_backward_tflops_fp32"] / (2 * FP32_LANE_OPS_T)
     assert dsa.dsa_device_error() == 0
     del pd, dw, dq, dkey, grad, lse
     torch.cuda.empty_cache()
@@ -733,7 +745,7 @@ def oracle_decode_sample(d, k, sm, nseq):
 
 
 def oracle_prefill_full(cfg, sm, block=512):
-    """The oracle on every query row of a prefill workload (prefill_8k: L=8192), in row blocks of
+    """The oracle on every query row of a prefill workload (tiny_256, prefill_8k), in row blocks of
     `block` rows to bound host memory; tokens/s = L / time (host copies outside the timed region)."""
     import oracle
     inp = synth.prefill_inputs(device="cuda", **cfg)
@@ -749,7 +761,7 @@ def oracle_prefill_full(cfg, sm, block=512):
     del inp
     torch.cuda.empty_cache()
     return {"value": L / secs, "unit": "tokens/s", "cores": blas_threads(), "host_cores": os.cpu_count(),
-            "kind": "oracle", "sample": f"the whole L={L} prefill (prefill_8k), every query row, {secs:.1f} s"}
+            "kind": "oracle", "sample": f"the whole L={L} prefill, every query row, {secs:.1f} s"}
 
 
 def run_e2e(args, dsa, inp, cfg, sm, n_blocks=32):
