@@ -39,7 +39,7 @@ DECODE = "decode_64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {
     "indexer_topk": ["indexer.cuh", "select.cuh", "sm100.cuh", "common.cuh"],
-    "sparse_mla": ["sparse_mla_pair.cuh", "sparse_mla.cuh", "sm100.cuh", "common.cuh"],
+    "sparse_mla": ["sparse_mla_pair.cuh", "mla_common.cuh", "sm100.cuh", "common.cuh"],
 }
 
 

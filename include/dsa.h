@@ -198,12 +198,11 @@ dsa_status dsa_sparse_mla_prefill_rows(const void* q, const dsa_kv_desc* latent,
  * Masked dense mode of sparse MLA prefill, for short sequences ("DeepSeek-V3.2 论文解读",
  * section 二, subsection "等性能验证": for short prefill a masked MHA mode simulates DSA): the same out/lse as
  * dsa_sparse_mla_prefill for the same arguments, computed by walking every causal 64-key chunk
- * of the contiguous latent with TMA tiles and masking the keys idx does not select.  Cost grows
- * with L^2 instead of L*k, so it pays only when most causal keys are selected (L up to ~2k).
- * idx rows must be ascending with the -1 padding at the end (as the top-k entry points write
- * them); entries outside [0, t] are ignored.  Same layouts, alignment and errors as
- * dsa_sparse_mla_prefill; additionally DSA_ERR_INVALID_ARGUMENT if the latent cannot be
- * described to the TMA unit.
+ * of the contiguous latent (rows read in order, none through idx) and masking the keys idx does
+ * not select.  Cost grows with L^2 instead of L*k, so it pays only when most causal keys are
+ * selected (L up to ~2k).  idx rows must be strictly ascending with the -1 padding at the end
+ * (as the top-k entry points write them); entries outside [0, t] are ignored (not reported).
+ * Same layouts, alignment and errors as dsa_sparse_mla_prefill.
  */
 dsa_status dsa_masked_mla_prefill(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B,
                                   int32_t H, int32_t k, float sm_scale, void* out, float* lse, void* stream);

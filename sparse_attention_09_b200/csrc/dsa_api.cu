@@ -17,7 +17,7 @@
 #include "indexer_bwd.cuh"
 #include "indexer_kl.cuh"
 #include "selftest.cuh"
-#include "sparse_mla.cuh"
+#include "mla_common.cuh"
 #include "sparse_mla_pair.cuh"
 #include "topk.cuh"
 
@@ -217,31 +217,16 @@ int decode_splits(int B, int k) {
   return s;
 }
 
-template <bool DECODE, bool DENSE = false>
-dsa_status launch_mla(const void* latent, const MlaParams& p, int64_t units, cudaStream_t s,
-                      const CUtensorMap* nope_map = nullptr, const CUtensorMap* rope_map = nullptr) {
-  auto kern = sparse_mla_kernel<DECODE, DENSE>;
-  const int smem = mla::kSmemBytes + 1024;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return DSA_ERR_CUDA;
-  CUtensorMap unused;
-  std::memset(&unused, 0, sizeof(unused));
-  const int clusters = static_cast<int>(units < kMlaClusters ? units : kMlaClusters);
-  kern<<<2 * clusters, mla::kThreads, smem, s>>>(static_cast<const __nv_bfloat16*>(latent), p,
-                                                  nope_map ? *nope_map : unused, rope_map ? *rope_map : unused);
-  return launch_status();
-}
-
-// Sparse prefill and decode: the head-split pair kernel.  Q is read by TMA as a [q_rows * H, 576]
-// bf16 matrix in 64 x 64 tiles (128-byte swizzle).
-template <bool DECODE>
+// Sparse prefill, masked prefill and decode: the head-split pair kernel.  Q is read by TMA as a
+// [q_rows * H, 576] bf16 matrix in 64 x 64 tiles (128-byte swizzle).
+template <bool DECODE, bool MASKED = false>
 dsa_status launch_mla_pair(const void* latent, const void* q, int64_t q_rows, const MlaParams& p, int64_t units,
                            cudaStream_t s) {
   CUtensorMap qm;
   if (!make_map_2d(&qm, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kLatentDim, static_cast<uint64_t>(q_rows) * p.H,
                    kLatentDim * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_INVALID_ARGUMENT;
-  auto kern = sparse_mla_pair_kernel<DECODE>;
+  auto kern = sparse_mla_pair_kernel<DECODE, MASKED>;
   const int smem = mlap::kSmemBytes + 1024;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return DSA_ERR_CUDA;
@@ -644,15 +629,6 @@ dsa_status dsa_masked_mla_prefill(const void* q, const dsa_kv_desc* latent, cons
     return DSA_ERR_INVALID_ARGUMENT;
   if (!mla_shape_ok(H, k)) return DSA_ERR_UNSUPPORTED;
   if (latent->total_tokens > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
-  // the contiguous latent [T, 576] bf16 as two tiled views: 64-dim nope blocks (128-byte
-  // swizzle) and the 32-dim rope halves (64-byte swizzle), 64 rows per tile
-  CUtensorMap nope_map, rope_map;
-  const uint64_t T = static_cast<uint64_t>(latent->total_tokens);
-  if (!make_map_2d(&nope_map, latent->data, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kLatentDim, T, kLatentDim * 2, 64, 64,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&rope_map, latent->data, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kLatentDim, T, kLatentDim * 2, 32, 64,
-                   CU_TENSOR_MAP_SWIZZLE_64B))
-    return DSA_ERR_INVALID_ARGUMENT;
   MlaParams p;
   std::memset(&p, 0, sizeof(p));
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -666,7 +642,7 @@ dsa_status dsa_masked_mla_prefill(const void* q, const dsa_kv_desc* latent, cons
   p.scale_log2 = sm_scale * 1.4426950408889634f;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  return launch_mla<false, true>(latent->data, p, p.rows, as_stream(stream), &nope_map, &rope_map);
+  return launch_mla_pair<false, true>(latent->data, q, p.rows, p, p.rows, as_stream(stream));
 }
 
 dsa_status dsa_sparse_mla_decode(const void* q, const dsa_kv_desc* latent, const int32_t* idx, int32_t B, int32_t H,

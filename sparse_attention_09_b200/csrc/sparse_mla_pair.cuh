@@ -52,11 +52,20 @@
 // paged latent cache.  A split selection's unnormalised partial results (O, M, l) go to a
 // workspace that a small kernel merges by log-sum-exp; an unsplit one is written as out / lse
 // directly, as in prefill.
+//
+// And the masked dense mode for short prefill (MASKED): the attention a dense MHA kernel gives
+// under a mask that simulates the sparse pattern ("DeepSeek-V3.2 论文解读", section 二,
+// subsection "等性能验证").  Chunk c of token t is then the 64 contiguous latent rows
+// [64c, 64c + 64) of its sequence, for every c up to t / 64, and the keys that the (ascending)
+// selection row does not hold, or that lie past t, are masked in the softmax.  The gather warps
+// read no selection entries; each softmax warp walks the selection row with a cursor (the
+// entries of chunk c are one run of at most 64 starting where chunk c - 1's run ended) and
+// loads the next run while it works on the current chunk.
 #pragma once
 
 #include "common.cuh"
+#include "mla_common.cuh"
 #include "sm100.cuh"
-#include "sparse_mla.cuh"
 
 namespace dsa {
 namespace mlap {
@@ -107,8 +116,8 @@ struct Unit {
   int seq, seq_start, seq_len, sp, c0, c1;
 };
 
-// Warp-collective (scans the selection row).
-template <bool DECODE>
+// Warp-collective (scans the selection row).  Masked mode: every causal chunk of the token.
+template <bool DECODE, bool MASKED>
 __device__ __forceinline__ Unit unit_of(const MlaParams& p, int64_t u) {
   Unit r;
   int kbeg, kend;
@@ -136,6 +145,11 @@ __device__ __forceinline__ Unit unit_of(const MlaParams& p, int64_t u) {
     r.seq = lo;
     r.seq_start = p.cu_seqlens[lo];
     r.seq_len = p.cu_seqlens[lo + 1] - r.seq_start;
+  }
+  if constexpr (MASKED) {
+    r.c0 = 0;
+    r.c1 = static_cast<int>(u + p.unit0 - r.seq_start) / kChunk + 1;
+    return r;
   }
   const int act = mla::active_chunks(p.idx + r.qrow * p.k, p.k);
   r.c0 = kbeg / kChunk;
@@ -166,7 +180,7 @@ __device__ __forceinline__ bool key_of(const MlaParams& p, const int32_t* bt, in
 
 }  // namespace mlap
 
-template <bool DECODE>
+template <bool DECODE, bool MASKED = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mlap::kThreads, 1)
     sparse_mla_pair_kernel(const __nv_bfloat16* __restrict__ latent, const MlaParams p,
                            const __grid_constant__ CUtensorMap q_map) {
@@ -243,7 +257,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mlap::kThreads, 1)
     uint32_t g = 0;
     bool ok = true;
     for (int64_t u = cid; ok && u < nunits; u += ncl) {
-      const Unit un = unit_of<DECODE>(p, u);
+      const Unit un = unit_of<DECODE, MASKED>(p, u);
       const int32_t* row = p.idx + un.qrow * p.k;
       const int32_t* bt = DECODE ? p.block_table + static_cast<int64_t>(un.seq) * p.max_blocks_per_seq : nullptr;
       // masked entries still copy a real row (never NaN bits): the sequence's first key; in
@@ -263,8 +277,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mlap::kThreads, 1)
           }
           int prow = pad_row;
           bool bad;
-          key_of<DECODE>(p, bt, row[c * kChunk + 32 * static_cast<int>(rank) + 16 * pw + (lane & 15)], un, prow, bad);
-          if (bad && lane < 16) record_device_error(DSA_ERR_DEVICE_CHECK);  // the entry is masked
+          const int e = c * kChunk + 32 * static_cast<int>(rank) + 16 * pw + (lane & 15);
+          key_of<DECODE>(p, bt, MASKED ? e : row[e], un, prow, bad);
+          if (!MASKED && bad && lane < 16) record_device_error(DSA_ERR_DEVICE_CHECK);  // the entry is masked
           const uint32_t kq = smem_addr(sKQ + s * kKQBytes);
 #pragma unroll 4
           for (int j = 0; j < 16; ++j) {
@@ -294,7 +309,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mlap::kThreads, 1)
           }
           int prow = pad_row;
           bool bad;
-          key_of<DECODE>(p, bt, row[c * kChunk + 32 * pw + lane], un, prow, bad);
+          const int e = c * kChunk + 32 * pw + lane;
+          key_of<DECODE>(p, bt, MASKED ? e : row[e], un, prow, bad);
           const uint32_t vb = smem_addr(sV + s * kVBytes);
           const int seg = lane >> 4, pc = lane & 15;  // segment m: dims 256m + 128 rank + 8 pc
           const int blk = 2 * seg + (pc >> 3), ch = pc & 7;
@@ -345,7 +361,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mlap::kThreads, 1)
     auto enter_unit = [&](Cursor& cu) {
       cu.valid = cu.u < nunits;
       if (!cu.valid) return;
-      const Unit un = unit_of<DECODE>(p, cu.u);
+      const Unit un = unit_of<DECODE, MASKED>(p, cu.u);
       cu.c0 = un.c0;
       cu.c1 = un.c1;
       cu.c = cu.c0;
@@ -535,16 +551,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mlap::kThreads, 1)
     uint32_t g = 0;
     bool aborted = false;
     for (int64_t u = cid; !aborted && u < nunits; u += ncl) {
-      const Unit un = unit_of<DECODE>(p, u);
+      const Unit un = unit_of<DECODE, MASKED>(p, u);
       const int32_t* row = p.idx + un.qrow * p.k;
       const int32_t* bt = DECODE ? p.block_table + static_cast<int64_t>(un.seq) * p.max_blocks_per_seq : nullptr;
       float m = -INFINITY, l = 0.f;
+      // masked mode: the token's position, the selection cursor and the 64 entries from it
+      const int t = MASKED ? static_cast<int>(u + p.unit0 - un.seq_start) : 0;
+      int cur = 0, va = -1, vb = -1;
+      if constexpr (MASKED) {
+        va = row[lane];
+        vb = row[32 + lane];
+      }
       for (int c = un.c0; c < un.c1; ++c, ++g) {
         const int s = static_cast<int>(g & 1u);
-        int prow_unused = 0;
-        bool bad_unused;
-        const bool valid = key_of<DECODE>(p, bt, row[c * kChunk + 32 * kh + lane], un, prow_unused, bad_unused);
-        const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+        uint32_t vmask;
+        if constexpr (MASKED) {
+          // chunk c's entries are the run [cur, cur + n) of entries below 64c + 64 (at most 64
+          // when the row is ascending and distinct); this warp keeps those of its key half that
+          // lie in the causal prefix, then loads the 64 entries after the run
+          const int lo = c * kChunk, half = lo + 32 * kh;
+          const bool ina = va >= 0 && va < lo + kChunk, inb = vb >= 0 && vb < lo + kChunk;
+          const int n = __popc(__ballot_sync(0xffffffffu, ina)) + __popc(__ballot_sync(0xffffffffu, inb));
+          uint32_t bits = 0u;
+          if (ina && va >= half && va < half + 32 && va <= t) bits |= 1u << (va - half);
+          if (inb && vb >= half && vb < half + 32 && vb <= t) bits |= 1u << (vb - half);
+          vmask = __reduce_or_sync(0xffffffffu, bits);
+          cur += n;
+          va = cur + lane < p.k ? row[cur + lane] : -1;
+          vb = cur + 32 + lane < p.k ? row[cur + 32 + lane] : -1;
+        } else {
+          int prow_unused = 0;
+          bool bad_unused;
+          const bool valid = key_of<DECODE>(p, bt, row[c * kChunk + 32 * kh + lane], un, prow_unused, bad_unused);
+          vmask = __ballot_sync(0xffffffffu, valid);
+        }
         if (!pair_wait(&bar_s_full[s], (g >> 1) & 1u)) {
           aborted = true;
           break;
