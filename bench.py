@@ -193,6 +193,16 @@ def blas_threads():
 # ------------------------------------------------------------------------------------------
 # our arm
 # ------------------------------------------------------------------------------------------
+def prefill_config(workload, world, cfg):
+    """The JSON `config` of a prefill line (the same for both arms)."""
+    return {"workload": (f"{PREFILL}: DSA prefill, batch 1 per GPU, L=131072, top-k 2048, 64 e4m3 "
+                         "indexer heads d_I=128, 128-head MLA-MQA (576 qk / 512 v), bf16, 5% planted keys")
+            if workload == PREFILL else f"{workload} (profiling case, not the headline)",
+            "global_batch": world * len(cfg["seqlens"]), "seq_len": cfg["seqlens"][0], "k": cfg["k"],
+            "parallelism": f"independent problems x{world}",
+            "l2": "inputs (~40 GB/step) larger than L2; no flush"}
+
+
 def prefill_work(cfg):
     L = cfg["seqlens"][0]
     pairs = sum(s * (s + 1) // 2 for s in cfg["seqlens"])
@@ -379,12 +389,7 @@ def run_ours(args, world, rank, local):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
-            "config": {"workload": (f"{PREFILL}: DSA prefill, batch 1 per GPU, L=131072, top-k 2048, 64 e4m3 "
-                                    "indexer heads d_I=128, 128-head MLA-MQA (576 qk / 512 v), bf16, 5% planted keys")
-                       if args.workload == PREFILL else f"{args.workload} (profiling case, not the headline)",
-                       "global_batch": world * len(cfg["seqlens"]), "seq_len": L, "k": k,
-                       "parallelism": f"independent problems x{world}",
-                       "l2": "inputs (~40 GB/step) larger than L2; no flush"},
+            "config": prefill_config(args.workload, world, cfg),
             "roofline": roofline, "kernels": kernels, "decode": decode, "next_rows": next_rows,
             "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk, "gpu_launches": 2 * args.steps,
@@ -896,10 +901,10 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{PREFILL}: DSA prefill, L=131072, top-k 2048 (oracle on {per_step} sampled "
-                                   "query rows per step)", "seq_len": L, "k": k},
+            "config": prefill_config(PREFILL, world, cfg),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "host_cores": os.cpu_count(), "kind": "oracle",
-                             "sample": f"{per_step} random query rows per step of the L=131072 prefill"},
+                             "sample": f"{per_step} random query rows per step of the L=131072 prefill (each row's "
+                                       "whole causal prefix: indexer, top-k, attention); tokens/s = rows / time"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
