@@ -256,17 +256,20 @@ __device__ __noinline__ uint32_t cut_exact(const Group& G, Cands& C, Scratch& S,
   });
 }
 
-// Bucket of a key under a monotone map of [lo, hi] onto kBuckets buckets.  Any monotone map
-// is enough: a key in a higher bucket is never smaller than one in a lower bucket.
-__device__ __forceinline__ int bucket_of(uint32_t key, uint32_t lo, float inv) {
-  const int b = static_cast<int>(static_cast<float>(key - lo) * inv);
-  return b < 0 ? 0 : (b > kBuckets - 1 ? kBuckets - 1 : b);
+// Buckets of a key range [lo, hi]: key -> (key - lo) >> shift, with the smallest shift that
+// leaves at most kBuckets buckets (kBuckets is a power of two).  Bucket b holds exactly the keys
+// [lo + (b << shift), lo + ((b + 1) << shift) - 1], so a bucket's bounds are exact and the keys
+// of a bucket and everything above it are those >= its smallest key.
+__device__ __forceinline__ int bucket_shift(uint32_t lo, uint32_t hi) {
+  const uint32_t span = hi - lo;
+  const int bits = 32 - __clz(span);  // bits of the largest offset
+  constexpr int kBucketBits = 10;
+  static_assert((1 << kBucketBits) == kBuckets, "kBuckets is 2^kBucketBits");
+  return bits > kBucketBits ? bits - kBucketBits : 0;
 }
 
 struct Boundary {
-  uint32_t lo, hi;  // the candidates in the boundary bucket have keys in [lo, hi]
-  float inv;
-  int bucket;
+  uint32_t lo, hi;  // the boundary bucket's keys: exactly [lo, hi]
   int above;        // candidates ranked above the boundary bucket
   int inb;          // candidates in the boundary bucket
 };
@@ -277,7 +280,7 @@ struct Boundary {
 __device__ __forceinline__ Boundary boundary_round(const Group& G, const Cands& C, Scratch& S, uint32_t lo,
                                                    uint32_t hi, int want) {
   const int tid = G.tid;
-  const float inv = static_cast<float>(kBuckets) / (static_cast<float>(hi - lo) + 1.f);
+  const int shift = bucket_shift(lo, hi);
 #pragma unroll
   for (int i = 0; i < kBuckets / 128; ++i) S.hist[tid * (kBuckets / 128) + i] = 0u;
   if (tid == 0) S.above = 0u;
@@ -286,7 +289,7 @@ __device__ __forceinline__ Boundary boundary_round(const Group& G, const Cands& 
   for_region(G, C, [&](uint32_t key, int32_t, bool v) {
     const bool in = v && key >= lo && key <= hi;
     above += (v && key > hi) ? 1u : 0u;
-    hist_add(S.hist, in ? static_cast<uint32_t>(bucket_of(key, lo, inv)) : 0u, in);
+    hist_add(S.hist, in ? (key - lo) >> shift : 0u, in);
   });
   above = __reduce_add_sync(0xffffffffu, above);
   if (G.lane() == 0) atomicAdd(&S.above, above);
@@ -317,16 +320,11 @@ __device__ __forceinline__ Boundary boundary_round(const Group& G, const Cands& 
   }
   gsync(G);
   Boundary b;
-  b.bucket = static_cast<int>(S.bin);
   b.above = static_cast<int>(S.rem);
   b.inb = static_cast<int>(S.eqcount);
-  b.inv = inv;
-  // key range of the bucket, widened by one bucket on each side (float rounding), clamped
-  const float lo_f = static_cast<float>(b.bucket - 1) / inv, hi_f = static_cast<float>(b.bucket + 2) / inv;
-  const float span = static_cast<float>(hi - lo);
-  b.lo = lo + static_cast<uint32_t>(lo_f <= 0.f ? 0.f : (lo_f >= span ? span : lo_f));
-  b.hi = lo + static_cast<uint32_t>(hi_f >= span ? span : (hi_f <= 0.f ? 0.f : hi_f));
-  if (b.hi < b.lo) b.hi = b.lo;
+  b.lo = lo + (S.bin << shift);
+  const uint64_t top = static_cast<uint64_t>(b.lo) + ((1ull << shift) - 1u);
+  b.hi = top < hi ? static_cast<uint32_t>(top) : hi;
   gsync(G);
   return b;
 }
@@ -345,13 +343,9 @@ __device__ __noinline__ uint32_t cut_stream(const Group& G, Cands& C, Scratch& S
   for (int round = 0; round < 3; ++round) {
     const Boundary bd = boundary_round(G, C, S, rlo, rhi, k);
     const int kept = bd.above + bd.inb;
-    if (kept <= limit && kept < n) {
-      const uint32_t blo = rlo, bhi = rhi;
-      const float inv = bd.inv;
-      const int bk = bd.bucket;
-      return compact(G, C, S, [=](uint32_t key, int32_t) {
-        return key > bhi || (key >= blo && bucket_of(key, blo, inv) >= bk);
-      });
+    if (kept <= limit && kept < n) {  // keep the boundary bucket and everything above it
+      const uint32_t kf = bd.lo;
+      return compact(G, C, S, [=](uint32_t key, int32_t) { return key >= kf; });
     }
     if (bd.lo >= bd.hi || (bd.lo == rlo && bd.hi == rhi)) break;
     rlo = bd.lo;
@@ -370,20 +364,13 @@ __device__ __noinline__ void cut_final(const Group& G, Cands& C, Scratch& S, int
 #pragma unroll 1
   for (int round = 0; round < 3; ++round) {
     bd = boundary_round(G, C, S, rlo, rhi, m);
-    bd.lo = rlo;  // the boundary bucket is defined relative to this round's interval
-    bd.hi = rhi;
     if (bd.inb <= 128) {
       found = true;
       break;
     }
-    const Boundary nb = bd;
-    const float lo_f = static_cast<float>(nb.bucket - 1) / nb.inv, hi_f = static_cast<float>(nb.bucket + 2) / nb.inv;
-    const float span = static_cast<float>(rhi - rlo);
-    const uint32_t nlo = rlo + static_cast<uint32_t>(lo_f <= 0.f ? 0.f : (lo_f >= span ? span : lo_f));
-    const uint32_t nhi = rlo + static_cast<uint32_t>(hi_f >= span ? span : (hi_f <= 0.f ? 0.f : hi_f));
-    if (nlo >= nhi || (nlo == rlo && nhi == rhi)) break;
-    rlo = nlo;
-    rhi = nhi;
+    if (bd.lo >= bd.hi || (bd.lo == rlo && bd.hi == rhi)) break;
+    rlo = bd.lo;
+    rhi = bd.hi;
   }
   if (!found) {  // many equal keys: resolve by index with the radix path
     cut_exact(G, C, S, m);
@@ -391,12 +378,9 @@ __device__ __noinline__ void cut_final(const Group& G, Cands& C, Scratch& S, int
   }
   const int need = m - bd.above;  // 1 <= need <= inb
   const uint32_t blo = bd.lo, bhi = bd.hi;
-  const float inv = bd.inv;
-  const int bk = bd.bucket;
-  auto in_bucket = [=](uint32_t key) { return key >= blo && key <= bhi && bucket_of(key, blo, inv) == bk; };
-  auto above_bucket = [=](uint32_t key) { return key > bhi || (key >= blo && bucket_of(key, blo, inv) > bk); };
-  if (need == bd.inb) {
-    compact(G, C, S, [=](uint32_t key, int32_t) { return above_bucket(key) || in_bucket(key); });
+  auto in_bucket = [=](uint32_t key) { return key >= blo && key <= bhi; };
+  if (need == bd.inb) {  // the whole boundary bucket and everything above it
+    compact(G, C, S, [=](uint32_t key, int32_t) { return key >= blo; });
     return;
   }
   // gather the boundary bucket and find its need-th best by ranking
@@ -422,10 +406,11 @@ __device__ __noinline__ void cut_final(const Group& G, Cands& C, Scratch& S, int
     }
   }
   gsync(G);
+  // the m-th best is (kstar, istar): every key above the boundary bucket is > kstar (buckets are
+  // monotone) and every key below it < kstar, so the m best are those ranked at or before it
   const uint32_t kstar = S.bin, istar = S.eqcount;
   compact(G, C, S, [=](uint32_t key, int32_t id) {
-    return above_bucket(key) ||
-           (in_bucket(key) && (key > kstar || (key == kstar && static_cast<uint32_t>(id) <= istar)));
+    return key > kstar || (key == kstar && static_cast<uint32_t>(id) <= istar);
   });
 }
 
