@@ -125,9 +125,10 @@ __device__ __forceinline__ void group_minmax(const Group& G, Scratch& S, uint32_
 
 // Keeps the entries with keep(key, idx), spreads them round-robin over the 4 regions and
 // returns the smallest kept key.  Every entry of the warp's region is read into registers
-// before the barrier that precedes the first write, so no entry is overwritten unread.  Output
-// positions come from per-warp ballots and one group scan (no shared-memory atomics, which
-// would serialise the rounds).
+// before the barrier that precedes the first write, so no entry is overwritten unread.  The
+// order of entries inside a set carries no meaning (emission goes through a bitmap, cuts rank
+// by key and index), so each lane's kept entries take consecutive output positions: one warp
+// scan and one group scan place them (no shared-memory atomics, no per-round ballots).
 template <class Keep>
 __device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S, Keep keep) {
   constexpr int kMaxRounds = 36;  // Q <= 1152 = 32 lanes x 36 rounds
@@ -147,25 +148,24 @@ __device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S
       if (keep(key[r], id[r])) keepbits |= 1ull << r;
     }
   }
-  const int wcount = __reduce_add_sync(0xffffffffu, __popcll(keepbits));
+  const int mine = __popcll(keepbits);
+  const int incl = warp_inclusive_scan(mine);
+  const int wcount = __shfl_sync(0xffffffffu, incl, 31);
   int total;
   int base = gscan(G, lane == 0 ? wcount : 0, S.scan, total);  // its barriers order reads before writes
   base = __shfl_sync(0xffffffffu, base, 0);
+  uint32_t p = static_cast<uint32_t>(base + incl - mine);
   uint32_t mn = 0xFFFFFFFFu;
-  const uint32_t below = (1u << lane) - 1u;
 #pragma unroll
   for (int r = 0; r < kMaxRounds; ++r) {
-    if (r * 32 >= c) break;
-    const bool k = (keepbits >> r) & 1ull;
-    const uint32_t m = __ballot_sync(0xffffffffu, k);
-    if (k) {
-      const uint32_t p = static_cast<uint32_t>(base) + static_cast<uint32_t>(__popc(m & below));
+    if ((keepbits >> r) == 0ull) break;
+    if ((keepbits >> r) & 1ull) {
       const int slot = static_cast<int>(p & 3u) * C.Q + static_cast<int>(p >> 2);
       C.key[slot] = key[r];
       C.idx[slot] = id[r];
       mn = min(mn, key[r]);
+      ++p;
     }
-    base += __popc(m);
   }
   mn = __reduce_min_sync(0xffffffffu, mn);
   if (lane == 0) S.tmp_key[w] = mn;  // tmp_key is free here (cut_final is done with it)
