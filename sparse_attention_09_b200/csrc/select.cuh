@@ -133,7 +133,13 @@ template <class Keep>
 __device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S, Keep keep) {
   constexpr int kMaxRounds = 36;  // Q <= 1152 = 32 lanes x 36 rounds
   const int w = G.warp(), lane = G.lane();
-  const int c = C.cnt[w];
+  // the set's fields in registers: stores through its pointers cannot then force reloads of
+  // the descriptor (which the compiler must otherwise assume they may overwrite)
+  uint32_t* const ckey = C.key;
+  int32_t* const cidx = C.idx;
+  int* const ccnt = C.cnt;
+  const int Q = C.Q;
+  const int c = ccnt[w];
   uint32_t key[kMaxRounds];
   int32_t id[kMaxRounds];
   uint64_t keepbits = 0u;  // bit r: this lane keeps its entry of round r
@@ -143,8 +149,8 @@ __device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S
     key[r] = 0u;
     id[r] = 0;
     if (i < c) {
-      key[r] = C.key[w * C.Q + i];
-      id[r] = C.idx[w * C.Q + i];
+      key[r] = ckey[w * Q + i];
+      id[r] = cidx[w * Q + i];
       if (keep(key[r], id[r])) keepbits |= 1ull << r;
     }
   }
@@ -160,9 +166,9 @@ __device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S
   for (int r = 0; r < kMaxRounds; ++r) {
     if ((keepbits >> r) == 0ull) break;
     if ((keepbits >> r) & 1ull) {
-      const int slot = static_cast<int>(p & 3u) * C.Q + static_cast<int>(p >> 2);
-      C.key[slot] = key[r];
-      C.idx[slot] = id[r];
+      const int slot = static_cast<int>(p & 3u) * Q + static_cast<int>(p >> 2);
+      ckey[slot] = key[r];
+      cidx[slot] = id[r];
       mn = min(mn, key[r]);
       ++p;
     }
@@ -171,7 +177,7 @@ __device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S
   if (lane == 0) S.tmp_key[w] = mn;  // tmp_key is free here (cut_final is done with it)
   gsync(G);
   const uint32_t kmin = min(min(S.tmp_key[0], S.tmp_key[1]), min(S.tmp_key[2], S.tmp_key[3]));
-  if (G.tid < 4) C.cnt[G.tid] = total / 4 + (G.tid < total % 4 ? 1 : 0);
+  if (G.tid < 4) ccnt[G.tid] = total / 4 + (G.tid < total % 4 ? 1 : 0);
   gsync(G);  // every thread has read tmp_key and C.cnt is published before anyone moves on
   return kmin;
 }
