@@ -130,7 +130,7 @@ __device__ __forceinline__ void group_minmax(const Group& G, Scratch& S, uint32_
 // by key and index), so each lane's kept entries take consecutive output positions: one warp
 // scan and one group scan place them (no shared-memory atomics, no per-round ballots).
 template <class Keep>
-__device__ __forceinline__ uint32_t compact(const Group& G, Cands& C, Scratch& S, Keep keep) {
+__device__ __forceinline__ uint32_t compact(const Group& G, const Cands& C, Scratch& S, Keep keep) {
   constexpr int kMaxRounds = 36;  // Q <= 1152 = 32 lanes x 36 rounds
   const int w = G.warp(), lane = G.lane();
   // the set's fields in registers: stores through its pointers cannot then force reloads of
@@ -213,7 +213,7 @@ __device__ __forceinline__ void find_bin256(const Group& G, Scratch& S, uint32_t
 
 // Exact cut to the m best by radix select (key, then index among equal keys).  Used when
 // many candidates share one key.  Requires 1 <= m < total_count.  Returns the smallest kept key.
-__device__ __noinline__ uint32_t cut_exact(const Group& G, Cands& C, Scratch& S, int m) {
+__device__ __noinline__ uint32_t cut_exact(const Group G, const Cands C, Scratch& S, int m) {
   const int tid = G.tid;
   uint32_t prefix = 0, mask = 0, remaining = static_cast<uint32_t>(m);
 #pragma unroll 1
@@ -341,7 +341,7 @@ __device__ __forceinline__ Boundary boundary_round(const Group& G, const Cands& 
 // bounds the keys of the set.  Returns the new acceptance threshold (the smallest kept key):
 // later keys enter only if key > thr, which is exact because later candidates have larger
 // indices than every kept one and at least k kept candidates are >= the smallest kept key.
-__device__ __noinline__ uint32_t cut_stream(const Group& G, Cands& C, Scratch& S, int k, int limit, uint32_t lo,
+__device__ __noinline__ uint32_t cut_stream(const Group G, const Cands C, Scratch& S, int k, int limit, uint32_t lo,
                                             uint32_t hi) {
   const int n = total_count(C);
   uint32_t rlo = lo, rhi = hi;
@@ -361,7 +361,7 @@ __device__ __noinline__ uint32_t cut_stream(const Group& G, Cands& C, Scratch& S
 }
 
 // Final exact cut to the m best (key descending, index ascending).
-__device__ __noinline__ void cut_final(const Group& G, Cands& C, Scratch& S, int m, uint32_t lo, uint32_t hi) {
+__device__ __noinline__ void cut_final(const Group G, const Cands C, Scratch& S, int m, uint32_t lo, uint32_t hi) {
   const int n = total_count(C);
   if (n <= m) return;
   uint32_t rlo = lo, rhi = hi;
@@ -422,7 +422,7 @@ __device__ __noinline__ void cut_final(const Group& G, Cands& C, Scratch& S, int
 
 // Writes the (already cut) set to out[0..k) in ascending index order, -1 padded.  `bitmap`
 // has room for `positions` bits.
-__device__ __noinline__ void emit_sorted(const Group& G, const Cands& C, Scratch& S, uint32_t* bitmap, int positions,
+__device__ __noinline__ void emit_sorted(const Group G, const Cands C, Scratch& S, uint32_t* bitmap, int positions,
                                          int32_t* out, int k) {
   const int tid = G.tid, warp = G.warp(), lane = G.lane();
   const int nwords = (positions + 31) / 32;
